@@ -1,0 +1,188 @@
+/*
+ * tri_attn.h -- C ABI of the B200 (sm_100a) triangle-attention library
+ * (libtriattn.so).  Plain pointers and sizes only; no framework types.
+ *
+ * What it computes.  Triangle attention around the starting node of an
+ * AlphaFold3 / OpenFold3 Pairformer pair tensor: for batch b, pair row i,
+ * head h and query j,
+ *
+ *   out[b,i,j,h,:] = sum_k softmax_k( scale * q[b,i,j,h,:].k[b,i,k,h,:]
+ *                                     + bias[b,h,j,k] + mask[b,i,k] ) v[b,i,k,h,:]
+ *
+ * with ONE pair bias shared by all N rows i, so the work is cubic in the crop
+ * size N and the bias gradient is a reduction over rows.  Pages this follows:
+ *   (A) "16张H100，训练步提速1.73倍：TurboPairFormer为什么不是'装个包就能加速AlphaFold3'"
+ *       (biocloudservice.com), sections "先看清'1.73倍'对应什么" (cubic cost) and
+ *       "它优化了什么，而不是只'少存一点张量'" (the four gradients and the shared
+ *       pair bias; the BF16 output-rounding residual with an FP32 correction);
+ *   (B) "TurboPairFormer: более быстрое, стабильное и точное дообучение OpenFold3"
+ *       (dev48.org), section "Как работает TurboPairFormer" (probabilities
+ *       recomputed in the backward, residual compensation, fixed accumulation
+ *       order giving bitwise-identical gradients).
+ *
+ * Ending-node orientation is the same operation on the transposed pair
+ * tensor: pass every 5-D tensor (inputs AND outputs) with stride[1] and
+ * stride[2] swapped.  bias and mask are always given in the attention's own
+ * frame ((j,k) and (i,k)); the caller builds them from the transposed pair
+ * representation, as AlphaFold does.
+ *
+ * Conventions (every entry point):
+ *  - Ownership: the caller allocates and frees every buffer (inputs, outputs,
+ *    saved forward state, workspace).  The library never allocates device or
+ *    host memory for data, never frees, and never synchronises the stream.
+ *  - Asynchrony: work is enqueued on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream).  Argument errors are detected on the host and
+ *    returned before anything is enqueued; nothing is launched on error.
+ *  - Device: the current CUDA device must be compute capability 10.0
+ *    (B200, sm_100a); otherwise TRI_ATTN_ERR_ARCH.
+ *  - Types: q, k, v, bias, dout, o, resid and all gradients are BF16; mask
+ *    and lse are FP32.
+ *  - Strides are in ELEMENTS.  The innermost (channel / key) stride must be 1;
+ *    every other stride must be a non-negative multiple of 8 elements (16
+ *    bytes) except the mask's, which may be anything (0 broadcasts).  Data
+ *    pointers must be 16-byte aligned (mask: 4-byte).
+ *  - Supported sizes: 1 <= B, 1 <= N <= 4096, 1 <= H, d in {32, 64}.
+ *  - Rows whose every key is masked (all mask values <= -1e8) are outside
+ *    the contract: their outputs are unspecified.
+ *  - Determinism: for fixed inputs and shapes every output is bitwise
+ *    identical from run to run (no floating-point atomics; every reduction
+ *    has a fixed order independent of scheduling and SM count).
+ *  - Thread safety: all entry points are reentrant.
+ */
+#ifndef TRI_ATTN_H
+#define TRI_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TRI_ATTN_ABI_VERSION 1
+
+/* A cudaStream_t without pulling in the CUDA headers. */
+typedef struct CUstream_st *tri_attn_stream_t;
+
+typedef enum {
+    TRI_ATTN_OK = 0,
+    TRI_ATTN_ERR_NULL = 1,           /* a required pointer is NULL                     */
+    TRI_ATTN_ERR_SHAPE = 2,          /* B, N or H out of range                         */
+    TRI_ATTN_ERR_STRIDE = 3,         /* innermost stride != 1, or a stride not a
+                                        non-negative multiple of 8 elements          */
+    TRI_ATTN_ERR_ALIGN = 4,          /* a data pointer is not 16-byte aligned          */
+    TRI_ATTN_ERR_DTYPE = 5,          /* reserved for bindings: wrong element type      */
+    TRI_ATTN_ERR_UNSUPPORTED = 6,    /* d not in {32, 64}, or N > 4096                 */
+    TRI_ATTN_ERR_WORKSPACE = 7,      /* workspace NULL or smaller than required        */
+    TRI_ATTN_ERR_ARCH = 8,           /* current device is not sm_100                   */
+    TRI_ATTN_ERR_CUDA = 9,           /* a CUDA runtime/driver call failed              */
+    TRI_ATTN_ERR_DEVICE_TIMEOUT = 10 /* a kernel's bounded wait expired (see
+                                        tri_attn_device_error)                        */
+} tri_attn_status;
+
+/* BF16 pair tensor [B,N,N,H,d]; stride[] = element strides of (b,i,j,h,c), c-stride 1. */
+typedef struct {
+    void *ptr;
+    int64_t stride[5];
+} tri_attn_tensor5;
+
+/* BF16 bias / bias gradient [B,H,N,N]; stride[] = element strides of (b,h,j,k), k-stride 1. */
+typedef struct {
+    void *ptr;
+    int64_t stride[4];
+} tri_attn_tensor4;
+
+/* FP32 additive mask [B,N,N] indexed (b,i,k); ptr may be NULL (no mask); any strides. */
+typedef struct {
+    const float *ptr;
+    int64_t stride[3];
+} tri_attn_mask;
+
+/*
+ * Forward arguments.
+ *   q, k, v, bias, mask : inputs (read only)
+ *   o     : output, BF16 round-to-nearest-even of the FP32 result O32
+ *   resid : output, BF16 RNE of (O32 - float(o)), the output-rounding residual
+ *           (page A, section "它优化了什么": saved so that the backward's softmax
+ *           correction can be formed in FP32 from o + resid)
+ *   lse   : output, FP32 log-sum-exp of each softmax row (natural log), a
+ *           contiguous [B,H,N,N] array indexed (b,h,i,j)
+ *   scale : multiplies q.k only; 0 means 1/sqrt(d)
+ */
+typedef struct {
+    int B, N, H, d;
+    float scale;
+    tri_attn_tensor5 q, k, v;
+    tri_attn_tensor4 bias;
+    tri_attn_mask mask;
+    tri_attn_tensor5 o, resid;
+    float *lse;
+} tri_attn_fwd_args;
+
+/* Backward flag: form the softmax correction D from o alone, ignoring resid
+ * (the uncompensated variant, for measuring what the residual buys). */
+#define TRI_ATTN_BWD_NO_RESIDUAL 1u
+
+/*
+ * Backward arguments.
+ *   f     : the forward's inputs plus its saved state (o, resid, lse), all read only
+ *   dout  : upstream gradient of o (read only)
+ *   dq, dk, dv : outputs, BF16, same layout rules as q
+ *   dbias : output, BF16 [B,H,N,N], the sum over rows i of the score gradient
+ *   workspace, workspace_bytes : caller-owned device scratch of at least
+ *           tri_attn_bwd_workspace_bytes(B,N,H,d) bytes, 256-byte aligned;
+ *           contents on entry are ignored and on exit are unspecified
+ *   flags : 0, or TRI_ATTN_BWD_NO_RESIDUAL
+ * No gradient is produced for mask.
+ */
+typedef struct {
+    tri_attn_fwd_args f;
+    tri_attn_tensor5 dout;
+    tri_attn_tensor5 dq, dk, dv;
+    tri_attn_tensor4 dbias;
+    void *workspace;
+    size_t workspace_bytes;
+    unsigned flags;
+} tri_attn_bwd_args;
+
+/* Enqueue the forward on `stream`.  Returns TRI_ATTN_OK or the first argument
+ * error found (nothing enqueued), or TRI_ATTN_ERR_CUDA if a launch failed. */
+tri_attn_status tri_attn_fwd(const tri_attn_fwd_args *args, tri_attn_stream_t stream);
+
+/* Bytes of device workspace tri_attn_bwd needs for these sizes (a pure
+ * function of the sizes; 0 for invalid sizes).  No device access. */
+size_t tri_attn_bwd_workspace_bytes(int B, int N, int H, int d);
+
+/* Enqueue the backward (dq, dk, dv, dbias) on `stream`.  Same error rules as
+ * tri_attn_fwd, plus TRI_ATTN_ERR_WORKSPACE. */
+tri_attn_status tri_attn_bwd(const tri_attn_bwd_args *args, tri_attn_stream_t stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char *tri_attn_strerror(tri_attn_status status);
+
+/* Reads (and, if clear != 0, resets) the library's device error word on the
+ * current device.  Every spin-wait inside the kernels is bounded; a wait that
+ * expires records its site there and the kernel returns early instead of
+ * hanging.  Synchronises the device.  Returns TRI_ATTN_OK,
+ * TRI_ATTN_ERR_DEVICE_TIMEOUT (and stores the raw word in *word if non-NULL),
+ * or TRI_ATTN_ERR_CUDA. */
+tri_attn_status tri_attn_device_error(int clear, uint32_t *word);
+
+/* Sets the bound of every kernel spin-wait, in nanoseconds of GPU global
+ * timer (default 2e9 = 2 s).  Affects launches enqueued afterwards. */
+void tri_attn_set_wait_limit_ns(uint64_t ns);
+
+/* Test hook for the timeout path: enqueues a one-CTA kernel whose bounded
+ * wait is on a barrier that nothing ever completes, so the wait must expire
+ * (after the current limit) and record TRI_ATTN_ERR_DEVICE_TIMEOUT in the
+ * device error word.  Faults nothing; the context stays usable. */
+tri_attn_status tri_attn_selftest_expire_wait(tri_attn_stream_t stream);
+
+/* TRI_ATTN_ABI_VERSION of the loaded library. */
+int tri_attn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TRI_ATTN_H */

@@ -1,0 +1,204 @@
+"""GPU parity: the CUDA path (through the C ABI) against the FP64 oracle on the
+same seeded BF16 inputs.
+
+Gates (relative RMSE = ||x - x_ref|| / ||x_ref|| over the compared elements,
+FP64): output and dV <= 1e-2; dQ, dK and dBias <= 2e-2.  Small cases compare
+every element; crop-sized cases compare sampled pair rows (every element of
+those rows) and sampled dBias rows (each a sum over all N pair rows), at the
+same launch configuration the benchmark times.
+Repeatability: fixed inputs run 5 times give bitwise-identical outputs and
+gradients ("TurboPairFormer: более быстрое, стабильное и точное дообучение
+OpenFold3", section "Воспроизводимость и стабильность").
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from triangle_attention_biomolecular_b200 import _binding as Bd
+from triangle_attention_biomolecular_b200 import api
+from triangle_attention_biomolecular_b200 import synthetic as S
+
+pytestmark = pytest.mark.gpu
+
+GATES = {"out": 1e-2, "dv": 1e-2, "dq": 2e-2, "dk": 2e-2, "dbias": 2e-2}
+
+
+def rel(a, b):
+    a = np.asarray(a, dtype=np.float64).ravel()
+    b = np.asarray(b, dtype=np.float64).ravel()
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def run_gpu(x, orientation, flags=0):
+    dev = torch.device("cuda")
+    q, k, v, do = (S.to_attention_frame(x[n].to(dev), orientation) for n in ("q", "k", "v", "dout"))
+    bias = x["bias"].to(dev)
+    mask = x["mask"].to(dev) if x["mask"] is not None else None
+    o, r, lse = api.forward(q, k, v, bias, mask)
+    dq, dk, dv, db = api.backward(q, k, v, bias, mask, o, r, lse, do, flags=flags)
+    torch.cuda.synchronize()
+    st, word = Bd.tri_attn_device_error(True)
+    assert st == Bd.TRI_ATTN_OK, f"device error word {word:#x}"
+    cpu = lambda t: t.float().cpu()
+    return {"out": cpu(o), "resid": cpu(r), "lse": lse.cpu(), "dq": cpu(dq), "dk": cpu(dk), "dv": cpu(dv),
+            "dbias": cpu(db)}
+
+
+def oracle_inputs(x, orientation):
+    f = lambda n: S.to_attention_frame(x[n], orientation)
+    return f("q"), f("k"), f("v"), x["bias"], x["mask"], f("dout")
+
+
+def check_full(x, got, orientation="start"):
+    q, k, v, bias, mask, do = oracle_inputs(x, orientation)
+    out, lse = O.fwd(q, k, v, bias, mask)
+    dq, dk, dv, db = O.bwd(q, k, v, bias, mask, do)
+    ref = {"out": out, "dq": dq, "dk": dk, "dv": dv, "dbias": db}
+    errs = {n: rel(got[n].numpy(), ref[n]) for n in ref}
+    for n, e in errs.items():
+        assert np.all(np.isfinite(got[n].numpy())), n
+        assert e <= GATES[n], f"{n}: rel-RMSE {e:.3e} > {GATES[n]}"
+    assert np.max(np.abs(got["lse"].numpy() - lse)) < 2e-3
+    return errs, ref
+
+
+def check_sampled(x, got, rows, sel, orientation="start"):
+    q, k, v, bias, mask, do = oracle_inputs(x, orientation)
+    out, lse = O.fwd(q, k, v, bias, mask, rows=rows)
+    dq, dk, dv = O.bwd_rows(q, k, v, bias, mask, do, rows=rows)
+    db = O.dbias(q, k, v, bias, mask, do, sel=sel)
+    errs = {}
+    for n, ref in (("out", out), ("dq", dq), ("dk", dk), ("dv", dv)):
+        g = np.stack([got[n].numpy()[b, i] for b, i in rows])
+        r = np.stack([ref[b, i] for b, i in rows])
+        assert np.all(np.isfinite(g)), n
+        errs[n] = rel(g, r)
+    g = np.stack([got["dbias"].numpy()[b, h, j] for b, h, j in sel])
+    r = np.stack([db[b, h, j] for b, h, j in sel])
+    errs["dbias"] = rel(g, r)
+    for n, e in errs.items():
+        assert e <= GATES[n], f"{n}: rel-RMSE {e:.3e} > {GATES[n]}"
+    lg = np.stack([got["lse"].numpy()[b, :, i] for b, i in rows])
+    lr = np.stack([lse[b, :, i] for b, i in rows])
+    assert np.max(np.abs(lg - lr)) < 2e-3
+    return errs
+
+
+def sample_rows(wl, n, seed):
+    rng = np.random.default_rng(seed)
+    rows = {(0, 0), (wl.B - 1, wl.N - 1)}
+    while len(rows) < n:
+        rows.add((int(rng.integers(wl.B)), int(rng.integers(wl.N))))
+    sel = {(0, 0, 0), (wl.B - 1, wl.H - 1, wl.N - 1)}
+    while len(sel) < n:
+        sel.add((int(rng.integers(wl.B)), int(rng.integers(wl.H)), int(rng.integers(wl.N))))
+    return sorted(rows), sorted(sel)
+
+
+# ---------------------------------------------------------------------------
+# full comparisons on small cases (several tiles, ragged tails)
+# ---------------------------------------------------------------------------
+
+def test_tiny_full():
+    x = S.make_inputs(S.TINY, S.seed_for(0, 0))
+    got = run_gpu(x, "start")
+    errs, ref = check_full(x, got)
+    # the BF16 rounding residual carries what BF16 rounding dropped from O
+    assert rel(got["out"].numpy() + got["resid"].numpy(), ref["out"]) < 0.05 * errs["out"]
+
+
+@pytest.mark.parametrize("d", [32, 64])
+def test_two_tiles_ragged_mask_full(d):
+    wl = S.Workload("small ragged", 2, 136, 2, d, mask="ragged", len_lo=70, len_hi=136)
+    x = S.make_inputs(wl, 77 + d)
+    check_full(x, run_gpu(x, "start"))
+
+
+def test_odd_N_with_padded_bias_rows():
+    # N odd (the last pair of rows has a single row) and not a multiple of 8: the
+    # bias lives in a [.., N, 40] buffer so its row stride stays 16-byte aligned
+    wl = S.Workload("odd", 1, 37, 2, 32, mask="ragged", len_lo=20, len_hi=37)
+    x = S.make_inputs(wl, 5)
+    pad = torch.zeros(1, 2, 37, 40, dtype=torch.bfloat16)
+    pad[..., :37] = x["bias"]
+    x["bias"] = pad[..., :37]
+    check_full(x, run_gpu(x, "start"))
+
+
+def test_ending_node_full():
+    wl = S.Workload("end small", 1, 72, 2, 32, mask="ragged", len_lo=40, len_hi=72, orientation="end")
+    x = S.make_inputs(wl, 9)
+    check_full(x, run_gpu(x, "end"), "end")
+
+
+def test_no_mask_equals_zero_mask_bitwise():
+    wl = S.Workload("zeros", 1, 96, 2, 32, mask="zeros")
+    x = S.make_inputs(wl, 3)
+    a = run_gpu(x, "start")
+    x2 = dict(x)
+    x2["mask"] = None
+    b = run_gpu(x2, "start")
+    for n in a:
+        assert torch.equal(a[n], b[n]), n
+
+
+# ---------------------------------------------------------------------------
+# crop-sized workloads: sampled rows at full size
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("wl,idx", [(S.CROP384, 1), (S.CROP640, 2),
+                                    (S.CROP640.with_(orientation="end"), 2)])
+def test_crop_sampled(wl, idx):
+    x = S.make_inputs(wl, S.seed_for(idx, 0))
+    got = run_gpu(x, wl.orientation)
+    rows, sel = sample_rows(wl, 6, idx)
+    check_sampled(x, got, rows, sel, wl.orientation)
+
+
+def test_crop768_sampled_and_bitwise_repeatable():
+    wl = S.CROP768
+    x = S.make_inputs(wl, S.seed_for(3, 0))
+    runs = [run_gpu(x, "start") for _ in range(5)]
+    for r in runs[1:]:
+        for n in runs[0]:
+            assert torch.equal(r[n].view(torch.int32) if r[n].dtype == torch.float32 else r[n],
+                               runs[0][n].view(torch.int32) if runs[0][n].dtype == torch.float32 else runs[0][n]), n
+    rows, sel = sample_rows(wl, 6, 3)
+    check_sampled(x, runs[0], rows, sel)
+
+
+@pytest.mark.parametrize("N", S.SWEEP_NS)
+@pytest.mark.parametrize("d", S.SWEEP_DS)
+def test_sweep_sampled(N, d):
+    wl = S.sweep(N, d)
+    x = S.make_inputs(wl, S.seed_for(4, 10 * d + N // 128))
+    got = run_gpu(x, "start")
+    rows, sel = sample_rows(wl, 4, N + d)
+    check_sampled(x, got, rows, sel)
+
+
+# ---------------------------------------------------------------------------
+# residual compensation variant and the bounded-wait path
+# ---------------------------------------------------------------------------
+
+def test_uncompensated_variant_runs_and_stays_within_gates():
+    wl = S.Workload("ablation", 1, 128, 4, 32)
+    x = S.make_inputs(wl, 11)
+    got = run_gpu(x, "start", flags=Bd.TRI_ATTN_BWD_NO_RESIDUAL)
+    check_full(x, got)
+
+
+def test_bounded_wait_expires_and_context_survives():
+    Bd.tri_attn_device_error(True)
+    Bd.tri_attn_set_wait_limit_ns(2_000_000)  # 2 ms
+    try:
+        Bd.tri_attn_selftest_expire_wait()
+        torch.cuda.synchronize()
+        st, word = Bd.tri_attn_device_error(True)
+        assert st == Bd.TRI_ATTN_ERR_DEVICE_TIMEOUT and word != 0
+    finally:
+        Bd.tri_attn_set_wait_limit_ns(2_000_000_000)
+    # the context is still usable
+    x = S.make_inputs(S.TINY, 1)
+    check_full(x, run_gpu(x, "start"))

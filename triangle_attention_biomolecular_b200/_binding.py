@@ -1,0 +1,240 @@
+"""ctypes binding of libtriattn.so (include/tri_attn.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI.  PyTorch tensors supply device memory and the
+stream; their data pointers and element strides are copied into the C
+argument structs.  If the shared library is missing the first call raises --
+there is no other implementation to fall back to.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtriattn.so")
+
+TRI_ATTN_OK = 0
+TRI_ATTN_ERR_NULL = 1
+TRI_ATTN_ERR_SHAPE = 2
+TRI_ATTN_ERR_STRIDE = 3
+TRI_ATTN_ERR_ALIGN = 4
+TRI_ATTN_ERR_DTYPE = 5
+TRI_ATTN_ERR_UNSUPPORTED = 6
+TRI_ATTN_ERR_WORKSPACE = 7
+TRI_ATTN_ERR_ARCH = 8
+TRI_ATTN_ERR_CUDA = 9
+TRI_ATTN_ERR_DEVICE_TIMEOUT = 10
+TRI_ATTN_BWD_NO_RESIDUAL = 1
+
+
+class TriAttnError(RuntimeError):
+    def __init__(self, status: int, where: str = ""):
+        self.status = int(status)
+        msg = tri_attn_strerror(self.status) if _lib is not None else f"status {status}"
+        super().__init__(f"{where}: {msg} (status {self.status})" if where else msg)
+
+
+class Tensor5(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("stride", ctypes.c_int64 * 5)]
+
+
+class Tensor4(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("stride", ctypes.c_int64 * 4)]
+
+
+class Mask(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("stride", ctypes.c_int64 * 3)]
+
+
+class FwdArgs(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("N", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int),
+                ("scale", ctypes.c_float),
+                ("q", Tensor5), ("k", Tensor5), ("v", Tensor5), ("bias", Tensor4), ("mask", Mask),
+                ("o", Tensor5), ("resid", Tensor5), ("lse", ctypes.c_void_p)]
+
+
+class BwdArgs(ctypes.Structure):
+    _fields_ = [("f", FwdArgs), ("dout", Tensor5), ("dq", Tensor5), ("dk", Tensor5), ("dv", Tensor5),
+                ("dbias", Tensor4), ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+                ("flags", ctypes.c_uint)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def load() -> ctypes.CDLL:
+    """Load libtriattn.so (built in-tree by build.py); raise if it is missing."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"libtriattn.so not found at {LIB_PATH}; build it with "
+                    "`python -m triangle_attention_biomolecular_b200.build`")
+            lib = ctypes.CDLL(LIB_PATH)
+            lib.tri_attn_fwd.argtypes = [ctypes.POINTER(FwdArgs), ctypes.c_void_p]
+            lib.tri_attn_fwd.restype = ctypes.c_int
+            lib.tri_attn_bwd.argtypes = [ctypes.POINTER(BwdArgs), ctypes.c_void_p]
+            lib.tri_attn_bwd.restype = ctypes.c_int
+            lib.tri_attn_bwd_workspace_bytes.argtypes = [ctypes.c_int] * 4
+            lib.tri_attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+            lib.tri_attn_strerror.argtypes = [ctypes.c_int]
+            lib.tri_attn_strerror.restype = ctypes.c_char_p
+            lib.tri_attn_device_error.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_uint32)]
+            lib.tri_attn_device_error.restype = ctypes.c_int
+            lib.tri_attn_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+            lib.tri_attn_set_wait_limit_ns.restype = None
+            lib.tri_attn_selftest_expire_wait.argtypes = [ctypes.c_void_p]
+            lib.tri_attn_selftest_expire_wait.restype = ctypes.c_int
+            lib.tri_attn_abi_version.argtypes = []
+            lib.tri_attn_abi_version.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+# ---------------------------------------------------------------------------
+# marshalling helpers (torch tensors -> C structs)
+# ---------------------------------------------------------------------------
+
+def _check_tensor(t, name, dtype, dims):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TriAttnError(TRI_ATTN_ERR_DTYPE, f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != dims:
+        raise TriAttnError(TRI_ATTN_ERR_SHAPE, f"{name} must have {dims} dims")
+
+
+def t5(t, name="tensor") -> Tensor5:
+    import torch
+    _check_tensor(t, name, torch.bfloat16, 5)
+    s = Tensor5()
+    s.ptr = t.data_ptr()
+    for a in range(5):
+        s.stride[a] = t.stride(a)
+    return s
+
+
+def t4(t, name="bias") -> Tensor4:
+    import torch
+    _check_tensor(t, name, torch.bfloat16, 4)
+    s = Tensor4()
+    s.ptr = t.data_ptr()
+    for a in range(4):
+        s.stride[a] = t.stride(a)
+    return s
+
+
+def mask3(m) -> Mask:
+    import torch
+    s = Mask()
+    if m is None:
+        s.ptr = None
+        return s
+    _check_tensor(m, "mask", torch.float32, 3)
+    s.ptr = m.data_ptr()
+    for a in range(3):
+        s.stride[a] = m.stride(a)
+    return s
+
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def fwd_args(q, k, v, bias, mask, o, resid, lse, scale: float = 0.0) -> FwdArgs:
+    import torch
+    B, N, N2, H, d = q.shape
+    if N2 != N:
+        raise TriAttnError(TRI_ATTN_ERR_SHAPE, "q must be [B,N,N,H,d]")
+    for name, t in (("k", k), ("v", v), ("o", o), ("resid", resid)):
+        if tuple(t.shape) != (B, N, N, H, d):
+            raise TriAttnError(TRI_ATTN_ERR_SHAPE, f"{name} shape {tuple(t.shape)} != {(B, N, N, H, d)}")
+    if tuple(bias.shape) != (B, H, N, N):
+        raise TriAttnError(TRI_ATTN_ERR_SHAPE, "bias must be [B,H,N,N]")
+    if mask is not None and tuple(mask.shape) != (B, N, N):
+        raise TriAttnError(TRI_ATTN_ERR_SHAPE, "mask must be [B,N,N] (b,i,k)")
+    _check_tensor(lse, "lse", torch.float32, 4)
+    if tuple(lse.shape) != (B, H, N, N) or not lse.is_contiguous():
+        raise TriAttnError(TRI_ATTN_ERR_SHAPE, "lse must be a contiguous [B,H,N,N] float32 tensor")
+    a = FwdArgs()
+    a.B, a.N, a.H, a.d = B, N, H, d
+    a.scale = float(scale)
+    a.q, a.k, a.v = t5(q, "q"), t5(k, "k"), t5(v, "v")
+    a.bias = t4(bias)
+    a.mask = mask3(mask)
+    a.o, a.resid = t5(o, "o"), t5(resid, "resid")
+    a.lse = lse.data_ptr()
+    return a
+
+
+# ---------------------------------------------------------------------------
+# the C entry points, same names
+# ---------------------------------------------------------------------------
+
+def tri_attn_strerror(status: int) -> str:
+    return load().tri_attn_strerror(int(status)).decode()
+
+
+def tri_attn_abi_version() -> int:
+    return load().tri_attn_abi_version()
+
+
+def tri_attn_bwd_workspace_bytes(B: int, N: int, H: int, d: int) -> int:
+    return int(load().tri_attn_bwd_workspace_bytes(B, N, H, d))
+
+
+def tri_attn_fwd(q, k, v, bias, mask, o, resid, lse, scale: float = 0.0, stream=None) -> None:
+    """Enqueue the forward; o, resid (BF16) and lse (FP32 [B,H,N,N]) are written."""
+    a = fwd_args(q, k, v, bias, mask, o, resid, lse, scale)
+    st = load().tri_attn_fwd(ctypes.byref(a), _stream_handle(stream))
+    if st != TRI_ATTN_OK:
+        raise TriAttnError(st, "tri_attn_fwd")
+
+
+def tri_attn_bwd(q, k, v, bias, mask, o, resid, lse, dout, dq, dk, dv, dbias, workspace,
+                 scale: float = 0.0, flags: int = 0, stream=None) -> None:
+    """Enqueue the backward; dq, dk, dv, dbias (BF16) are written.  workspace is a
+    caller-owned uint8 CUDA tensor of at least tri_attn_bwd_workspace_bytes bytes."""
+    import torch
+    a = BwdArgs()
+    a.f = fwd_args(q, k, v, bias, mask, o, resid, lse, scale)
+    a.dout = t5(dout, "dout")
+    a.dq, a.dk, a.dv = t5(dq, "dq"), t5(dk, "dk"), t5(dv, "dv")
+    a.dbias = t4(dbias, "dbias")
+    if workspace is None:
+        a.workspace, a.workspace_bytes = None, 0
+    else:
+        if workspace.dtype != torch.uint8:
+            raise TriAttnError(TRI_ATTN_ERR_DTYPE, "workspace must be a uint8 tensor")
+        a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    a.flags = int(flags)
+    st = load().tri_attn_bwd(ctypes.byref(a), _stream_handle(stream))
+    if st != TRI_ATTN_OK:
+        raise TriAttnError(st, "tri_attn_bwd")
+
+
+def tri_attn_device_error(clear: bool = True):
+    """(status, raw word) of the device error word; synchronises the device."""
+    w = ctypes.c_uint32(0)
+    st = load().tri_attn_device_error(1 if clear else 0, ctypes.byref(w))
+    return int(st), int(w.value)
+
+
+def tri_attn_set_wait_limit_ns(ns: int) -> None:
+    load().tri_attn_set_wait_limit_ns(int(ns))
+
+
+def tri_attn_selftest_expire_wait(stream=None) -> None:
+    st = load().tri_attn_selftest_expire_wait(_stream_handle(stream))
+    if st != TRI_ATTN_OK:
+        raise TriAttnError(st, "tri_attn_selftest_expire_wait")

@@ -1,0 +1,415 @@
+// api.cu -- the C ABI of libtriattn.so (declared in include/tri_attn.h):
+// host-side validation, TMA descriptor encoding and kernel launches.
+//
+// Validation happens entirely on the host before any CUDA call, so argument
+// errors are reported without touching the device.  The driver's tensor-map
+// encoder is fetched through the runtime's driver entry point, so the library
+// has no link-time dependency on libcuda.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/tri_attn.h"
+#include "sm100.cuh"
+#include "fwd.cuh"
+#include "bwd.cuh"
+
+namespace {
+
+std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+
+constexpr int kMaxN = 4096;
+constexpr int kMaxDevices = 64;
+
+// ---------------------------------------------------------------------------
+// validation helpers
+// ---------------------------------------------------------------------------
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+tri_attn_status check_t5(const tri_attn_tensor5& t) {
+    if (!t.ptr) return TRI_ATTN_ERR_NULL;
+    if (t.stride[4] != 1) return TRI_ATTN_ERR_STRIDE;
+    for (int a = 0; a < 4; ++a)
+        if (t.stride[a] < 0 || (t.stride[a] % 8) != 0) return TRI_ATTN_ERR_STRIDE;
+    if (!aligned16(t.ptr)) return TRI_ATTN_ERR_ALIGN;
+    return TRI_ATTN_OK;
+}
+tri_attn_status check_t4(const tri_attn_tensor4& t) {
+    if (!t.ptr) return TRI_ATTN_ERR_NULL;
+    if (t.stride[3] != 1) return TRI_ATTN_ERR_STRIDE;
+    for (int a = 0; a < 3; ++a)
+        if (t.stride[a] < 0 || (t.stride[a] % 8) != 0) return TRI_ATTN_ERR_STRIDE;
+    if (!aligned16(t.ptr)) return TRI_ATTN_ERR_ALIGN;
+    return TRI_ATTN_OK;
+}
+
+tri_attn_status check_sizes(int B, int N, int H, int d) {
+    if (B < 1 || N < 1 || H < 1) return TRI_ATTN_ERR_SHAPE;
+    if (d != 32 && d != 64) return TRI_ATTN_ERR_UNSUPPORTED;
+    if (N > kMaxN) return TRI_ATTN_ERR_UNSUPPORTED;
+    // 32-bit work-item and index arithmetic inside the kernels
+    const double items = static_cast<double>(B) * H * N * ((N + 127) / 128);
+    if (items > 2.0e9) return TRI_ATTN_ERR_SHAPE;
+    return TRI_ATTN_OK;
+}
+
+tri_attn_status check_fwd_args(const tri_attn_fwd_args* a) {
+    if (!a) return TRI_ATTN_ERR_NULL;
+    tri_attn_status st = check_sizes(a->B, a->N, a->H, a->d);
+    if (st) return st;
+    const tri_attn_tensor5* t5[] = {&a->q, &a->k, &a->v, &a->o, &a->resid};
+    for (const auto* t : t5)
+        if ((st = check_t5(*t))) return st;
+    if ((st = check_t4(a->bias))) return st;
+    if (!a->lse) return TRI_ATTN_ERR_NULL;
+    if (!aligned16(a->lse)) return TRI_ATTN_ERR_ALIGN;
+    if (a->mask.ptr && (reinterpret_cast<uintptr_t>(a->mask.ptr) & 3u)) return TRI_ATTN_ERR_ALIGN;
+    if (!std::isfinite(a->scale)) return TRI_ATTN_ERR_SHAPE;
+    return TRI_ATTN_OK;
+}
+
+// ---------------------------------------------------------------------------
+// device checks and the driver's tensor-map encoder
+// ---------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encoder() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+// 0 unknown, 1 ok (sm_100 and kernel attributes set), 2 wrong arch
+std::atomic<int> g_dev_state[kMaxDevices];
+
+tri_attn_status ensure_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+        cudaGetLastError();
+        return TRI_ATTN_ERR_CUDA;
+    }
+    if (dev >= kMaxDevices) return TRI_ATTN_ERR_CUDA;
+    int s = g_dev_state[dev].load();
+    if (s == 1) return TRI_ATTN_OK;
+    if (s == 2) return TRI_ATTN_ERR_ARCH;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return TRI_ATTN_ERR_CUDA;
+    }
+    if (major != 10 || minor != 0) {
+        g_dev_state[dev].store(2);
+        return TRI_ATTN_ERR_ARCH;
+    }
+    bool ok = true;
+    ok &= cudaFuncSetAttribute(tri::tri_attn_fwd_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               tri::FwdLayout<32>::SMEM) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(tri::tri_attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               tri::FwdLayout<64>::SMEM) == cudaSuccess;
+    ok &= tri::bwd_set_attributes();
+    if (!ok || !encoder()) {
+        cudaGetLastError();
+        return TRI_ATTN_ERR_CUDA;
+    }
+    g_dev_state[dev].store(1);
+    return TRI_ATTN_OK;
+}
+
+// Outer (non-innermost) dimensions of a tensor map, sorted by increasing
+// byte stride so the descriptor always sees an ascending stride order.
+struct OuterDim {
+    uint64_t size, stride_bytes;
+    uint32_t box;
+    int tag;
+};
+
+// Encode a tiled BF16 map.  inner = innermost extent (contiguous), inner_box
+// its box; outer dims are sorted by stride and their final positions (1-based
+// in the map) are returned through pos[tag].
+bool encode_map(CUtensorMap* m, void* ptr, uint64_t inner, uint32_t inner_box, OuterDim* od, int nouter,
+                CUtensorMapSwizzle swz, int* pos) {
+    // size-1 dims may carry any stride; give them a harmless valid one
+    for (int a = 0; a < nouter; ++a)
+        if (od[a].size == 1 || od[a].stride_bytes == 0) od[a].stride_bytes = 0;
+    std::stable_sort(od, od + nouter, [](const OuterDim& x, const OuterDim& y) { return x.stride_bytes < y.stride_bytes; });
+    uint64_t prev = inner * 2;
+    for (int a = 0; a < nouter; ++a) {
+        if (od[a].stride_bytes == 0) od[a].stride_bytes = ((prev + 15) / 16) * 16;
+        prev = od[a].stride_bytes * od[a].size;
+    }
+    cuuint64_t dims[5], strides[4];
+    cuuint32_t box[5], estr[5] = {1, 1, 1, 1, 1};
+    dims[0] = inner;
+    box[0] = inner_box;
+    for (int a = 0; a < nouter; ++a) {
+        dims[a + 1] = od[a].size;
+        strides[a] = od[a].stride_bytes;
+        box[a + 1] = od[a].box;
+        pos[od[a].tag] = a + 1;
+        if (od[a].stride_bytes % 16 || od[a].stride_bytes >= (1ull << 40)) return false;
+    }
+    CUresult r = encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 1 + nouter, ptr, dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Pair tensor [B,N,N,H,d] map with a 128-row box along j (or along i when
+// `rows_along_i`): tags 0=h, 1=j, 2=i, 3=b.
+bool map_pair(CUtensorMap* m, const tri_attn_tensor5& t, int B, int N, int H, int d, bool rows_along_i,
+              int* pos) {
+    OuterDim od[4] = {
+        {static_cast<uint64_t>(H), static_cast<uint64_t>(t.stride[3]) * 2, 1, 0},
+        {static_cast<uint64_t>(N), static_cast<uint64_t>(t.stride[2]) * 2, rows_along_i ? 1u : 128u, 1},
+        {static_cast<uint64_t>(N), static_cast<uint64_t>(t.stride[1]) * 2, rows_along_i ? 128u : 1u, 2},
+        {static_cast<uint64_t>(B), static_cast<uint64_t>(t.stride[0]) * 2, 1, 3},
+    };
+    return encode_map(m, t.ptr, d, d, od, 4, d == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                      pos);
+}
+
+// Bias [B,H,N,N] map: box 64 keys x 128 query rows, 128-byte swizzle; tags 0=j, 1=h, 2=b.
+bool map_bias(CUtensorMap* m, const tri_attn_tensor4& t, int B, int N, int H, int* pos) {
+    OuterDim od[3] = {
+        {static_cast<uint64_t>(N), static_cast<uint64_t>(t.stride[2]) * 2, 128, 0},
+        {static_cast<uint64_t>(H), static_cast<uint64_t>(t.stride[1]) * 2, 1, 1},
+        {static_cast<uint64_t>(B), static_cast<uint64_t>(t.stride[0]) * 2, 1, 2},
+    };
+    return encode_map(m, t.ptr, N, 64, od, 3, CU_TENSOR_MAP_SWIZZLE_128B, pos);
+}
+
+float eff_scale(float s, int d) { return s == 0.f ? 1.0f / std::sqrt(static_cast<float>(d)) : s; }
+
+}  // namespace
+
+// ===========================================================================
+// backward launch (declared in bwd.cuh)
+// ===========================================================================
+namespace tri {
+
+bool bwd_set_attributes() {
+    bool ok = true;
+    ok &= cudaFuncSetAttribute(tri_attn_bwd_main_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               MainLayout<32>::SMEM) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(tri_attn_bwd_main_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               MainLayout<64>::SMEM) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(tri_attn_bwd_dbias_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               DbLayout<32>::SMEM) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(tri_attn_bwd_dbias_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               DbLayout<64>::SMEM) == cudaSuccess;
+    return ok;
+}
+
+tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, float scale, uint64_t wait_ns,
+                           cudaStream_t stream) {
+    const tri_attn_fwd_args& f = a->f;
+    const int B = f.B, N = f.N, H = f.H, d = f.d;
+    CUtensorMap mq, mk, mv, mdo, mb;
+    int pq[4], pk[4], pv[4], pdo[4], pb[3];
+    if (!map_pair(&mq, f.q, B, N, H, d, false, pq) || !map_pair(&mk, f.k, B, N, H, d, false, pk) ||
+        !map_pair(&mv, f.v, B, N, H, d, false, pv) || !map_pair(&mdo, a->dout, B, N, H, d, false, pdo) ||
+        !map_bias(&mb, f.bias, B, N, H, pb))
+        return TRI_ATTN_ERR_STRIDE;
+    if (std::memcmp(pq, pk, sizeof pq) || std::memcmp(pq, pv, sizeof pq) || std::memcmp(pq, pdo, sizeof pq))
+        return TRI_ATTN_ERR_STRIDE;
+    uint8_t* wsb = static_cast<uint8_t*>(a->workspace);
+    BwdParams p{};
+    p.B = B; p.N = N; p.H = H;
+    p.nt = (N + 127) / 128;
+    p.scale = scale;
+    p.qpos_h = pq[0]; p.qpos_j = pq[1]; p.qpos_i = pq[2]; p.qpos_b = pq[3];
+    p.bpos_j = pb[0]; p.bpos_h = pb[1]; p.bpos_b = pb[2];
+    p.mask = f.mask.ptr;
+    p.ms0 = f.mask.stride[0]; p.ms1 = f.mask.stride[1]; p.ms2 = f.mask.stride[2];
+    p.lse = f.lse;
+    p.Dv = reinterpret_cast<float*>(wsb + ws.off_D);
+    p.dq_slots = reinterpret_cast<float*>(wsb + ws.off_dq);
+    p.part = reinterpret_cast<float*>(wsb + ws.off_part);
+    p.chunks = ws.chunks;
+    p.dq = static_cast<__nv_bfloat16*>(a->dq.ptr);
+    p.dk = static_cast<__nv_bfloat16*>(a->dk.ptr);
+    p.dv = static_cast<__nv_bfloat16*>(a->dv.ptr);
+    p.dbias = static_cast<__nv_bfloat16*>(a->dbias.ptr);
+    for (int x = 0; x < 5; ++x) { p.dqs[x] = a->dq.stride[x]; p.dks[x] = a->dk.stride[x]; p.dvs[x] = a->dv.stride[x]; }
+    for (int x = 0; x < 4; ++x) p.dbs[x] = a->dbias.stride[x];
+    p.wait_limit_ns = wait_ns;
+
+    const int64_t rows = static_cast<int64_t>(B) * H * N * N;
+    const unsigned prep_grid = static_cast<unsigned>(std::min<int64_t>((rows + 255) / 256, 148 * 16));
+    const int use_resid = (a->flags & TRI_ATTN_BWD_NO_RESIDUAL) ? 0 : 1;
+    const unsigned db_grid = static_cast<unsigned>(B) * H * p.nt * p.nt * ws.chunks;
+    const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(f.bias.ptr);
+    const auto& so = f.o.stride; const auto& sr = f.resid.stride; const auto& sd = a->dout.stride;
+    if (d == 32) {
+        tri_attn_bwd_prep_kernel<32><<<prep_grid, 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(a->dout.ptr), sd[0], sd[1], sd[2], sd[3],
+            static_cast<const __nv_bfloat16*>(f.o.ptr), so[0], so[1], so[2], so[3],
+            static_cast<const __nv_bfloat16*>(f.resid.ptr), sr[0], sr[1], sr[2], sr[3], use_resid, p.Dv, B, N, H);
+        tri_attn_bwd_main_kernel<32><<<ws.grid_main, 320, MainLayout<32>::SMEM, stream>>>(mq, mk, mv, mdo, mb, p);
+        tri_attn_bwd_dbias_kernel<32><<<db_grid, 320, DbLayout<32>::SMEM, stream>>>(
+            mq, mk, mv, mdo, bias, f.bias.stride[0], f.bias.stride[1], f.bias.stride[2], p);
+    } else {
+        tri_attn_bwd_prep_kernel<64><<<prep_grid, 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(a->dout.ptr), sd[0], sd[1], sd[2], sd[3],
+            static_cast<const __nv_bfloat16*>(f.o.ptr), so[0], so[1], so[2], so[3],
+            static_cast<const __nv_bfloat16*>(f.resid.ptr), sr[0], sr[1], sr[2], sr[3], use_resid, p.Dv, B, N, H);
+        tri_attn_bwd_main_kernel<64><<<ws.grid_main, 320, MainLayout<64>::SMEM, stream>>>(mq, mk, mv, mdo, mb, p);
+        tri_attn_bwd_dbias_kernel<64><<<db_grid, 320, DbLayout<64>::SMEM, stream>>>(
+            mq, mk, mv, mdo, bias, f.bias.stride[0], f.bias.stride[1], f.bias.stride[2], p);
+    }
+    if (ws.chunks > 1) {
+        const unsigned rg = static_cast<unsigned>(std::min<int64_t>((rows + 255) / 256, 148 * 16));
+        tri_attn_bwd_dbias_reduce_kernel<<<rg, 256, 0, stream>>>(p.part, ws.chunks, B, H, N, p.dbias,
+                                                                  a->dbias.stride[0], a->dbias.stride[1],
+                                                                  a->dbias.stride[2]);
+    }
+    return cudaGetLastError() == cudaSuccess ? TRI_ATTN_OK : TRI_ATTN_ERR_CUDA;
+}
+
+}  // namespace tri
+
+// ===========================================================================
+// exported entry points
+// ===========================================================================
+extern "C" {
+
+int tri_attn_abi_version(void) { return TRI_ATTN_ABI_VERSION; }
+
+const char* tri_attn_strerror(tri_attn_status s) {
+    switch (s) {
+        case TRI_ATTN_OK: return "ok";
+        case TRI_ATTN_ERR_NULL: return "a required pointer is NULL";
+        case TRI_ATTN_ERR_SHAPE: return "B, N or H out of range";
+        case TRI_ATTN_ERR_STRIDE: return "innermost stride must be 1 and other strides non-negative multiples of 8 elements";
+        case TRI_ATTN_ERR_ALIGN: return "a data pointer is not 16-byte aligned";
+        case TRI_ATTN_ERR_DTYPE: return "wrong element type";
+        case TRI_ATTN_ERR_UNSUPPORTED: return "unsupported size (d must be 32 or 64, N <= 4096)";
+        case TRI_ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+        case TRI_ATTN_ERR_ARCH: return "current device is not compute capability 10.0 (sm_100)";
+        case TRI_ATTN_ERR_CUDA: return "a CUDA call failed";
+        case TRI_ATTN_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel expired";
+    }
+    return "unknown status";
+}
+
+void tri_attn_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns ? ns : 1); }
+
+tri_attn_status tri_attn_fwd(const tri_attn_fwd_args* a, tri_attn_stream_t stream) {
+    tri_attn_status st = check_fwd_args(a);
+    if (st) return st;
+    if ((st = ensure_device())) return st;
+    const int B = a->B, N = a->N, H = a->H, d = a->d;
+    CUtensorMap mq, mk, mv, mb;
+    int pq[4], pk[4], pv[4], pb[3];
+    if (!map_pair(&mq, a->q, B, N, H, d, false, pq) || !map_pair(&mk, a->k, B, N, H, d, false, pk) ||
+        !map_pair(&mv, a->v, B, N, H, d, false, pv) || !map_bias(&mb, a->bias, B, N, H, pb))
+        return TRI_ATTN_ERR_STRIDE;
+    if (std::memcmp(pq, pk, sizeof pq) || std::memcmp(pq, pv, sizeof pq)) return TRI_ATTN_ERR_STRIDE;
+    tri::FwdParams p{};
+    p.B = B; p.N = N; p.H = H;
+    p.nt = (N + 127) / 128;
+    p.npairs = (N + 1) / 2;
+    p.scale = eff_scale(a->scale, d);
+    p.qpos_h = pq[0]; p.qpos_j = pq[1]; p.qpos_i = pq[2]; p.qpos_b = pq[3];
+    p.bpos_j = pb[0]; p.bpos_h = pb[1]; p.bpos_b = pb[2];
+    p.mask = a->mask.ptr;
+    p.ms0 = a->mask.stride[0]; p.ms1 = a->mask.stride[1]; p.ms2 = a->mask.stride[2];
+    p.o = static_cast<__nv_bfloat16*>(a->o.ptr);
+    p.r = static_cast<__nv_bfloat16*>(a->resid.ptr);
+    for (int x = 0; x < 5; ++x) { p.os[x] = a->o.stride[x]; p.rs[x] = a->resid.stride[x]; }
+    p.lse = a->lse;
+    p.wait_limit_ns = g_wait_limit_ns.load();
+    const unsigned grid = static_cast<unsigned>(B) * p.npairs * H * p.nt;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (d == 32)
+        tri::tri_attn_fwd_kernel<32><<<grid, 320, tri::FwdLayout<32>::SMEM, s>>>(mq, mk, mv, mb, p);
+    else
+        tri::tri_attn_fwd_kernel<64><<<grid, 320, tri::FwdLayout<64>::SMEM, s>>>(mq, mk, mv, mb, p);
+    return cudaGetLastError() == cudaSuccess ? TRI_ATTN_OK : TRI_ATTN_ERR_CUDA;
+}
+
+size_t tri_attn_bwd_workspace_bytes(int B, int N, int H, int d) {
+    if (check_sizes(B, N, H, d)) return 0;
+    return tri::bwd_workspace_layout(B, N, H, d).total;
+}
+
+tri_attn_status tri_attn_bwd(const tri_attn_bwd_args* a, tri_attn_stream_t stream) {
+    if (!a) return TRI_ATTN_ERR_NULL;
+    tri_attn_status st = check_fwd_args(&a->f);
+    if (st) return st;
+    const tri_attn_tensor5* t5[] = {&a->dout, &a->dq, &a->dk, &a->dv};
+    for (const auto* t : t5)
+        if ((st = check_t5(*t))) return st;
+    if ((st = check_t4(a->dbias))) return st;
+    const int B = a->f.B, N = a->f.N, H = a->f.H, d = a->f.d;
+    const tri::BwdWorkspace ws = tri::bwd_workspace_layout(B, N, H, d);
+    if (!a->workspace || a->workspace_bytes < ws.total) return TRI_ATTN_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(a->workspace) & 255u) return TRI_ATTN_ERR_ALIGN;
+    if ((st = ensure_device())) return st;
+    return tri::bwd_launch(a, ws, eff_scale(a->f.scale, d), g_wait_limit_ns.load(),
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+tri_attn_status tri_attn_device_error(int clear, uint32_t* word) {
+    uint32_t w = 0;
+    if (cudaMemcpyFromSymbol(&w, tri::g_error_word, sizeof w) != cudaSuccess) {
+        cudaGetLastError();
+        return TRI_ATTN_ERR_CUDA;
+    }
+    if (word) *word = w;
+    if (clear) {
+        const uint32_t z = 0;
+        if (cudaMemcpyToSymbol(tri::g_error_word, &z, sizeof z) != cudaSuccess) {
+            cudaGetLastError();
+            return TRI_ATTN_ERR_CUDA;
+        }
+    }
+    return w ? TRI_ATTN_ERR_DEVICE_TIMEOUT : TRI_ATTN_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// self-test of the bounded-wait path: a barrier that nothing ever completes
+// ---------------------------------------------------------------------------
+namespace tri {
+__global__ void selftest_expire_kernel(uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        mbar_init(smem_addr(&bar), 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const WaitCtx wc{limit_ns, KERNEL_SELFTEST, &abort_flag};
+        (void)mbar_wait(smem_addr(&bar), 0, wc, 1);
+    }
+    __syncthreads();
+}
+}  // namespace tri
+
+extern "C" tri_attn_status tri_attn_selftest_expire_wait(tri_attn_stream_t stream) {
+    tri_attn_status st = ensure_device();
+    if (st) return st;
+    tri::selftest_expire_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(g_wait_limit_ns.load());
+    return cudaGetLastError() == cudaSuccess ? TRI_ATTN_OK : TRI_ATTN_ERR_CUDA;
+}

@@ -1,0 +1,932 @@
+// bwd.cuh -- triangle-attention backward for sm_100a.
+//
+// Pages: "TurboPairFormer: более быстрое, стабильное и точное дообучение
+// OpenFold3" (dev48.org), section "Как работает TurboPairFormer" (probability
+// tiles recomputed in the backward; BF16 output-rounding residual used for
+// the gradients; fixed accumulation order for bitwise-repeatable gradients),
+// and "16张H100，训练步提速1.73倍：TurboPairFormer…" (biocloudservice.com),
+// section "它优化了什么": the correction term is formed in FP32 from the saved
+// residual; no floating-point atomics.
+//
+// Three reductions meet in this backward: dK/dV sum over queries j, dQ sums
+// over keys k, and dBias sums over pair rows i (the bias is shared by every
+// row).  A CTA cannot keep accumulators for all three on chip at N=768 (TMEM
+// holds 128 x 512 FP32), so the work is split:
+//
+//  1. tri_attn_bwd_prep_kernel: D[b,h,i,j] = sum_c dout * (o + resid), FP32.
+//  2. tri_attn_bwd_main_kernel (problem-stationary): one persistent CTA walks
+//     whole problems (b,i,h): key tiles kt outer, query tiles jt inner.  Per
+//     tile it recomputes S and dP with tcgen05, forms P and dS once, stages
+//     them in SMEM (BF16, 128B-swizzled) and issues dV += P^T dO,
+//     dK += dS^T Q, dQ_tile = dS K.  dK/dV finish in TMEM per key tile; dQ
+//     accumulates over key tiles in a per-CTA FP32 slot of the workspace, in
+//     ascending kt order, by the same thread each time.
+//  3. tri_attn_bwd_dbias_kernel (tile-stationary): one CTA per (b,h,jt,kt)
+//     and row chunk walks i in ascending order, recomputes S, dP -> dS and
+//     accumulates dBias in FP32 registers.  Chunks (only when there are
+//     fewer tiles than SMs) are summed in ascending chunk order by
+//     tri_attn_bwd_dbias_reduce_kernel.
+// Every reduction therefore has one fixed order: results are bitwise
+// repeatable and independent of the SM count.
+#pragma once
+
+#include "../../include/tri_attn.h"
+#include "sm100.cuh"
+#include "fwd.cuh"
+
+namespace tri {
+
+constexpr int kDqSlots = 148;   // persistent CTAs of the main kernel (B200 SM count)
+constexpr int kChunkTarget = 148;
+
+struct BwdWorkspace {
+    size_t off_D, off_dq, off_part, total;
+    int chunks;     // row chunks of the dBias kernel
+    int grid_main;  // CTAs of the main kernel
+};
+
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+inline BwdWorkspace bwd_workspace_layout(int B, int N, int H, int d) {
+    BwdWorkspace w{};
+    const size_t nt = (N + 127) / 128;
+    const size_t tiles = static_cast<size_t>(B) * H * nt * nt;
+    int chunks = 1;
+    if (tiles < static_cast<size_t>(kChunkTarget)) {
+        chunks = static_cast<int>(kChunkTarget / tiles);
+        chunks = chunks < 1 ? 1 : chunks;
+        const int max_chunks = (N + 7) / 8;  // at least 8 rows per chunk
+        chunks = chunks > max_chunks ? max_chunks : chunks;
+    }
+    w.chunks = chunks;
+    const size_t problems = static_cast<size_t>(B) * N * H;
+    w.grid_main = static_cast<int>(problems < static_cast<size_t>(kDqSlots) ? problems : kDqSlots);
+    const size_t bhnn = static_cast<size_t>(B) * H * N * N;
+    w.off_D = 0;
+    w.off_dq = align256(bhnn * 4);
+    w.off_part = w.off_dq + align256(static_cast<size_t>(kDqSlots) * N * d * 4);
+    w.total = w.off_part + (chunks > 1 ? align256(static_cast<size_t>(chunks) * bhnn * 4) : 0);
+    return w;
+}
+
+struct BwdParams {
+    int B, N, H, nt;
+    float scale;
+    int qpos_h, qpos_j, qpos_i, qpos_b;  // tensor-map coordinate positions (pair tensors)
+    int bpos_j, bpos_h, bpos_b;          // bias tensor map
+    const float* mask;
+    int64_t ms0, ms1, ms2;
+    const float* lse;  // [B,H,N,N]
+    float* Dv;         // [B,H,N,N] workspace
+    float* dq_slots;   // [kDqSlots][N][d]
+    float* part;       // [chunks][B,H,N,N] (chunks > 1)
+    int chunks;
+    __nv_bfloat16 *dq, *dk, *dv, *dbias;
+    int64_t dqs[5], dks[5], dvs[5], dbs[4];
+    uint64_t wait_limit_ns;
+};
+
+// ===========================================================================
+// 1. D = rowsum(dout * (o + resid))
+// ===========================================================================
+template <int D>
+__global__ void __launch_bounds__(256) tri_attn_bwd_prep_kernel(
+    const __nv_bfloat16* __restrict__ dout, int64_t s0, int64_t s1, int64_t s2, int64_t s3,
+    const __nv_bfloat16* __restrict__ o, int64_t o0, int64_t o1, int64_t o2, int64_t o3,
+    const __nv_bfloat16* __restrict__ r, int64_t r0, int64_t r1, int64_t r2, int64_t r3, int use_resid,
+    float* __restrict__ Dout, int B, int N, int H) {
+    const int64_t total = static_cast<int64_t>(B) * H * N * N;
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        int64_t t = idx;
+        const int j = static_cast<int>(t % N);
+        t /= N;
+        const int i = static_cast<int>(t % N);
+        t /= N;
+        const int h = static_cast<int>(t % H);
+        const int b = static_cast<int>(t / H);
+        const uint4* pd = reinterpret_cast<const uint4*>(dout + b * s0 + i * s1 + j * s2 + h * s3);
+        const uint4* po = reinterpret_cast<const uint4*>(o + b * o0 + i * o1 + j * o2 + h * o3);
+        const uint4* pr = reinterpret_cast<const uint4*>(r + b * r0 + i * r1 + j * r2 + h * r3);
+        float acc = 0.f;
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+            const uint4 a = __ldg(pd + c), bo = __ldg(po + c);
+            uint4 br = make_uint4(0, 0, 0, 0);
+            if (use_resid) br = __ldg(pr + c);
+            const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, ow[4] = {bo.x, bo.y, bo.z, bo.w},
+                           rw[4] = {br.x, br.y, br.z, br.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                acc = fmaf(bf16lo(aw[e]), bf16lo(ow[e]) + bf16lo(rw[e]), acc);
+                acc = fmaf(bf16hi(aw[e]), bf16hi(ow[e]) + bf16hi(rw[e]), acc);
+            }
+        }
+        Dout[idx] = acc;
+    }
+}
+
+// ===========================================================================
+// 2. main backward kernel: dq, dk, dv
+// ===========================================================================
+template <int D>
+struct MainLayout {
+    static constexpr int KVS = (D == 32) ? 2 : 1;  // K/V buffers
+    static constexpr int NS = 2;                   // per-tile stages (Q, dO, bias, vectors)
+    static constexpr int ROWB = D * 2;
+    static constexpr int QKV_TILE = 128 * ROWB;
+    static constexpr int BIAS_TILE = 128 * 128 * 2;
+    static constexpr int PT_TILE = 128 * 128 * 2;  // P or dS, BF16, two 64-column SW128 halves
+    // 1 KB aligned tiles
+    static constexpr int OFF_KV = 0;  // [KVS][K, V]
+    static constexpr int OFF_T = OFF_KV + KVS * 2 * QKV_TILE;  // [NS][Q, dO, bias]
+    static constexpr int T_STAGE = 2 * QKV_TILE + BIAS_TILE;
+    static constexpr int OFF_P = OFF_T + NS * T_STAGE;
+    static constexpr int OFF_DS = OFF_P + PT_TILE;
+    // vectors
+    static constexpr int OFF_MASKV = OFF_DS + PT_TILE;      // [KVS][128] fp32
+    static constexpr int OFF_VEC = OFF_MASKV + KVS * 512;   // [NS][lse2 128, D 128] fp32
+    static constexpr int OFF_BAR = OFF_VEC + NS * 1024;
+    static constexpr int B_KVFULL = 0, B_KVEMPTY = KVS, B_TFULL = 2 * KVS, B_TEMPTY = 2 * KVS + NS,
+                         B_SDPFULL = 2 * KVS + 2 * NS, B_SDPFREE = B_SDPFULL + 1, B_PDSFULL = B_SDPFULL + 2,
+                         B_PDSFREE = B_SDPFULL + 3, B_DQFULL = B_SDPFULL + 4, B_DQFREE = B_SDPFULL + 5,
+                         B_DKVFULL = B_SDPFULL + 6, B_DKVFREE = B_SDPFULL + 7, B_DRAIN = B_SDPFULL + 8,
+                         NBAR = B_DRAIN + 1;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag, mask flags[KVS]
+    static constexpr int SMEM = OFF_MISC + 16 + KVS * 4;
+    static_assert(SMEM <= 232448, "shared memory budget");
+    // TMEM columns
+    static constexpr int T_S = 0, T_DP = 128, T_DK = 256, T_DV = 256 + D, T_DQ = 256 + 2 * D;
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    tri_attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                             const __grid_constant__ CUtensorMap tm_bias, const BwdParams p) {
+    using L = MainLayout<D>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t sb = smem_addr(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    auto BAR = [&](int idx) -> uint32_t { return sb + L::OFF_BAR + idx * 8; };
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+    volatile int* mask_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 16);
+
+    const int nt = p.nt;
+    const int problems = p.B * p.N * p.H;
+    // problem index -> (b, h, i) with i fastest so concurrent CTAs share a head's bias
+    auto decode = [&](int pr, int& b, int& h, int& i) {
+        i = pr % p.N;
+        const int t = pr / p.N;
+        h = t % p.H;
+        b = t / p.H;
+    };
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        if (sb & 1023u) {
+            atomicCAS(&g_error_word, 0u, ERR_TIMEOUT_BIT | KERNEL_BWD_MAIN | 0xFFu);
+            *abort_flag = 1;
+        }
+        for (int s = 0; s < L::KVS; ++s) {
+            mbar_init(BAR(L::B_KVFULL + s), 1);
+            mbar_init(BAR(L::B_KVEMPTY + s), 1 + 8);
+        }
+        for (int s = 0; s < L::NS; ++s) {
+            mbar_init(BAR(L::B_TFULL + s), 1);
+            mbar_init(BAR(L::B_TEMPTY + s), 1 + 8);
+        }
+        mbar_init(BAR(L::B_SDPFULL), 1);
+        mbar_init(BAR(L::B_SDPFREE), 8);
+        mbar_init(BAR(L::B_PDSFULL), 8);
+        mbar_init(BAR(L::B_PDSFREE), 1);
+        mbar_init(BAR(L::B_DQFULL), 1);
+        mbar_init(BAR(L::B_DQFREE), 8);
+        mbar_init(BAR(L::B_DKVFULL), 1);
+        mbar_init(BAR(L::B_DKVFREE), 8);
+        mbar_init(BAR(L::B_DRAIN), 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_addr(const_cast<uint32_t*>(tmem_slot)), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const WaitCtx wc{p.wait_limit_ns, KERNEL_BWD_MAIN, abort_flag};
+    const bool aborted_early = *abort_flag != 0;
+    constexpr float LOG2E = 1.4426950408889634f;
+
+    if (warp == 8) {
+        // =========================== producer ===============================
+        int armed_kv[L::KVS], armed_t[L::NS];
+#pragma unroll
+        for (int s = 0; s < L::KVS; ++s) armed_kv[s] = 0;
+#pragma unroll
+        for (int s = 0; s < L::NS; ++s) armed_t[s] = 0;
+        if (!aborted_early) {
+            if (lane == 0) {
+                tma_prefetch_map(&tm_q);
+                tma_prefetch_map(&tm_k);
+                tma_prefetch_map(&tm_v);
+                tma_prefetch_map(&tm_do);
+                tma_prefetch_map(&tm_bias);
+            }
+            int gk = 0, g = 0;
+            bool ok = true;
+            for (int pr = blockIdx.x; ok && pr < problems; pr += gridDim.x) {
+                int b, h, i;
+                decode(pr, b, h, i);
+                auto load_pair = [&](uint32_t dst, const CUtensorMap* m, uint32_t bar, int row0) {
+                    int c[5] = {0, 0, 0, 0, 0};
+                    c[p.qpos_h] = h;
+                    c[p.qpos_j] = row0;
+                    c[p.qpos_i] = i;
+                    c[p.qpos_b] = b;
+                    tma_load_5d(dst, m, bar, c[0], c[1], c[2], c[3], c[4]);
+                };
+                auto load_bias = [&](uint32_t dst, uint32_t bar, int k0, int j0) {
+                    int c[4] = {0, 0, 0, 0};
+                    c[0] = k0;
+                    c[p.bpos_j] = j0;
+                    c[p.bpos_h] = h;
+                    c[p.bpos_b] = b;
+                    tma_load_4d(dst, &tm_bias, bar, c[0], c[1], c[2], c[3]);
+                };
+                for (int kt = 0; ok && kt < nt; ++kt) {
+                    const int ks = gk % L::KVS;
+                    if (gk >= L::KVS && !mbar_wait_warp(BAR(L::B_KVEMPTY + ks), ((gk / L::KVS) - 1) & 1, wc, 1)) {
+                        ok = false;
+                        break;
+                    }
+                    {  // key mask row (user mask, -inf past N)
+                        float v[4];
+                        bool nz = false;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int k = kt * 128 + lane * 4 + e;
+                            float x = -INFINITY;
+                            if (k < p.N) x = p.mask ? __ldg(p.mask + b * p.ms0 + i * p.ms1 + k * p.ms2) : 0.f;
+                            v[e] = x;
+                            nz |= (x != 0.f);
+                        }
+                        *reinterpret_cast<float4*>(smem + L::OFF_MASKV + ks * 512 + lane * 16) =
+                            make_float4(v[0], v[1], v[2], v[3]);
+                        const unsigned any = __any_sync(0xFFFFFFFFu, nz);
+                        if (lane == 0) mask_flag[ks] = any ? 1 : 0;
+                    }
+                    __syncwarp();
+                    if (lane == 0) {
+                        const uint32_t bar = BAR(L::B_KVFULL + ks);
+                        const uint32_t base = sb + L::OFF_KV + ks * 2 * L::QKV_TILE;
+                        mbar_arrive_expect_tx(bar, 2 * L::QKV_TILE);
+                        load_pair(base, &tm_k, bar, kt * 128);
+                        load_pair(base + L::QKV_TILE, &tm_v, bar, kt * 128);
+                    }
+                    armed_kv[ks]++;
+                    ++gk;
+                    for (int jt = 0; jt < nt; ++jt) {
+                        const int ts = g % L::NS;
+                        if (g >= L::NS && !mbar_wait_warp(BAR(L::B_TEMPTY + ts), ((g / L::NS) - 1) & 1, wc, 2)) {
+                            ok = false;
+                            break;
+                        }
+                        {  // lse (log2 units) and D rows for this query tile
+                            float* vec = reinterpret_cast<float*>(smem + L::OFF_VEC + ts * 1024);
+                            const int64_t rowbase = ((static_cast<int64_t>(b) * p.H + h) * p.N + i) * p.N;
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int jj = lane * 4 + e;
+                                const int j = jt * 128 + jj;
+                                float lv = INFINITY, dv = 0.f;
+                                if (j < p.N) {
+                                    lv = __ldg(p.lse + rowbase + j) * LOG2E;
+                                    dv = p.Dv[rowbase + j];
+                                }
+                                vec[jj] = lv;
+                                vec[128 + jj] = dv;
+                            }
+                        }
+                        __syncwarp();
+                        if (lane == 0) {
+                            const uint32_t bar = BAR(L::B_TFULL + ts);
+                            const uint32_t base = sb + L::OFF_T + ts * L::T_STAGE;
+                            mbar_arrive_expect_tx(bar, 2 * L::QKV_TILE + L::BIAS_TILE);
+                            load_pair(base, &tm_q, bar, jt * 128);
+                            load_pair(base + L::QKV_TILE, &tm_do, bar, jt * 128);
+                            load_bias(base + 2 * L::QKV_TILE, bar, kt * 128, jt * 128);
+                            load_bias(base + 2 * L::QKV_TILE + L::BIAS_TILE / 2, bar, kt * 128 + 64, jt * 128);
+                        }
+                        armed_t[ts]++;
+                        ++g;
+                    }
+                }
+            }
+        }
+        if (lane == 0) {
+#pragma unroll
+            for (int s = 0; s < L::KVS; ++s)
+                if (armed_kv[s] > 0) drain_wait(BAR(L::B_KVFULL + s), (armed_kv[s] - 1) & 1, 100000000ull);
+#pragma unroll
+            for (int s = 0; s < L::NS; ++s)
+                if (armed_t[s] > 0) drain_wait(BAR(L::B_TFULL + s), (armed_t[s] - 1) & 1, 100000000ull);
+        }
+    } else if (warp == 9) {
+        // =========================== MMA issuer =============================
+        if (lane == 0 && !aborted_early) {
+            constexpr uint32_t SW = (D == 32) ? SWZ_64B : SWZ_128B;
+            constexpr uint32_t SBO = 8 * L::ROWB;
+            constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);  // Q K^T, dO V^T
+            constexpr uint32_t IDESC_G = idesc_bf16_f32(128, D, true, true);      // P^T dO, dS^T Q
+            constexpr uint32_t IDESC_Q = idesc_bf16_f32(128, D, false, true);     // dS K
+            struct Pending {
+                int g, ts, ks, jt, kcount;
+                bool valid;
+            } pend{0, 0, 0, 0, 0, false};
+            bool ok = true;
+            auto issue_grads = [&](const Pending& t) -> bool {
+                if (!mbar_wait(BAR(L::B_PDSFULL), t.g & 1, wc, 3)) return false;
+                if (t.g > 0 && !mbar_wait(BAR(L::B_DQFREE), (t.g - 1) & 1, wc, 4)) return false;
+                if (t.jt == 0 && t.kcount > 0 && !mbar_wait(BAR(L::B_DKVFREE), (t.kcount - 1) & 1, wc, 5))
+                    return false;
+                tc_fence_after();
+                const uint32_t tb = sb + L::OFF_T + t.ts * L::T_STAGE;
+                const uint32_t qa = tb, doa = tb + L::QKV_TILE;
+                const uint32_t ka = sb + L::OFF_KV + t.ks * 2 * L::QKV_TILE;
+                const uint32_t pa = sb + L::OFF_P, dsa = sb + L::OFF_DS;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {  // contraction over 128 queries
+                    const uint32_t acc = (t.jt > 0 || kk > 0) ? 1u : 0u;
+                    // A = P^T / dS^T: MN-major, 64-element chunks 16 KB apart, 8-row groups 1 KB apart
+                    const uint64_t adp = smem_desc(pa + kk * 2048, L::PT_TILE / 2, 1024, SWZ_128B);
+                    const uint64_t ads = smem_desc(dsa + kk * 2048, L::PT_TILE / 2, 1024, SWZ_128B);
+                    // B = dO / Q rows j: MN-major over channels
+                    const uint64_t bdo = smem_desc(doa + kk * 16 * L::ROWB, L::QKV_TILE, SBO, SW);
+                    const uint64_t bq = smem_desc(qa + kk * 16 * L::ROWB, L::QKV_TILE, SBO, SW);
+                    mma_ss(tmem + L::T_DV, adp, bdo, IDESC_G, acc);
+                    mma_ss(tmem + L::T_DK, ads, bq, IDESC_G, acc);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {  // contraction over 128 keys
+                    // A = dS rows j: K-major, two 64-key halves 16 KB apart
+                    const uint64_t a = smem_desc(dsa + (kk >> 2) * (L::PT_TILE / 2) + (kk & 3) * 32, 16, 1024, SWZ_128B);
+                    const uint64_t bk = smem_desc(ka + kk * 16 * L::ROWB, L::QKV_TILE, SBO, SW);
+                    mma_ss(tmem + L::T_DQ, a, bk, IDESC_Q, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(BAR(L::B_PDSFREE));
+                mma_commit(BAR(L::B_TEMPTY + t.ts));
+                mma_commit(BAR(L::B_DQFULL));
+                if (t.jt == nt - 1) {
+                    mma_commit(BAR(L::B_DKVFULL));
+                    mma_commit(BAR(L::B_KVEMPTY + t.ks));
+                }
+                return true;
+            };
+            int gk = 0, g = 0;
+            for (int pr = blockIdx.x; ok && pr < problems; pr += gridDim.x) {
+                for (int kt = 0; ok && kt < nt; ++kt) {
+                    const int ks = gk % L::KVS;
+                    if (L::KVS == 1 && pend.valid && pend.jt == nt - 1) {
+                        // the single K/V buffer is released only by this tile's gradients
+                        if (!(ok = issue_grads(pend))) break;
+                        pend.valid = false;
+                    }
+                    if (!mbar_wait(BAR(L::B_KVFULL + ks), (gk / L::KVS) & 1, wc, 6)) { ok = false; break; }
+                    const uint32_t ka = sb + L::OFF_KV + ks * 2 * L::QKV_TILE;
+                    const uint32_t va = ka + L::QKV_TILE;
+                    for (int jt = 0; jt < nt; ++jt) {
+                        const int ts = g % L::NS;
+                        if (!mbar_wait(BAR(L::B_TFULL + ts), (g / L::NS) & 1, wc, 7)) { ok = false; break; }
+                        if (g > 0 && !mbar_wait(BAR(L::B_SDPFREE), (g - 1) & 1, wc, 8)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t tb = sb + L::OFF_T + ts * L::T_STAGE;
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            mma_ss(tmem + L::T_S, smem_desc(tb + kk * 32, 16, SBO, SW),
+                                   smem_desc(ka + kk * 32, 16, SBO, SW), IDESC_S, kk > 0 ? 1u : 0u);
+                            mma_ss(tmem + L::T_DP, smem_desc(tb + L::QKV_TILE + kk * 32, 16, SBO, SW),
+                                   smem_desc(va + kk * 32, 16, SBO, SW), IDESC_S, kk > 0 ? 1u : 0u);
+                        }
+                        mma_commit(BAR(L::B_SDPFULL));
+                        if (pend.valid) {
+                            if (!(ok = issue_grads(pend))) break;
+                        }
+                        pend = Pending{g, ts, ks, jt, gk, true};
+                        ++g;
+                    }
+                    ++gk;
+                }
+            }
+            if (ok && pend.valid) ok = issue_grads(pend);
+            mma_commit(BAR(L::B_DRAIN));
+            drain_wait(BAR(L::B_DRAIN), 0, 100000000ull);
+        }
+        __syncwarp();
+    } else if (!aborted_early) {
+        // =========================== softmax + epilogue warps ===============
+        const int w = warp >> 2;  // column half of every tile handled by this warpgroup
+        const int qd = warp & 3;
+        const int row = qd * 32 + lane;
+        const uint32_t tl = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+        const float scale = p.scale, c2 = p.scale * LOG2E;
+        struct Done {
+            int g, jt, kt, kcount, b, h, i;
+            bool valid;
+        } prev{0, 0, 0, 0, 0, 0, 0, false};
+        bool ok = true;
+
+        auto epilogue = [&](const Done& t) -> bool {
+            // ---- dQ tile: this warpgroup's D/2 columns, accumulated over kt in the slot ----
+            if (!mbar_wait_warp(BAR(L::B_DQFULL), t.g & 1, wc, 10)) return false;
+            tc_fence_after();
+            uint32_t dqr[D / 2];
+            if constexpr (D == 32) {
+                uint32_t x[16];
+                tmem_ld16(tl + L::T_DQ + w * 16, x);
+                tmem_wait_ld();
+                asm volatile("" : "+r"(x[0]), "+r"(x[1]), "+r"(x[2]), "+r"(x[3]), "+r"(x[4]), "+r"(x[5]),
+                             "+r"(x[6]), "+r"(x[7]), "+r"(x[8]), "+r"(x[9]), "+r"(x[10]), "+r"(x[11]),
+                             "+r"(x[12]), "+r"(x[13]), "+r"(x[14]), "+r"(x[15]));
+#pragma unroll
+                for (int e = 0; e < 16; ++e) dqr[e] = x[e];
+            } else {
+                uint32_t x[32];
+                tmem_ld32(tl + L::T_DQ + w * 32, x);
+                tmem_wait_ld();
+                reg_fence32(x);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) dqr[e] = x[e];
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(BAR(L::B_DQFREE));
+            const int j = t.jt * 128 + row;
+            if (j < p.N) {
+                float* slot = p.dq_slots + (static_cast<int64_t>(blockIdx.x) * p.N + j) * D + w * (D / 2);
+                float acc[D / 2];
+#pragma unroll
+                for (int e = 0; e < D / 2; ++e) acc[e] = __uint_as_float(dqr[e]);
+                if (t.kt > 0) {
+#pragma unroll
+                    for (int e = 0; e < D / 2; e += 4) {
+                        const float4 v = *reinterpret_cast<const float4*>(slot + e);
+                        acc[e] += v.x;
+                        acc[e + 1] += v.y;
+                        acc[e + 2] += v.z;
+                        acc[e + 3] += v.w;
+                    }
+                }
+                if (t.kt < nt - 1) {
+#pragma unroll
+                    for (int e = 0; e < D / 2; e += 4)
+                        *reinterpret_cast<float4*>(slot + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+                } else {
+                    __nv_bfloat16* dst = p.dq + t.b * p.dqs[0] + t.i * p.dqs[1] + j * p.dqs[2] + t.h * p.dqs[3] + w * (D / 2);
+#pragma unroll
+                    for (int e = 0; e < D / 2; e += 8) {
+                        uint4 v;
+                        v.x = pack_bf16(acc[e] * scale, acc[e + 1] * scale);
+                        v.y = pack_bf16(acc[e + 2] * scale, acc[e + 3] * scale);
+                        v.z = pack_bf16(acc[e + 4] * scale, acc[e + 5] * scale);
+                        v.w = pack_bf16(acc[e + 6] * scale, acc[e + 7] * scale);
+                        *reinterpret_cast<uint4*>(dst + e) = v;
+                    }
+                }
+            }
+            // ---- dK (warpgroup 0) or dV (warpgroup 1) of a finished key tile ----
+            if (t.jt == nt - 1) {
+                if (!mbar_wait_warp(BAR(L::B_DKVFULL), t.kcount & 1, wc, 11)) return false;
+                tc_fence_after();
+                uint32_t g16[D];
+#pragma unroll
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t x[32];
+                    tmem_ld32(tl + (w == 0 ? L::T_DK : L::T_DV) + c0, x);
+                    tmem_wait_ld();
+                    reg_fence32(x);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) g16[c0 + e] = x[e];
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(BAR(L::B_DKVFREE));
+                const int k = t.kt * 128 + row;
+                if (k < p.N) {
+                    const float f = (w == 0) ? scale : 1.f;
+                    __nv_bfloat16* dst = (w == 0)
+                        ? p.dk + t.b * p.dks[0] + t.i * p.dks[1] + k * p.dks[2] + t.h * p.dks[3]
+                        : p.dv + t.b * p.dvs[0] + t.i * p.dvs[1] + k * p.dvs[2] + t.h * p.dvs[3];
+#pragma unroll
+                    for (int e = 0; e < D; e += 8) {
+                        uint4 v;
+                        v.x = pack_bf16(__uint_as_float(g16[e]) * f, __uint_as_float(g16[e + 1]) * f);
+                        v.y = pack_bf16(__uint_as_float(g16[e + 2]) * f, __uint_as_float(g16[e + 3]) * f);
+                        v.z = pack_bf16(__uint_as_float(g16[e + 4]) * f, __uint_as_float(g16[e + 5]) * f);
+                        v.w = pack_bf16(__uint_as_float(g16[e + 6]) * f, __uint_as_float(g16[e + 7]) * f);
+                        *reinterpret_cast<uint4*>(dst + e) = v;
+                    }
+                }
+            }
+            return true;
+        };
+
+        int gk = 0, g = 0;
+        for (int pr = blockIdx.x; ok && pr < problems; pr += gridDim.x) {
+            int b, h, i;
+            decode(pr, b, h, i);
+            for (int kt = 0; ok && kt < nt; ++kt) {
+                const int ks = gk % L::KVS;
+                if (!mbar_wait_warp(BAR(L::B_KVFULL + ks), (gk / L::KVS) & 1, wc, 12)) { ok = false; break; }
+                const bool has_mask = mask_flag[ks] != 0;
+                const uint32_t maskv = sb + L::OFF_MASKV + ks * 512 + w * 256;
+                for (int jt = 0; jt < nt; ++jt) {
+                    const int ts = g % L::NS;
+                    if (!mbar_wait_warp(BAR(L::B_SDPFULL), g & 1, wc, 13)) { ok = false; break; }
+                    tc_fence_after();
+                    uint32_t s0[32], s1[32], d0[32], d1[32];
+                    tmem_ld32(tl + L::T_S + w * 64, s0);
+                    tmem_ld32(tl + L::T_S + w * 64 + 32, s1);
+                    tmem_ld32(tl + L::T_DP + w * 64, d0);
+                    tmem_ld32(tl + L::T_DP + w * 64 + 32, d1);
+                    tmem_wait_ld();
+                    reg_fence32(s0);
+                    reg_fence32(s1);
+                    reg_fence32(d0);
+                    reg_fence32(d1);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(BAR(L::B_SDPFREE));
+                    if (!mbar_wait_warp(BAR(L::B_TFULL + ts), (g / L::NS) & 1, wc, 14)) { ok = false; break; }
+                    const uint32_t tb = sb + L::OFF_T + ts * L::T_STAGE;
+                    const float* vec = reinterpret_cast<const float*>(smem + L::OFF_VEC + ts * 1024);
+                    const float lse2 = vec[row];
+                    const float Dj = vec[128 + row];
+                    // bias row j, this warpgroup's 64-key half
+                    const uint32_t brow = tb + 2 * L::QKV_TILE + w * (L::BIAS_TILE / 2) + row * 128;
+                    // P and dS rows go straight into the SW128 K-major tiles (this warpgroup's half)
+                    if (g > 0 && !mbar_wait_warp(BAR(L::B_PDSFREE), (g - 1) & 1, wc, 15)) { ok = false; break; }
+                    const uint32_t prow = sb + L::OFF_P + w * (L::PT_TILE / 2) + row * 128;
+                    const uint32_t drow = sb + L::OFF_DS + w * (L::PT_TILE / 2) + row * 128;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint32_t off = (c ^ (row & 7)) << 4;
+                        const uint4 bb = lds128(brow + off);
+                        const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+                        float mk[8];
+                        if (has_mask) {
+                            const float4 m0 = lds128f(maskv + c * 32), m1 = lds128f(maskv + c * 32 + 16);
+                            mk[0] = m0.x; mk[1] = m0.y; mk[2] = m0.z; mk[3] = m0.w;
+                            mk[4] = m1.x; mk[5] = m1.y; mk[6] = m1.z; mk[7] = m1.w;
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) mk[e] = 0.f;
+                        }
+                        uint32_t pw[4], dw[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int x0 = c * 8 + 2 * e;
+                            const uint32_t sv0 = (x0 < 32) ? s0[x0] : s1[x0 - 32];
+                            const uint32_t sv1 = (x0 + 1 < 32) ? s0[x0 + 1] : s1[x0 + 1 - 32];
+                            const uint32_t dv0 = (x0 < 32) ? d0[x0] : d1[x0 - 32];
+                            const uint32_t dv1 = (x0 + 1 < 32) ? d0[x0 + 1] : d1[x0 + 1 - 32];
+                            // y*log2e = S*scale*log2e + (bias + mask)*log2e
+                            const float y0 = fmaf(__uint_as_float(sv0), c2, (bf16lo(bw[e]) + mk[2 * e]) * LOG2E);
+                            const float y1 = fmaf(__uint_as_float(sv1), c2, (bf16hi(bw[e]) + mk[2 * e + 1]) * LOG2E);
+                            const float p0 = ex2(y0 - lse2), p1 = ex2(y1 - lse2);
+                            const float ds0 = p0 * (__uint_as_float(dv0) - Dj);
+                            const float ds1 = p1 * (__uint_as_float(dv1) - Dj);
+                            pw[e] = pack_bf16(p0, p1);
+                            dw[e] = pack_bf16(ds0, ds1);
+                        }
+                        sts128(prow + off, make_uint4(pw[0], pw[1], pw[2], pw[3]));
+                        sts128(drow + off, make_uint4(dw[0], dw[1], dw[2], dw[3]));
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(BAR(L::B_PDSFULL));
+                        mbar_arrive(BAR(L::B_TEMPTY + ts));
+                        if (jt == nt - 1) mbar_arrive(BAR(L::B_KVEMPTY + ks));
+                    }
+                    if (prev.valid && !(ok = epilogue(prev))) break;
+                    prev = Done{g, jt, kt, gk, b, h, i, true};
+                    ++g;
+                }
+                ++gk;
+            }
+        }
+        if (ok && prev.valid) epilogue(prev);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ===========================================================================
+// 3. dBias kernel: one CTA per (b, h, jt, kt, row chunk), rows i ascending
+// ===========================================================================
+template <int D>
+struct DbLayout {
+    static constexpr int NS = (D == 32) ? 3 : 2;
+    static constexpr int ROWB = D * 2;
+    static constexpr int QKV_TILE = 128 * ROWB;
+    static constexpr int STAGE = 4 * QKV_TILE;  // Q, dO, K, V
+    static constexpr int OFF_BIAS = NS * STAGE;  // [128 rows][128 keys] fp32, log2 units, swizzled
+    static constexpr int OFF_VEC = OFF_BIAS + 128 * 128 * 4;  // [NS][lse2 128, D 128, mask 128] fp32
+    static constexpr int VEC = 1536;
+    static constexpr int OFF_BAR = OFF_VEC + NS * VEC;
+    static constexpr int B_FULL = 0, B_EMPTY = NS, B_SDPFULL = 2 * NS, B_SDPFREE = 2 * NS + 2,
+                         B_DRAIN = 2 * NS + 4, NBAR = B_DRAIN + 1;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort, mask flags[NS]
+    static constexpr int SMEM = OFF_MISC + 16 + NS * 4;
+    static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    tri_attn_bwd_dbias_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                              const __nv_bfloat16* __restrict__ bias, int64_t bs0, int64_t bs1, int64_t bs2,
+                              const BwdParams p) {
+    using L = DbLayout<D>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t sb = smem_addr(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    auto BAR = [&](int idx) -> uint32_t { return sb + L::OFF_BAR + idx * 8; };
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+    volatile int* mask_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 16);
+
+    const int nt = p.nt;
+    int item = blockIdx.x;
+    const int chunk = item % p.chunks;
+    item /= p.chunks;
+    const int kt = item % nt;
+    item /= nt;
+    const int jt = item % nt;
+    item /= nt;
+    const int h = item % p.H;
+    const int b = item / p.H;
+    const int rows_per = (p.N + p.chunks - 1) / p.chunks;
+    const int i_begin = chunk * rows_per;
+    const int i_end = min(p.N, i_begin + rows_per);
+    const int nrows = max(0, i_end - i_begin);
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        if (sb & 1023u) {
+            atomicCAS(&g_error_word, 0u, ERR_TIMEOUT_BIT | KERNEL_BWD_DBIAS | 0xFFu);
+            *abort_flag = 1;
+        }
+        for (int s = 0; s < L::NS; ++s) {
+            mbar_init(BAR(L::B_FULL + s), 1);
+            mbar_init(BAR(L::B_EMPTY + s), 1 + 8);
+        }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(BAR(L::B_SDPFULL + x), 1);
+            mbar_init(BAR(L::B_SDPFREE + x), 8);
+        }
+        mbar_init(BAR(L::B_DRAIN), 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_addr(const_cast<uint32_t*>(tmem_slot)), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const WaitCtx wc{p.wait_limit_ns, KERNEL_BWD_DBIAS, abort_flag};
+    const bool aborted_early = *abort_flag != 0;
+    constexpr float LOG2E = 1.4426950408889634f;
+
+    if (warp == 8) {
+        int armed[L::NS];
+#pragma unroll
+        for (int s = 0; s < L::NS; ++s) armed[s] = 0;
+        if (!aborted_early) {
+            if (lane == 0) {
+                tma_prefetch_map(&tm_q);
+                tma_prefetch_map(&tm_k);
+                tma_prefetch_map(&tm_v);
+                tma_prefetch_map(&tm_do);
+            }
+            for (int n = 0; n < nrows; ++n) {
+                const int i = i_begin + n;
+                const int s = n % L::NS;
+                if (n >= L::NS && !mbar_wait_warp(BAR(L::B_EMPTY + s), ((n / L::NS) - 1) & 1, wc, 1)) break;
+                float* vec = reinterpret_cast<float*>(smem + L::OFF_VEC + s * L::VEC);
+                const int64_t rowbase = ((static_cast<int64_t>(b) * p.H + h) * p.N + i) * p.N;
+                bool nz = false;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int jj = lane * 4 + e;
+                    const int j = jt * 128 + jj;
+                    float lv = INFINITY, dv = 0.f;
+                    if (j < p.N) {
+                        lv = __ldg(p.lse + rowbase + j) * LOG2E;
+                        dv = p.Dv[rowbase + j];
+                    }
+                    vec[jj] = lv;
+                    vec[128 + jj] = dv;
+                    const int k = kt * 128 + jj;
+                    float mv = -INFINITY;
+                    if (k < p.N) mv = p.mask ? __ldg(p.mask + b * p.ms0 + i * p.ms1 + k * p.ms2) : 0.f;
+                    vec[256 + jj] = mv * LOG2E;
+                    nz |= (mv != 0.f);
+                }
+                const unsigned any = __any_sync(0xFFFFFFFFu, nz);
+                if (lane == 0) mask_flag[s] = any ? 1 : 0;
+                __syncwarp();
+                if (lane == 0) {
+                    const uint32_t bar = BAR(L::B_FULL + s);
+                    const uint32_t base = sb + s * L::STAGE;
+                    mbar_arrive_expect_tx(bar, L::STAGE);
+                    auto ld = [&](uint32_t dst, const CUtensorMap* m, int row0) {
+                        int c[5] = {0, 0, 0, 0, 0};
+                        c[p.qpos_h] = h;
+                        c[p.qpos_j] = row0;
+                        c[p.qpos_i] = i;
+                        c[p.qpos_b] = b;
+                        tma_load_5d(dst, m, bar, c[0], c[1], c[2], c[3], c[4]);
+                    };
+                    ld(base, &tm_q, jt * 128);
+                    ld(base + L::QKV_TILE, &tm_do, jt * 128);
+                    ld(base + 2 * L::QKV_TILE, &tm_k, kt * 128);
+                    ld(base + 3 * L::QKV_TILE, &tm_v, kt * 128);
+                }
+                armed[s]++;
+            }
+        }
+        if (lane == 0) {
+#pragma unroll
+            for (int s = 0; s < L::NS; ++s)
+                if (armed[s] > 0) drain_wait(BAR(L::B_FULL + s), (armed[s] - 1) & 1, 100000000ull);
+        }
+    } else if (warp == 9) {
+        if (lane == 0 && !aborted_early) {
+            constexpr uint32_t SW = (D == 32) ? SWZ_64B : SWZ_128B;
+            constexpr uint32_t SBO = 8 * L::ROWB;
+            constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
+            for (int n = 0; n < nrows; ++n) {
+                const int s = n % L::NS, x = n & 1;
+                if (!mbar_wait(BAR(L::B_FULL + s), (n / L::NS) & 1, wc, 2)) break;
+                if (n >= 2 && !mbar_wait(BAR(L::B_SDPFREE + x), ((n >> 1) - 1) & 1, wc, 3)) break;
+                tc_fence_after();
+                const uint32_t base = sb + s * L::STAGE;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    mma_ss(tmem + x * 256, smem_desc(base + kk * 32, 16, SBO, SW),
+                           smem_desc(base + 2 * L::QKV_TILE + kk * 32, 16, SBO, SW), IDESC_S, kk > 0 ? 1u : 0u);
+                    mma_ss(tmem + x * 256 + 128, smem_desc(base + L::QKV_TILE + kk * 32, 16, SBO, SW),
+                           smem_desc(base + 3 * L::QKV_TILE + kk * 32, 16, SBO, SW), IDESC_S, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(BAR(L::B_SDPFULL + x));
+                mma_commit(BAR(L::B_EMPTY + s));
+            }
+            mma_commit(BAR(L::B_DRAIN));
+            drain_wait(BAR(L::B_DRAIN), 0, 100000000ull);
+        }
+        __syncwarp();
+    } else if (!aborted_early) {
+        const int w = warp >> 2;
+        const int qd = warp & 3;
+        const int row = qd * 32 + lane;
+        const uint32_t tl = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+        const int j = jt * 128 + row;
+        const float c2 = p.scale * LOG2E;
+        // this thread's 64 bias values (row j, keys kt*128 + 64w ..), log2 units, kept in
+        // shared memory (row = 256 B = 16 chunks, chunk index xor (row & 15))
+        const uint32_t brow = sb + L::OFF_BIAS + row * 512 + w * 256;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            float v[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int k = kt * 128 + w * 64 + 4 * c + e;
+                float bv = 0.f;
+                if (j < p.N && k < p.N)
+                    bv = __bfloat162float(bias[b * bs0 + h * bs1 + static_cast<int64_t>(j) * bs2 + k]);
+                v[e] = bv * LOG2E;
+            }
+            sts128(brow + ((c ^ (row & 15)) << 4),
+                   make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]), __float_as_uint(v[3])));
+        }
+        float acc[64];
+#pragma unroll
+        for (int e = 0; e < 64; ++e) acc[e] = 0.f;
+        bool ok = true;
+        for (int n = 0; n < nrows; ++n) {
+            const int x = n & 1, s = n % L::NS;
+            if (!mbar_wait_warp(BAR(L::B_SDPFULL + x), (n >> 1) & 1, wc, 4)) { ok = false; break; }
+            tc_fence_after();
+            if (!mbar_wait_warp(BAR(L::B_FULL + s), (n / L::NS) & 1, wc, 5)) { ok = false; break; }
+            const float* vec = reinterpret_cast<const float*>(smem + L::OFF_VEC + s * L::VEC);
+            const float lse2 = vec[row];
+            const float Dj = vec[128 + row];
+            const bool has_mask = mask_flag[s] != 0;
+            const uint32_t ma = sb + L::OFF_VEC + s * L::VEC + 1024 + w * 256;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t sv[32], dv[32];
+                tmem_ld32(tl + x * 256 + w * 64 + half * 32, sv);
+                tmem_ld32(tl + x * 256 + 128 + w * 64 + half * 32, dv);
+                tmem_wait_ld();
+                reg_fence32(sv);
+                reg_fence32(dv);
+                if (half == 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(BAR(L::B_SDPFREE + x));
+                }
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const int cc = half * 8 + c;
+                    const float4 bq = lds128f(brow + ((cc ^ (row & 15)) << 4));
+                    float4 mq = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (has_mask) mq = lds128f(ma + cc * 16);
+                    const float bb[4] = {bq.x + mq.x, bq.y + mq.y, bq.z + mq.z, bq.w + mq.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int xl = 4 * c + e;
+                        const float pv = ex2(fmaf(__uint_as_float(sv[xl]), c2, bb[e]) - lse2);
+                        acc[32 * half + xl] = fmaf(pv, __uint_as_float(dv[xl]) - Dj, acc[32 * half + xl]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(BAR(L::B_EMPTY + s));
+        }
+        if (ok && j < p.N) {
+            const int k0 = kt * 128 + w * 64;
+            if (p.chunks == 1) {
+                __nv_bfloat16* dst = p.dbias + b * p.dbs[0] + h * p.dbs[1] + static_cast<int64_t>(j) * p.dbs[2] + k0;
+#pragma unroll
+                for (int e = 0; e < 64; e += 8) {
+                    if (k0 + e + 8 <= p.N) {
+                        uint4 v;
+                        v.x = pack_bf16(acc[e], acc[e + 1]);
+                        v.y = pack_bf16(acc[e + 2], acc[e + 3]);
+                        v.z = pack_bf16(acc[e + 4], acc[e + 5]);
+                        v.w = pack_bf16(acc[e + 6], acc[e + 7]);
+                        *reinterpret_cast<uint4*>(dst + e) = v;
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            if (k0 + e + u < p.N) dst[e + u] = __float2bfloat16_rn(acc[e + u]);
+                    }
+                }
+            } else {
+                float* dst = p.part + (((static_cast<int64_t>(chunk) * p.B + b) * p.H + h) * p.N + j) * p.N + k0;
+#pragma unroll
+                for (int e = 0; e < 64; ++e)
+                    if (k0 + e < p.N) dst[e] = acc[e];
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ascending-chunk sum of the dBias partials -> BF16
+__global__ void __launch_bounds__(256) tri_attn_bwd_dbias_reduce_kernel(const float* __restrict__ part, int chunks,
+                                                                        int B, int H, int N,
+                                                                        __nv_bfloat16* __restrict__ dbias,
+                                                                        int64_t s0, int64_t s1, int64_t s2) {
+    const int64_t total = static_cast<int64_t>(B) * H * N * N;
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        float acc = part[idx];
+        for (int c = 1; c < chunks; ++c) acc += part[static_cast<int64_t>(c) * total + idx];
+        int64_t t = idx;
+        const int k = static_cast<int>(t % N);
+        t /= N;
+        const int j = static_cast<int>(t % N);
+        t /= N;
+        const int h = static_cast<int>(t % H);
+        const int b = static_cast<int>(t / H);
+        dbias[b * s0 + h * s1 + static_cast<int64_t>(j) * s2 + k] = __float2bfloat16_rn(acc);
+    }
+}
+
+// ===========================================================================
+// host side
+// ===========================================================================
+bool bwd_set_attributes();
+tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, float scale, uint64_t wait_ns,
+                           cudaStream_t stream);
+
+}  // namespace tri

@@ -1,0 +1,457 @@
+// fwd.cuh -- triangle-attention forward for sm_100a.
+//
+// Computes, for one batch b, head h, query tile jt (128 queries) and TWO pair
+// rows i0, i1 (one per softmax warpgroup):
+//   S = Q K^T (tcgen05, BF16 -> FP32 in TMEM), y = scale*S + bias + mask,
+//   online softmax over key tiles, O += P V (tcgen05, P from TMEM),
+//   epilogue O32 = O / l, o = bf16(O32), resid = bf16(O32 - float(o)),
+//   lse = m + log(l).
+// The page "16张H100，训练步提速1.73倍：TurboPairFormer…" (biocloudservice.com),
+// section "它优化了什么，而不是只'少存一点张量'", describes keeping the BF16
+// output-rounding residual for an FP32 softmax-backward correction; the
+// residual and the log-sum-exp are the state this kernel saves for the
+// backward.
+//
+// B200 mapping:
+//  * one CTA = 320 threads: warps 0-3 softmax for row i0, warps 4-7 softmax
+//    for row i1, warp 8 TMA producer, warp 9 MMA issuer (one thread);
+//  * both rows share every bias tile (the bias is the same for all rows i),
+//    so each 32 KB bias tile crosses L2->SMEM once per two rows;
+//  * TMEM (512 columns): per warpgroup w, S at 256w, P (BF16 pairs) at
+//    256w+128, O at 256w+192;
+//  * O is rescaled lazily: the exponent reference only moves when the row
+//    maximum grows by more than 8 (base-2 units), which keeps P <= 256 and
+//    makes the TMEM read-modify-write of O rare;
+//  * the key tail (k >= N) and the user mask arrive as one FP32 row per key
+//    tile, written by the producer warp (-inf past N); an all-zero row is
+//    flagged so the add is skipped.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace tri {
+
+struct FwdParams {
+    int B, N, H, nt, npairs;
+    float scale;
+    // positions (1..4) of the h, j, i, b coordinates in the Q/K/V tensor maps
+    int qpos_h, qpos_j, qpos_i, qpos_b;
+    // positions (1..3) of the j, h, b coordinates in the bias tensor map
+    int bpos_j, bpos_h, bpos_b;
+    const float* mask;
+    int64_t ms0, ms1, ms2;
+    __nv_bfloat16* o;
+    int64_t os[5];
+    __nv_bfloat16* r;
+    int64_t rs[5];
+    float* lse;
+    uint64_t wait_limit_ns;
+};
+
+template <int D>
+struct FwdLayout {
+    static constexpr int NS = (D == 32) ? 3 : 2;  // pipeline stages
+    static constexpr int ROWB = D * 2;            // bytes per Q/K/V row
+    static constexpr int QKV_TILE = 128 * ROWB;   // one 128-row Q/K/V tile
+    static constexpr int BIAS_TILE = 128 * 128 * 2;
+    static constexpr int OFF_K0 = 0, OFF_V0 = QKV_TILE, OFF_K1 = 2 * QKV_TILE, OFF_V1 = 3 * QKV_TILE;
+    static constexpr int OFF_BIAS = 4 * QKV_TILE;
+    static constexpr int OFF_MASK = OFF_BIAS + BIAS_TILE;  // [2][128] fp32
+    static constexpr int STAGE = OFF_MASK + 1024;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_STAGES = 2 * QKV_TILE;
+    static constexpr int OFF_BAR = OFF_STAGES + NS * STAGE;
+    // barrier indices
+    static constexpr int B_Q = 0, B_FULL = 1, B_EMPTY = 1 + NS, B_SFULL = 1 + 2 * NS,
+                         B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2, B_PVDONE = B_PFULL + 2,
+                         B_DRAIN = B_PVDONE + 2, NBAR = B_DRAIN + 1;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag, mask flags[NS][2]
+    static constexpr int SMEM = OFF_MISC + 16 + NS * 2 * 4;
+    static_assert(SMEM <= 232448, "shared memory budget");
+    static_assert(QKV_TILE % 1024 == 0 && STAGE % 1024 == 0, "1 KB tile alignment");
+};
+
+// Bounded wait used only while draining on the way out: ignores the abort flag.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > limit_ns) break;
+    }
+}
+
+__device__ __forceinline__ void reg_fence32(uint32_t (&r)[32]) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
+                   "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]),
+                   "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
+                   "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]),
+                   "+r"(r[31]));
+}
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    tri_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_bias,
+                        const FwdParams p) {
+    using L = FwdLayout<D>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t sb = smem_addr(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    auto BAR = [&](int idx) -> uint32_t { return sb + L::OFF_BAR + idx * 8; };
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+    volatile int* mask_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 16);
+
+    // ---- work item: (b, h, pair of rows, query tile), query tile fastest ----
+    int item = blockIdx.x;
+    const int jt = item % p.nt;
+    item /= p.nt;
+    const int ip = item % p.npairs;
+    item /= p.npairs;
+    const int h = item % p.H;
+    const int b = item / p.H;
+    const int i0 = 2 * ip;
+    const int i1 = min(2 * ip + 1, p.N - 1);
+    const bool has1 = (2 * ip + 1) < p.N;
+    const int nkt = p.nt;
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        if (sb & 1023u) {  // swizzled TMA tiles need 1 KB alignment
+            atomicCAS(&g_error_word, 0u, ERR_TIMEOUT_BIT | KERNEL_FWD | 0xFFu);
+            *abort_flag = 1;
+        }
+        mbar_init(BAR(L::B_Q), 1);
+        for (int s = 0; s < L::NS; ++s) {
+            mbar_init(BAR(L::B_FULL + s), 1);
+            mbar_init(BAR(L::B_EMPTY + s), 1 + 8);  // MMA commit + 8 softmax warps
+        }
+        for (int w = 0; w < 2; ++w) {
+            mbar_init(BAR(L::B_SFULL + w), 1);
+            mbar_init(BAR(L::B_SFREE + w), 4);
+            mbar_init(BAR(L::B_PFULL + w), 4);
+            mbar_init(BAR(L::B_PVDONE + w), 1);
+        }
+        mbar_init(BAR(L::B_DRAIN), 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_addr(const_cast<uint32_t*>(tmem_slot)), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const WaitCtx wc{p.wait_limit_ns, KERNEL_FWD, abort_flag};
+    const bool aborted_early = *abort_flag != 0;
+
+    if (warp == 8) {
+        // =========================== TMA producer ===========================
+        int armed[L::NS];
+#pragma unroll
+        for (int s = 0; s < L::NS; ++s) armed[s] = 0;
+        auto load_qkv = [&](uint32_t dst, const CUtensorMap* m, uint32_t bar, int i, int j0) {
+            int c[5] = {0, 0, 0, 0, 0};
+            c[p.qpos_h] = h;
+            c[p.qpos_j] = j0;
+            c[p.qpos_i] = i;
+            c[p.qpos_b] = b;
+            tma_load_5d(dst, m, bar, c[0], c[1], c[2], c[3], c[4]);
+        };
+        auto load_bias = [&](uint32_t dst, uint32_t bar, int k0, int j0) {
+            int c[4] = {0, 0, 0, 0};
+            c[0] = k0;
+            c[p.bpos_j] = j0;
+            c[p.bpos_h] = h;
+            c[p.bpos_b] = b;
+            tma_load_4d(dst, &tm_bias, bar, c[0], c[1], c[2], c[3]);
+        };
+        if (!aborted_early) {
+            if (lane == 0) {
+                tma_prefetch_map(&tm_q);
+                tma_prefetch_map(&tm_k);
+                tma_prefetch_map(&tm_v);
+                tma_prefetch_map(&tm_bias);
+                mbar_arrive_expect_tx(BAR(L::B_Q), 2 * L::QKV_TILE);
+                load_qkv(sb + L::OFF_Q, &tm_q, BAR(L::B_Q), i0, jt * 128);
+                load_qkv(sb + L::OFF_Q + L::QKV_TILE, &tm_q, BAR(L::B_Q), i1, jt * 128);
+            }
+            for (int kt = 0; kt < nkt; ++kt) {
+                const int s = kt % L::NS;
+                if (kt >= L::NS && !mbar_wait_warp(BAR(L::B_EMPTY + s), ((kt / L::NS) - 1) & 1, wc, 1)) break;
+                const uint32_t st = sb + L::OFF_STAGES + s * L::STAGE;
+                // key-mask rows (user mask, -inf past N) for both rows i0, i1
+#pragma unroll
+                for (int w = 0; w < 2; ++w) {
+                    const int i = w ? i1 : i0;
+                    float v[4];
+                    bool nz = false;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int k = kt * 128 + lane * 4 + e;
+                        float x = -INFINITY;
+                        if (k < p.N) x = p.mask ? __ldg(p.mask + b * p.ms0 + i * p.ms1 + k * p.ms2) : 0.f;
+                        v[e] = x;
+                        nz |= (x != 0.f);
+                    }
+                    float4* dst = reinterpret_cast<float4*>(smem + (st - sb) + L::OFF_MASK + w * 512 + lane * 16);
+                    *dst = make_float4(v[0], v[1], v[2], v[3]);
+                    const unsigned any = __any_sync(0xFFFFFFFFu, nz);
+                    if (lane == 0) mask_flag[s * 2 + w] = any ? 1 : 0;
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    const uint32_t bar = BAR(L::B_FULL + s);
+                    mbar_arrive_expect_tx(bar, 4 * L::QKV_TILE + L::BIAS_TILE);
+                    load_qkv(st + L::OFF_K0, &tm_k, bar, i0, kt * 128);
+                    load_qkv(st + L::OFF_V0, &tm_v, bar, i0, kt * 128);
+                    load_qkv(st + L::OFF_K1, &tm_k, bar, i1, kt * 128);
+                    load_qkv(st + L::OFF_V1, &tm_v, bar, i1, kt * 128);
+                    load_bias(st + L::OFF_BIAS, bar, kt * 128, jt * 128);
+                    load_bias(st + L::OFF_BIAS + L::BIAS_TILE / 2, bar, kt * 128 + 64, jt * 128);
+                }
+                armed[s]++;
+            }
+        }
+        // never leave with bulk copies still writing into this CTA's shared memory
+        if (lane == 0) {
+            if (!aborted_early) drain_wait(BAR(L::B_Q), 0, 100000000ull);
+#pragma unroll
+            for (int s = 0; s < L::NS; ++s)
+                if (armed[s] > 0) drain_wait(BAR(L::B_FULL + s), (armed[s] - 1) & 1, 100000000ull);
+        }
+    } else if (warp == 9) {
+        // =========================== MMA issuer =============================
+        if (lane == 0 && !aborted_early) {
+            constexpr uint32_t SW = (D == 32) ? SWZ_64B : SWZ_128B;
+            constexpr uint32_t SBO = 8 * L::ROWB;
+            constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false, false);
+            constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
+            auto issue_pv = [&](int w, uint32_t stage, int ktile) {
+                const uint32_t va = stage + (w ? L::OFF_V1 : L::OFF_V0);
+                const uint32_t tS = tmem + w * 256;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tS + 192, tS + 128 + kk * 8, smem_desc(va + kk * 16 * L::ROWB, L::QKV_TILE, SBO, SW),
+                           IDESC_PV, (ktile > 0 || kk > 0) ? 1u : 0u);
+            };
+            bool ok = mbar_wait(BAR(L::B_Q), 0, wc, 2);
+            for (int kt = 0; ok && kt < nkt; ++kt) {
+                const int s = kt % L::NS;
+                if (!mbar_wait(BAR(L::B_FULL + s), (kt / L::NS) & 1, wc, 3)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t st = sb + L::OFF_STAGES + s * L::STAGE;
+#pragma unroll
+                for (int w = 0; w < 2; ++w) {
+                    if (kt > 0) {
+                        if (!mbar_wait(BAR(L::B_SFREE + w), (kt - 1) & 1, wc, 4)) { ok = false; break; }
+                        tc_fence_after();
+                    }
+                    const uint32_t qa = sb + L::OFF_Q + w * L::QKV_TILE;
+                    const uint32_t ka = st + (w ? L::OFF_K1 : L::OFF_K0);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_ss(tmem + w * 256, smem_desc(qa + kk * 32, 16, SBO, SW),
+                               smem_desc(ka + kk * 32, 16, SBO, SW), IDESC_QK, kk > 0 ? 1u : 0u);
+                    mma_commit(BAR(L::B_SFULL + w));
+                }
+                if (!ok) break;
+                if (kt > 0) {
+                    const int sp = (kt - 1) % L::NS;
+                    const uint32_t pst = sb + L::OFF_STAGES + sp * L::STAGE;
+#pragma unroll
+                    for (int w = 0; w < 2; ++w) {
+                        if (!mbar_wait(BAR(L::B_PFULL + w), (kt - 1) & 1, wc, 5)) { ok = false; break; }
+                        tc_fence_after();
+                        issue_pv(w, pst, kt - 1);
+                        mma_commit(BAR(L::B_PVDONE + w));
+                    }
+                    if (!ok) break;
+                    mma_commit(BAR(L::B_EMPTY + sp));
+                }
+            }
+            if (ok) {
+                const int kl = nkt - 1;
+                const int sp = kl % L::NS;
+                const uint32_t pst = sb + L::OFF_STAGES + sp * L::STAGE;
+#pragma unroll
+                for (int w = 0; w < 2; ++w) {
+                    if (!mbar_wait(BAR(L::B_PFULL + w), kl & 1, wc, 5)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_pv(w, pst, kl);
+                    mma_commit(BAR(L::B_PVDONE + w));
+                }
+                if (ok) mma_commit(BAR(L::B_EMPTY + sp));
+            }
+            // every MMA this thread issued has completed before the CTA leaves
+            mma_commit(BAR(L::B_DRAIN));
+            drain_wait(BAR(L::B_DRAIN), 0, 100000000ull);
+        }
+        __syncwarp();
+    } else if (!aborted_early) {
+        // =========================== softmax warpgroups =====================
+        const int w = warp >> 2;
+        const int qd = warp & 3;
+        const int row = qd * 32 + lane;
+        const uint32_t tS = tmem + (static_cast<uint32_t>(qd * 32) << 16) + w * 256;
+        const uint32_t tP = tS + 128, tO = tS + 192;
+        const int j = jt * 128 + row;
+        const int i = w ? i1 : i0;
+        const float scale = p.scale;
+        constexpr float LOG2E = 1.4426950408889634f;
+        constexpr float RESCALE_AT = 5.545177444479562f;  // 8 * ln 2
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int kt = 0; kt < nkt; ++kt) {
+            const int s = kt % L::NS;
+            if (!mbar_wait_warp(BAR(L::B_SFULL + w), kt & 1, wc, 6)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t r0[32], r1[32], r2[32], r3[32];
+            tmem_ld32(tS + 0, r0);
+            tmem_ld32(tS + 32, r1);
+            tmem_ld32(tS + 64, r2);
+            tmem_ld32(tS + 96, r3);
+            tmem_wait_ld();
+            reg_fence32(r0);
+            reg_fence32(r1);
+            reg_fence32(r2);
+            reg_fence32(r3);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(BAR(L::B_SFREE + w));
+            if (!mbar_wait_warp(BAR(L::B_FULL + s), (kt / L::NS) & 1, wc, 7)) { ok = false; break; }
+            const uint32_t st = sb + L::OFF_STAGES + s * L::STAGE;
+            float x[128];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                x[e] = __uint_as_float(r0[e]);
+                x[32 + e] = __uint_as_float(r1[e]);
+                x[64 + e] = __uint_as_float(r2[e]);
+                x[96 + e] = __uint_as_float(r3[e]);
+            }
+            // y = scale * S + bias (+ mask)
+            const uint32_t brow = st + L::OFF_BIAS + row * 128;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const uint4 bb = lds128(brow + (c >> 3) * (L::BIAS_TILE / 2) + (((c & 7) ^ (row & 7)) << 4));
+                const int x0 = c * 8;
+                x[x0 + 0] = fmaf(x[x0 + 0], scale, bf16lo(bb.x));
+                x[x0 + 1] = fmaf(x[x0 + 1], scale, bf16hi(bb.x));
+                x[x0 + 2] = fmaf(x[x0 + 2], scale, bf16lo(bb.y));
+                x[x0 + 3] = fmaf(x[x0 + 3], scale, bf16hi(bb.y));
+                x[x0 + 4] = fmaf(x[x0 + 4], scale, bf16lo(bb.z));
+                x[x0 + 5] = fmaf(x[x0 + 5], scale, bf16hi(bb.z));
+                x[x0 + 6] = fmaf(x[x0 + 6], scale, bf16lo(bb.w));
+                x[x0 + 7] = fmaf(x[x0 + 7], scale, bf16hi(bb.w));
+            }
+            if (mask_flag[s * 2 + w]) {
+                const uint32_t ma = st + L::OFF_MASK + w * 512;
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float4 mv = lds128f(ma + c * 16);
+                    x[4 * c + 0] += mv.x;
+                    x[4 * c + 1] += mv.y;
+                    x[4 * c + 2] += mv.z;
+                    x[4 * c + 3] += mv.w;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(BAR(L::B_EMPTY + s));
+            float mt = x[0];
+#pragma unroll
+            for (int e = 1; e < 128; ++e) mt = fmaxf(mt, x[e]);
+            bool need = false;
+            float alpha = 1.f;
+            if (kt == 0) {
+                m_ref = mt;
+            } else if (mt > m_ref + RESCALE_AT) {
+                need = true;
+                alpha = ex2((m_ref - mt) * LOG2E);
+                m_ref = mt;
+                l *= alpha;
+            }
+            const float mb = fmaxf(m_ref, -3.0e38f) * LOG2E;
+            if (kt > 0) {
+                // PV of the previous tile has finished: the P columns are free and O is stable
+                if (!mbar_wait_warp(BAR(L::B_PVDONE + w), (kt - 1) & 1, wc, 8)) { ok = false; break; }
+                tc_fence_after();
+            }
+            float ls = 0.f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const float p0 = ex2(fmaf(x[32 * q + 2 * c], LOG2E, -mb));
+                    const float p1 = ex2(fmaf(x[32 * q + 2 * c + 1], LOG2E, -mb));
+                    ls += p0 + p1;
+                    pk[c] = pack_bf16(p0, p1);
+                }
+                tmem_st16(tP + 16 * q, pk);
+            }
+            l += ls;
+            if (kt > 0 && __any_sync(0xFFFFFFFFu, need)) {
+                // rare: the reference maximum moved, rescale this row of O before the next PV
+#pragma unroll 1
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + c0, o);
+                    tmem_wait_ld();
+                    reg_fence32(o);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st32(tO + c0, o);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(BAR(L::B_PFULL + w));
+        }
+        if (ok && mbar_wait_warp(BAR(L::B_PVDONE + w), (nkt - 1) & 1, wc, 9)) {
+            tc_fence_after();
+            const bool store = (j < p.N) && (w == 0 || has1);
+            const float inv_l = __frcp_rn(l);
+            __nv_bfloat16* op = p.o + b * p.os[0] + i * p.os[1] + j * p.os[2] + h * p.os[3];
+            __nv_bfloat16* rp = p.r + b * p.rs[0] + i * p.rs[1] + j * p.rs[2] + h * p.rs[3];
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t o[32];
+                tmem_ld32(tO + c0, o);
+                tmem_wait_ld();
+                reg_fence32(o);
+                if (store) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t ow[4], rw[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float a0 = __uint_as_float(o[8 * c + 2 * e]) * inv_l;
+                            const float a1 = __uint_as_float(o[8 * c + 2 * e + 1]) * inv_l;
+                            const uint32_t w16 = pack_bf16(a0, a1);
+                            ow[e] = w16;
+                            rw[e] = pack_bf16(a0 - bf16lo(w16), a1 - bf16hi(w16));
+                        }
+                        *reinterpret_cast<uint4*>(op + c0 + 8 * c) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                        *reinterpret_cast<uint4*>(rp + c0 + 8 * c) = make_uint4(rw[0], rw[1], rw[2], rw[3]);
+                    }
+                }
+            }
+            if (store) {
+                p.lse[((static_cast<int64_t>(b) * p.H + h) * p.N + i) * p.N + j] =
+                    m_ref + lg2(l) * 0.6931471805599453f;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace tri
