@@ -1,0 +1,355 @@
+#!/usr/bin/env python3
+"""Benchmark: triangle attention forward + backward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one forward (o, resid, lse) and one backward (dq, dk, dv, dbias) of
+the crop-768 training shape (B=1, N=768, H=4, d=32, BF16; q,k,v,dout ~ N(0,1),
+bias ~ 2 N(0,1), all-valid zero mask), synthetic inputs resident in HBM.  The
+metric counts 14*B*H*N^3*d flops per step (forward 4, backward 10 -- five
+GEMM-shaped products including the one recompute).  The inputs (604 MB) are
+larger than the 126 MB L2, so nothing is flushed between steps.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own replica of
+the workload (the path has no exchange step), so scaling is weak and the value
+is the flops of all ranks divided by the slowest rank's time.
+
+--impl reference times the FP64 CPU oracle (the only other implementation;
+test infrastructure) on the host cores: each step is a bounded sample of the
+same workload (a few pair rows), rank 0 only.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "tri-attn fwd+bwd TFLOP/s at N=768,H=4,d=32 BF16; % of B200 BF16 TC peak"
+WORKLOAD = "crop768 triangle attention fwd+bwd (starting node): B=1, N=768, H=4, d=32, BF16"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def flops(B, N, H, d):
+    cube = B * H * N ** 3 * d
+    return {"fwd": 4.0 * cube, "bwd": 10.0 * cube, "step": 14.0 * cube,
+            "bwd_main": 10.0 * cube, "bwd_dbias": 4.0 * cube}
+
+
+# ---------------------------------------------------------------------------
+# clock sampling during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", str(self.dev)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in out.strip().splitlines():
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from triangle_attention_biomolecular_b200 import _binding as Bd
+    from triangle_attention_biomolecular_b200 import synthetic as S
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = {"crop768": S.CROP768, "crop640": S.CROP640, "crop384": S.CROP384}[args.workload]
+    Bn, N, H, d = wl.B, wl.N, wl.H, wl.d
+    x = S.make_inputs(wl, S.seed_for(3, rank))
+    q, k, v, do, bias = (x[n].to(dev) for n in ("q", "k", "v", "dout", "bias"))
+    mask = x["mask"].to(dev)
+    o, r = torch.empty_like(q), torch.empty_like(q)
+    lse = torch.empty((Bn, H, N, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    db = torch.empty((Bn, H, N, N), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(Bd.tri_attn_bwd_workspace_bytes(Bn, N, H, d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        Bd.tri_attn_fwd(q, k, v, bias, mask, o, r, lse, 0.0, stream)
+        if ev is None:
+            Bd.tri_attn_bwd(q, k, v, bias, mask, o, r, lse, do, dq, dk, dv, db, ws, 0.0, 0, stream)
+        else:
+            Bd.tri_attn_bwd_marked(q, k, v, bias, mask, o, r, lse, do, dq, dk, dv, db, ws, ev[1:5], 0.0, 0,
+                                   stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, word = Bd.tri_attn_device_error(True)
+    if st != 0:
+        raise RuntimeError(f"device error word {word:#x} during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                           int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    st, word = Bd.tri_attn_device_error(True)
+    if st != 0:
+        raise RuntimeError(f"device error word {word:#x} during timing")
+
+    # per-kernel average durations, measured live on the launching stream
+    kern = {"fwd": [], "bwd_prep": [], "bwd_main": [], "bwd_dbias": []}
+    for e in evs:
+        kern["fwd"].append(e[0].elapsed_time(e[1]))
+        kern["bwd_prep"].append(e[1].elapsed_time(e[2]))
+        kern["bwd_main"].append(e[2].elapsed_time(e[3]))
+        kern["bwd_dbias"].append(e[3].elapsed_time(e[4]))
+    kern_ms = {n: statistics.mean(v) for n, v in kern.items()}
+
+    # end to end through the same C ABI: pinned host inputs -> device -> fwd+bwd -> host results
+    e2e = None
+    if not args.no_e2e:
+        host_in = [t.cpu().pin_memory() for t in (q, k, v, do, bias, mask)]
+        host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, dq, dk, dv, db)]
+        dev_in = [q, k, v, do, bias, mask]
+        h2d = sum(t.numel() * t.element_size() for t in host_in)
+        d2h = sum(t.numel() * t.element_size() for t in host_out)
+        n_e2e = max(1, min(args.steps, 10))
+
+        def e2e_step():
+            for h, dt in zip(host_in, dev_in):
+                dt.copy_(h, non_blocking=True)
+            step()
+            for h, dt in zip(host_out, (o, dq, dk, dv, db)):
+                h.copy_(dt, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        ems = a0.elapsed_time(a1)
+        if world > 1:
+            tt = torch.tensor([ems], dtype=torch.float64, device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ems = float(tt.item())
+        fl = flops(Bn, N, H, d)["step"]
+        e2e = {"value": round(world * fl * n_e2e / (ems * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
+               "ms_per_step": round(ems / n_e2e, 4)}
+    return {"ms": ms, "kern_ms": kern_ms, "clocks": clocks, "e2e": e2e, "shape": (Bn, N, H, d)}
+
+
+# ---------------------------------------------------------------------------
+# the oracle on host cores (CPU baseline and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(rows_n: int):
+    import numpy as np
+    from oracle import oracle as O
+    from triangle_attention_biomolecular_b200 import synthetic as S
+    wl = S.CROP768
+    x = S.make_inputs(wl, S.seed_for(3, 0))
+    f64 = lambda t: t.double().numpy()
+    q, k, v, do, bias = (f64(x[n]) for n in ("q", "k", "v", "dout", "bias"))
+    mask = x["mask"].numpy().astype(np.float64)
+    rows = [(0, (37 * r) % wl.N) for r in range(rows_n)]
+
+    def run(rs):
+        t = time.perf_counter()
+        O.fwd(q, k, v, bias, mask, rows=rs)
+        O.bwd_rows(q, k, v, bias, mask, do, rows=rs)
+        return time.perf_counter() - t
+    return wl, rows, run
+
+
+def cpu_rate(wl, nrows, seconds):
+    per_row = 14.0 * wl.H * wl.N ** 2 * wl.d  # the step's flops restricted to one pair row
+    return per_row * nrows / seconds / 1e12
+
+
+def run_cpu_baseline(target_s: float = 12.0):
+    wl, rows, run = oracle_sample(64)
+    t1 = run(rows[:1])
+    n = int(max(1, min(64, target_s / max(t1, 1e-3))))
+    t = run(rows[:n])
+    return {"value": round(cpu_rate(wl, n, t), 6), "unit": "TFLOP/s", "cores": os.cpu_count(),
+            "kind": "oracle", "seconds": round(t, 3),
+            "sample": f"{n} pair rows (all 4 heads) of the crop768 workload: FP64 oracle forward + dq/dk/dv; "
+                      f"rate counts 14*H*N^2*d flops per row"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    wl, rows, run = oracle_sample(64)
+    per_step_rows = 2
+    for s in range(args.warmup):
+        run(rows[:1])
+    times = []
+    for s in range(args.steps):
+        rr = [rows[(s * per_step_rows + e) % len(rows)] for e in range(per_step_rows)]
+        times.append(run(rr))
+    tot = sum(times)
+    val = cpu_rate(wl, per_step_rows * args.steps, tot)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * tot / max(1, args.steps), 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD + " -- each step a bounded sample of 2 pair rows"},
+        "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": f"{per_step_rows} pair rows per step (all 4 heads), FP64 oracle fwd + dq/dk/dv"},
+        "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=("crop768", "crop640", "crop384"), default="crop768",
+                    help="crop768 is the headline; the smaller crops serve profiler captures")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle on host cores")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    if rank != 0:
+        return
+    Bn, N, H, d = res["shape"]
+    fl = flops(Bn, N, H, d)
+    pk, src = peaks()
+    peak = float(pk["bf16_tflops"])
+    ms = res["ms"]
+    per_step_ms = ms / args.steps
+    value = world * fl["step"] * args.steps / (ms * 1e-3) / 1e12
+    km = res["kern_ms"]
+    algo = {"fwd": fl["fwd"], "bwd_main": fl["bwd_main"], "bwd_dbias": fl["bwd_dbias"]}
+    dom = max(algo, key=lambda n: km[n])
+    achieved = algo[dom] / (km[dom] * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(per_step_ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD if args.workload == "crop768" else args.workload, "B": Bn, "N": N, "H": H, "d": d, "bias": "2*N(0,1)", "mask": "zeros",
+                   "flops_per_step": fl["step"], "l2": "inputs (604 MB) larger than the 126 MB L2; no flush"},
+        "pct_of_bf16_peak": round(100.0 * value / world / peak, 2),
+        "pct_of_bf16_peak_sustained": round(100.0 * value / world / float(pk["bf16_tflops_sustained"]), 2),
+        "kernels_ms": {n: round(v, 4) for n, v in km.items()},
+        "fwd_tflops": round(fl["fwd"] / (km["fwd"] * 1e-3) / 1e12, 2),
+        "bwd_tflops": round(fl["bwd"] / ((km["bwd_prep"] + km["bwd_main"] + km["bwd_dbias"]) * 1e-3) / 1e12, 2),
+        "roofline": {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": f"{src} bf16_tflops (burst)"},
+        "gpu_launches": 4 * args.steps,
+        "clocks": res["clocks"],
+        "e2e": res["e2e"],
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = run_cpu_baseline()
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

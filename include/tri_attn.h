@@ -157,13 +157,23 @@ size_t tri_attn_bwd_workspace_bytes(int B, int N, int H, int d);
  * tri_attn_fwd, plus TRI_ATTN_ERR_WORKSPACE. */
 tri_attn_status tri_attn_bwd(const tri_attn_bwd_args *args, tri_attn_stream_t stream);
 
+/* tri_attn_bwd with timing markers: `markers` is NULL or an array of four
+ * cudaEvent_t handles (as void*) that are recorded on `stream` before the
+ * D pre-pass, before the dq/dk/dv kernel, before the dbias kernel(s) and
+ * after the last kernel, so a caller can time each phase with the events it
+ * owns.  Otherwise identical to tri_attn_bwd. */
+tri_attn_status tri_attn_bwd_marked(const tri_attn_bwd_args *args, tri_attn_stream_t stream,
+                                    void *const *markers);
+
 /* Static, NUL-terminated description of a status code. */
 const char *tri_attn_strerror(tri_attn_status status);
 
 /* Reads (and, if clear != 0, resets) the library's device error word on the
  * current device.  Every spin-wait inside the kernels is bounded; a wait that
  * expires records its site there and the kernel returns early instead of
- * hanging.  Synchronises the device.  Returns TRI_ATTN_OK,
+ * hanging.  While the word is set, every later launch of the library's
+ * kernels returns at once without computing (outputs untouched), until the
+ * word is cleared here.  Synchronises the device.  Returns TRI_ATTN_OK,
  * TRI_ATTN_ERR_DEVICE_TIMEOUT (and stores the raw word in *word if non-NULL),
  * or TRI_ATTN_ERR_CUDA. */
 tri_attn_status tri_attn_device_error(int clear, uint32_t *word);

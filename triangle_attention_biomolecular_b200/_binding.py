@@ -79,6 +79,9 @@ def load() -> ctypes.CDLL:
             lib.tri_attn_fwd.restype = ctypes.c_int
             lib.tri_attn_bwd.argtypes = [ctypes.POINTER(BwdArgs), ctypes.c_void_p]
             lib.tri_attn_bwd.restype = ctypes.c_int
+            lib.tri_attn_bwd_marked.argtypes = [ctypes.POINTER(BwdArgs), ctypes.c_void_p,
+                                                ctypes.POINTER(ctypes.c_void_p)]
+            lib.tri_attn_bwd_marked.restype = ctypes.c_int
             lib.tri_attn_bwd_workspace_bytes.argtypes = [ctypes.c_int] * 4
             lib.tri_attn_bwd_workspace_bytes.restype = ctypes.c_size_t
             lib.tri_attn_strerror.argtypes = [ctypes.c_int]
@@ -201,10 +204,8 @@ def tri_attn_fwd(q, k, v, bias, mask, o, resid, lse, scale: float = 0.0, stream=
         raise TriAttnError(st, "tri_attn_fwd")
 
 
-def tri_attn_bwd(q, k, v, bias, mask, o, resid, lse, dout, dq, dk, dv, dbias, workspace,
-                 scale: float = 0.0, flags: int = 0, stream=None) -> None:
-    """Enqueue the backward; dq, dk, dv, dbias (BF16) are written.  workspace is a
-    caller-owned uint8 CUDA tensor of at least tri_attn_bwd_workspace_bytes bytes."""
+def bwd_args(q, k, v, bias, mask, o, resid, lse, dout, dq, dk, dv, dbias, workspace,
+             scale: float = 0.0, flags: int = 0) -> BwdArgs:
     import torch
     a = BwdArgs()
     a.f = fwd_args(q, k, v, bias, mask, o, resid, lse, scale)
@@ -218,9 +219,28 @@ def tri_attn_bwd(q, k, v, bias, mask, o, resid, lse, dout, dq, dk, dv, dbias, wo
             raise TriAttnError(TRI_ATTN_ERR_DTYPE, "workspace must be a uint8 tensor")
         a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel()
     a.flags = int(flags)
+    return a
+
+
+def tri_attn_bwd(q, k, v, bias, mask, o, resid, lse, dout, dq, dk, dv, dbias, workspace,
+                 scale: float = 0.0, flags: int = 0, stream=None) -> None:
+    """Enqueue the backward; dq, dk, dv, dbias (BF16) are written.  workspace is a
+    caller-owned uint8 CUDA tensor of at least tri_attn_bwd_workspace_bytes bytes."""
+    a = bwd_args(q, k, v, bias, mask, o, resid, lse, dout, dq, dk, dv, dbias, workspace, scale, flags)
     st = load().tri_attn_bwd(ctypes.byref(a), _stream_handle(stream))
     if st != TRI_ATTN_OK:
         raise TriAttnError(st, "tri_attn_bwd")
+
+
+def tri_attn_bwd_marked(q, k, v, bias, mask, o, resid, lse, dout, dq, dk, dv, dbias, workspace,
+                        markers, scale: float = 0.0, flags: int = 0, stream=None) -> None:
+    """tri_attn_bwd recording four caller-owned torch.cuda.Event markers between
+    its phases (D pre-pass | dq/dk/dv | dbias | end)."""
+    a = bwd_args(q, k, v, bias, mask, o, resid, lse, dout, dq, dk, dv, dbias, workspace, scale, flags)
+    arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(int(ev.cuda_event)) for ev in markers])
+    st = load().tri_attn_bwd_marked(ctypes.byref(a), _stream_handle(stream), arr)
+    if st != TRI_ATTN_OK:
+        raise TriAttnError(st, "tri_attn_bwd_marked")
 
 
 def tri_attn_device_error(clear: bool = True):

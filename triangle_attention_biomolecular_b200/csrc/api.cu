@@ -218,7 +218,10 @@ bool bwd_set_attributes() {
 }
 
 tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, float scale, uint64_t wait_ns,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, void* const* markers) {
+    auto mark = [&](int m) {
+        if (markers && markers[m]) cudaEventRecord(static_cast<cudaEvent_t>(markers[m]), stream);
+    };
     const tri_attn_fwd_args& f = a->f;
     const int B = f.B, N = f.N, H = f.H, d = f.d;
     CUtensorMap mq, mk, mv, mdo, mb;
@@ -257,12 +260,15 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, f
     const unsigned db_grid = static_cast<unsigned>(B) * H * p.nt * p.nt * ws.chunks;
     const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(f.bias.ptr);
     const auto& so = f.o.stride; const auto& sr = f.resid.stride; const auto& sd = a->dout.stride;
+    mark(0);
     if (d == 32) {
         tri_attn_bwd_prep_kernel<32><<<prep_grid, 256, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(a->dout.ptr), sd[0], sd[1], sd[2], sd[3],
             static_cast<const __nv_bfloat16*>(f.o.ptr), so[0], so[1], so[2], so[3],
             static_cast<const __nv_bfloat16*>(f.resid.ptr), sr[0], sr[1], sr[2], sr[3], use_resid, p.Dv, B, N, H);
+        mark(1);
         tri_attn_bwd_main_kernel<32><<<ws.grid_main, 320, MainLayout<32>::SMEM, stream>>>(mq, mk, mv, mdo, mb, p);
+        mark(2);
         tri_attn_bwd_dbias_kernel<32><<<db_grid, 320, DbLayout<32>::SMEM, stream>>>(
             mq, mk, mv, mdo, bias, f.bias.stride[0], f.bias.stride[1], f.bias.stride[2], p);
     } else {
@@ -270,7 +276,9 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, f
             static_cast<const __nv_bfloat16*>(a->dout.ptr), sd[0], sd[1], sd[2], sd[3],
             static_cast<const __nv_bfloat16*>(f.o.ptr), so[0], so[1], so[2], so[3],
             static_cast<const __nv_bfloat16*>(f.resid.ptr), sr[0], sr[1], sr[2], sr[3], use_resid, p.Dv, B, N, H);
+        mark(1);
         tri_attn_bwd_main_kernel<64><<<ws.grid_main, 320, MainLayout<64>::SMEM, stream>>>(mq, mk, mv, mdo, mb, p);
+        mark(2);
         tri_attn_bwd_dbias_kernel<64><<<db_grid, 320, DbLayout<64>::SMEM, stream>>>(
             mq, mk, mv, mdo, bias, f.bias.stride[0], f.bias.stride[1], f.bias.stride[2], p);
     }
@@ -280,6 +288,7 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, f
                                                                   a->dbias.stride[0], a->dbias.stride[1],
                                                                   a->dbias.stride[2]);
     }
+    mark(3);
     return cudaGetLastError() == cudaSuccess ? TRI_ATTN_OK : TRI_ATTN_ERR_CUDA;
 }
 
@@ -351,6 +360,10 @@ size_t tri_attn_bwd_workspace_bytes(int B, int N, int H, int d) {
 }
 
 tri_attn_status tri_attn_bwd(const tri_attn_bwd_args* a, tri_attn_stream_t stream) {
+    return tri_attn_bwd_marked(a, stream, nullptr);
+}
+
+tri_attn_status tri_attn_bwd_marked(const tri_attn_bwd_args* a, tri_attn_stream_t stream, void* const* markers) {
     if (!a) return TRI_ATTN_ERR_NULL;
     tri_attn_status st = check_fwd_args(&a->f);
     if (st) return st;
@@ -364,7 +377,7 @@ tri_attn_status tri_attn_bwd(const tri_attn_bwd_args* a, tri_attn_stream_t strea
     if (reinterpret_cast<uintptr_t>(a->workspace) & 255u) return TRI_ATTN_ERR_ALIGN;
     if ((st = ensure_device())) return st;
     return tri::bwd_launch(a, ws, eff_scale(a->f.scale, d), g_wait_limit_ns.load(),
-                           reinterpret_cast<cudaStream_t>(stream));
+                           reinterpret_cast<cudaStream_t>(stream), markers);
 }
 
 tri_attn_status tri_attn_device_error(int clear, uint32_t* word) {

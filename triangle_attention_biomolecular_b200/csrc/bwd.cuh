@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(320, 1)
     };
 
     if (threadIdx.x == 0) {
-        *abort_flag = 0;
+        *abort_flag = device_error_pending() ? 1 : 0;
         if (sb & 1023u) {
             atomicCAS(&g_error_word, 0u, ERR_TIMEOUT_BIT | KERNEL_BWD_MAIN | 0xFFu);
             *abort_flag = 1;
@@ -680,7 +680,7 @@ __global__ void __launch_bounds__(320, 1)
     const int nrows = max(0, i_end - i_begin);
 
     if (threadIdx.x == 0) {
-        *abort_flag = 0;
+        *abort_flag = device_error_pending() ? 1 : 0;
         if (sb & 1023u) {
             atomicCAS(&g_error_word, 0u, ERR_TIMEOUT_BIT | KERNEL_BWD_DBIAS | 0xFFu);
             *abort_flag = 1;
@@ -927,6 +927,6 @@ __global__ void __launch_bounds__(256) tri_attn_bwd_dbias_reduce_kernel(const fl
 // ===========================================================================
 bool bwd_set_attributes();
 tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, float scale, uint64_t wait_ns,
-                           cudaStream_t stream);
+                           cudaStream_t stream, void* const* markers);
 
 }  // namespace tri

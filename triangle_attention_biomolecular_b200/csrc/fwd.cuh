@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(320, 1)
     const int nkt = p.nt;
 
     if (threadIdx.x == 0) {
-        *abort_flag = 0;
+        *abort_flag = device_error_pending() ? 1 : 0;
         if (sb & 1023u) {  // swizzled TMA tiles need 1 KB alignment
             atomicCAS(&g_error_word, 0u, ERR_TIMEOUT_BIT | KERNEL_FWD | 0xFFu);
             *abort_flag = 1;

@@ -64,6 +64,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// True if an earlier wait (this launch or an earlier one not yet cleared by
+// the host) expired; kernels then return at once without computing.
+__device__ __forceinline__ bool device_error_pending() {
+    return *reinterpret_cast<volatile uint32_t*>(&g_error_word) != 0u;
+}
+
 // Per-CTA wait context: the bound, the site tag and the CTA's abort flag.
 struct WaitCtx {
     uint64_t limit_ns;
@@ -83,6 +89,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
         for (int r = 0; r < 32; ++r)
             if (mbar_try_wait(bar, parity)) return true;
         if (*w.abort_flag) return false;
+        if (*reinterpret_cast<volatile uint32_t*>(&g_error_word) != 0u) {  // another CTA gave up
+            *w.abort_flag = 1;
+            return false;
+        }
         if (global_timer_ns() - t0 > w.limit_ns) {
             atomicCAS(&g_error_word, 0u, ERR_TIMEOUT_BIT | w.kernel | site);
             *w.abort_flag = 1;
