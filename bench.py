@@ -145,6 +145,9 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device error word {word:#x} during warm-up")
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    for e in evs:  # torch creates an event on its first record; the library re-records these handles
+        for ev in e:
+            ev.record(stream)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
                            int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))

@@ -30,10 +30,15 @@ def rel(a, b):
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
 
 
-def run_gpu(x, orientation, flags=0):
+def run_gpu(x, orientation, flags=0, bias_row_pad=None):
     dev = torch.device("cuda")
     q, k, v, do = (S.to_attention_frame(x[n].to(dev), orientation) for n in ("q", "k", "v", "dout"))
     bias = x["bias"].to(dev)
+    if bias_row_pad is not None:  # same values, rows padded on the device (row stride bias_row_pad)
+        N = bias.shape[-1]
+        buf = torch.zeros(bias.shape[:-1] + (bias_row_pad,), dtype=bias.dtype, device=dev)
+        buf[..., :N] = bias
+        bias = buf[..., :N]
     mask = x["mask"].to(dev) if x["mask"] is not None else None
     o, r, lse = api.forward(q, k, v, bias, mask)
     dq, dk, dv, db = api.backward(q, k, v, bias, mask, o, r, lse, do, flags=flags)
@@ -124,10 +129,7 @@ def test_odd_N_with_padded_bias_rows():
     # bias lives in a [.., N, 40] buffer so its row stride stays 16-byte aligned
     wl = S.Workload("odd", 1, 37, 2, 32, mask="ragged", len_lo=20, len_hi=37)
     x = S.make_inputs(wl, 5)
-    pad = torch.zeros(1, 2, 37, 40, dtype=torch.bfloat16)
-    pad[..., :37] = x["bias"]
-    x["bias"] = pad[..., :37]
-    check_full(x, run_gpu(x, "start"))
+    check_full(x, run_gpu(x, "start", bias_row_pad=40))
 
 
 def test_ending_node_full():

@@ -47,7 +47,9 @@ def backward(q, k, v, bias, mask, o, resid, lse, dout, scale: Optional[float] = 
     """Attention-frame backward.  Returns (dq, dk, dv, dbias)."""
     Bn, N, _, H, d = q.shape
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    dbias = torch.empty((Bn, H, N, N), dtype=torch.bfloat16, device=q.device)
+    # rows padded to a multiple of 8 elements (the ABI wants 16-byte aligned row strides)
+    Npad = (N + 7) // 8 * 8
+    dbias = torch.empty((Bn, H, N, Npad), dtype=torch.bfloat16, device=q.device)[..., :N]
     need = B.tri_attn_bwd_workspace_bytes(Bn, N, H, d)
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)

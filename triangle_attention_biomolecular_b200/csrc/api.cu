@@ -12,6 +12,8 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -168,6 +170,16 @@ bool encode_map(CUtensorMap* m, void* ptr, uint64_t inner, uint32_t inner_box, O
     CUresult r = encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 1 + nouter, ptr, dims, strides, box, estr,
                            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS && std::getenv("TRI_ATTN_DEBUG")) {
+        std::fprintf(stderr, "tri_attn: tensor-map encode failed (CUresult %d): rank %d ptr %p dims", static_cast<int>(r),
+                     1 + nouter, ptr);
+        for (int a = 0; a <= nouter; ++a) std::fprintf(stderr, " %llu", static_cast<unsigned long long>(dims[a]));
+        std::fprintf(stderr, " strides");
+        for (int a = 0; a < nouter; ++a) std::fprintf(stderr, " %llu", static_cast<unsigned long long>(strides[a]));
+        std::fprintf(stderr, " box");
+        for (int a = 0; a <= nouter; ++a) std::fprintf(stderr, " %u", box[a]);
+        std::fprintf(stderr, " swizzle %d\n", static_cast<int>(swz));
+    }
     return r == CUDA_SUCCESS;
 }
 
@@ -236,13 +248,16 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, f
     BwdParams p{};
     p.B = B; p.N = N; p.H = H;
     p.nt = (N + 127) / 128;
+    p.Np = ws.Np;
+    p.dq_tmem = (256 + 2 * d + p.nt * d <= 512) ? 1 : 0;
     p.scale = scale;
     p.qpos_h = pq[0]; p.qpos_j = pq[1]; p.qpos_i = pq[2]; p.qpos_b = pq[3];
     p.bpos_j = pb[0]; p.bpos_h = pb[1]; p.bpos_b = pb[2];
-    p.mask = f.mask.ptr;
-    p.ms0 = f.mask.stride[0]; p.ms1 = f.mask.stride[1]; p.ms2 = f.mask.stride[2];
-    p.lse = f.lse;
-    p.Dv = reinterpret_cast<float*>(wsb + ws.off_D);
+    float* Dv = reinterpret_cast<float*>(wsb + ws.off_D);
+    float* Lv = reinterpret_cast<float*>(wsb + ws.off_L);
+    float* Mv = reinterpret_cast<float*>(wsb + ws.off_M);
+    int* Fv = reinterpret_cast<int*>(wsb + ws.off_F);
+    p.Dv = Dv; p.Lv = Lv; p.Mv = Mv; p.Fv = Fv;
     p.dq_slots = reinterpret_cast<float*>(wsb + ws.off_dq);
     p.part = reinterpret_cast<float*>(wsb + ws.off_part);
     p.chunks = ws.chunks;
@@ -255,7 +270,10 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, f
     p.wait_limit_ns = wait_ns;
 
     const int64_t rows = static_cast<int64_t>(B) * H * N * N;
-    const unsigned prep_grid = static_cast<unsigned>(std::min<int64_t>((rows + 255) / 256, 148 * 16));
+    const int64_t prep_items = static_cast<int64_t>(B) * H * N * ws.Np + static_cast<int64_t>(B) * N * ws.Np +
+                               static_cast<int64_t>(B) * N * 32;
+    const unsigned prep_grid = static_cast<unsigned>(std::min<int64_t>((prep_items + 255) / 256, 148 * 16));
+    const auto& sm = f.mask.stride;
     const int use_resid = (a->flags & TRI_ATTN_BWD_NO_RESIDUAL) ? 0 : 1;
     const unsigned db_grid = static_cast<unsigned>(B) * H * p.nt * p.nt * ws.chunks;
     const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(f.bias.ptr);
@@ -265,21 +283,23 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, f
         tri_attn_bwd_prep_kernel<32><<<prep_grid, 256, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(a->dout.ptr), sd[0], sd[1], sd[2], sd[3],
             static_cast<const __nv_bfloat16*>(f.o.ptr), so[0], so[1], so[2], so[3],
-            static_cast<const __nv_bfloat16*>(f.resid.ptr), sr[0], sr[1], sr[2], sr[3], use_resid, p.Dv, B, N, H);
+            static_cast<const __nv_bfloat16*>(f.resid.ptr), sr[0], sr[1], sr[2], sr[3], use_resid, f.lse, f.mask.ptr,
+            sm[0], sm[1], sm[2], Dv, Lv, Mv, Fv, B, N, H, ws.Np, p.nt);
         mark(1);
-        tri_attn_bwd_main_kernel<32><<<ws.grid_main, 320, MainLayout<32>::SMEM, stream>>>(mq, mk, mv, mdo, mb, p);
+        tri_attn_bwd_main_kernel<32><<<ws.grid_main, 384, MainLayout<32>::SMEM, stream>>>(mq, mk, mv, mdo, mb, p);
         mark(2);
-        tri_attn_bwd_dbias_kernel<32><<<db_grid, 320, DbLayout<32>::SMEM, stream>>>(
+        tri_attn_bwd_dbias_kernel<32><<<db_grid, 384, DbLayout<32>::SMEM, stream>>>(
             mq, mk, mv, mdo, bias, f.bias.stride[0], f.bias.stride[1], f.bias.stride[2], p);
     } else {
         tri_attn_bwd_prep_kernel<64><<<prep_grid, 256, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(a->dout.ptr), sd[0], sd[1], sd[2], sd[3],
             static_cast<const __nv_bfloat16*>(f.o.ptr), so[0], so[1], so[2], so[3],
-            static_cast<const __nv_bfloat16*>(f.resid.ptr), sr[0], sr[1], sr[2], sr[3], use_resid, p.Dv, B, N, H);
+            static_cast<const __nv_bfloat16*>(f.resid.ptr), sr[0], sr[1], sr[2], sr[3], use_resid, f.lse, f.mask.ptr,
+            sm[0], sm[1], sm[2], Dv, Lv, Mv, Fv, B, N, H, ws.Np, p.nt);
         mark(1);
-        tri_attn_bwd_main_kernel<64><<<ws.grid_main, 320, MainLayout<64>::SMEM, stream>>>(mq, mk, mv, mdo, mb, p);
+        tri_attn_bwd_main_kernel<64><<<ws.grid_main, 384, MainLayout<64>::SMEM, stream>>>(mq, mk, mv, mdo, mb, p);
         mark(2);
-        tri_attn_bwd_dbias_kernel<64><<<db_grid, 320, DbLayout<64>::SMEM, stream>>>(
+        tri_attn_bwd_dbias_kernel<64><<<db_grid, 384, DbLayout<64>::SMEM, stream>>>(
             mq, mk, mv, mdo, bias, f.bias.stride[0], f.bias.stride[1], f.bias.stride[2], p);
     }
     if (ws.chunks > 1) {
@@ -348,9 +368,9 @@ tri_attn_status tri_attn_fwd(const tri_attn_fwd_args* a, tri_attn_stream_t strea
     const unsigned grid = static_cast<unsigned>(B) * p.npairs * H * p.nt;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (d == 32)
-        tri::tri_attn_fwd_kernel<32><<<grid, 320, tri::FwdLayout<32>::SMEM, s>>>(mq, mk, mv, mb, p);
+        tri::tri_attn_fwd_kernel<32><<<grid, 384, tri::FwdLayout<32>::SMEM, s>>>(mq, mk, mv, mb, p);
     else
-        tri::tri_attn_fwd_kernel<64><<<grid, 320, tri::FwdLayout<64>::SMEM, s>>>(mq, mk, mv, mb, p);
+        tri::tri_attn_fwd_kernel<64><<<grid, 384, tri::FwdLayout<64>::SMEM, s>>>(mq, mk, mv, mb, p);
     return cudaGetLastError() == cudaSuccess ? TRI_ATTN_OK : TRI_ATTN_ERR_CUDA;
 }
 

@@ -30,6 +30,8 @@
 // repeatable and independent of the SM count.
 #pragma once
 
+#include <type_traits>
+
 #include "../../include/tri_attn.h"
 #include "sm100.cuh"
 #include "fwd.cuh"
@@ -40,9 +42,10 @@ constexpr int kDqSlots = 148;   // persistent CTAs of the main kernel (B200 SM c
 constexpr int kChunkTarget = 148;
 
 struct BwdWorkspace {
-    size_t off_D, off_dq, off_part, total;
+    size_t off_D, off_L, off_M, off_F, off_dq, off_part, total;
     int chunks;     // row chunks of the dBias kernel
     int grid_main;  // CTAs of the main kernel
+    int Np;         // N rounded up to whole 128-wide tiles
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -59,27 +62,34 @@ inline BwdWorkspace bwd_workspace_layout(int B, int N, int H, int d) {
         chunks = chunks > max_chunks ? max_chunks : chunks;
     }
     w.chunks = chunks;
+    w.Np = static_cast<int>(nt * 128);
     const size_t problems = static_cast<size_t>(B) * N * H;
     w.grid_main = static_cast<int>(problems < static_cast<size_t>(kDqSlots) ? problems : kDqSlots);
-    const size_t bhnn = static_cast<size_t>(B) * H * N * N;
+    const size_t bhnp = static_cast<size_t>(B) * H * N * w.Np;
+    const size_t bnp = static_cast<size_t>(B) * N * w.Np;
     w.off_D = 0;
-    w.off_dq = align256(bhnn * 4);
+    w.off_L = align256(bhnp * 4);
+    w.off_M = w.off_L + align256(bhnp * 4);
+    w.off_F = w.off_M + align256(bnp * 4);
+    w.off_dq = w.off_F + align256(static_cast<size_t>(B) * N * 32 * 4);
     w.off_part = w.off_dq + align256(static_cast<size_t>(kDqSlots) * N * d * 4);
+    const size_t bhnn = static_cast<size_t>(B) * H * N * N;
     w.total = w.off_part + (chunks > 1 ? align256(static_cast<size_t>(chunks) * bhnn * 4) : 0);
     return w;
 }
 
 struct BwdParams {
-    int B, N, H, nt;
+    int B, N, H, nt, Np;
     float scale;
     int qpos_h, qpos_j, qpos_i, qpos_b;  // tensor-map coordinate positions (pair tensors)
     int bpos_j, bpos_h, bpos_b;          // bias tensor map
-    const float* mask;
-    int64_t ms0, ms1, ms2;
-    const float* lse;  // [B,H,N,N]
-    float* Dv;         // [B,H,N,N] workspace
-    float* dq_slots;   // [kDqSlots][N][d]
-    float* part;       // [chunks][B,H,N,N] (chunks > 1)
+    const float* Lv;  // [B,H,N,Np] lse * log2(e); +inf past N
+    const float* Dv;  // [B,H,N,Np] D; 0 past N
+    const float* Mv;  // [B,N,Np]   mask * log2(e); -inf past N
+    const int* Fv;    // [B,N,32]   1 where a key tile needs the mask add
+    float* dq_slots;  // [kDqSlots][N][d] (used when dq_tmem == 0)
+    int dq_tmem;      // 1: dQ for every query tile stays in TMEM across key tiles
+    float* part;      // [chunks][B,H,N,N] (chunks > 1)
     int chunks;
     __nv_bfloat16 *dq, *dk, *dv, *dbias;
     int64_t dqs[5], dks[5], dvs[5], dbs[4];
@@ -87,42 +97,82 @@ struct BwdParams {
 };
 
 // ===========================================================================
-// 1. D = rowsum(dout * (o + resid))
+// 1. pre-pass: the per-row vectors both backward kernels stream, laid out so
+//    that every 128-wide tile is one aligned 512-byte bulk copy:
+//      D  = rowsum(dout * (o + resid))  (FP32; the residual restores what BF16
+//           rounding of the output dropped), 0 past N
+//      L  = lse * log2(e), +inf past N (so padded query rows get P = 0)
+//      M  = mask * log2(e) (0 without a mask), -inf past N (padded keys)
+//      F  = per (b, i, key tile): 1 if that tile needs the mask add at all
 // ===========================================================================
 template <int D>
 __global__ void __launch_bounds__(256) tri_attn_bwd_prep_kernel(
     const __nv_bfloat16* __restrict__ dout, int64_t s0, int64_t s1, int64_t s2, int64_t s3,
     const __nv_bfloat16* __restrict__ o, int64_t o0, int64_t o1, int64_t o2, int64_t o3,
     const __nv_bfloat16* __restrict__ r, int64_t r0, int64_t r1, int64_t r2, int64_t r3, int use_resid,
-    float* __restrict__ Dout, int B, int N, int H) {
-    const int64_t total = static_cast<int64_t>(B) * H * N * N;
-    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+    const float* __restrict__ lse, const float* __restrict__ mask, int64_t m0, int64_t m1, int64_t m2,
+    float* __restrict__ Dv, float* __restrict__ Lv, float* __restrict__ Mv, int* __restrict__ Fv, int B, int N,
+    int H, int Np, int nt) {
+    constexpr float LOG2E = 1.4426950408889634f;
+    const int64_t n1 = static_cast<int64_t>(B) * H * N * Np;
+    const int64_t n2 = static_cast<int64_t>(B) * N * Np;
+    const int64_t n3 = static_cast<int64_t>(B) * N * 32;
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < n1 + n2 + n3;
          idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        int64_t t = idx;
-        const int j = static_cast<int>(t % N);
-        t /= N;
-        const int i = static_cast<int>(t % N);
-        t /= N;
-        const int h = static_cast<int>(t % H);
-        const int b = static_cast<int>(t / H);
-        const uint4* pd = reinterpret_cast<const uint4*>(dout + b * s0 + i * s1 + j * s2 + h * s3);
-        const uint4* po = reinterpret_cast<const uint4*>(o + b * o0 + i * o1 + j * o2 + h * o3);
-        const uint4* pr = reinterpret_cast<const uint4*>(r + b * r0 + i * r1 + j * r2 + h * r3);
-        float acc = 0.f;
+        if (idx < n1) {
+            int64_t t = idx;
+            const int j = static_cast<int>(t % Np);
+            t /= Np;
+            const int i = static_cast<int>(t % N);
+            t /= N;
+            const int h = static_cast<int>(t % H);
+            const int b = static_cast<int>(t / H);
+            float dsum = 0.f, lv = INFINITY;
+            if (j < N) {
+                const uint4* pd = reinterpret_cast<const uint4*>(dout + b * s0 + i * s1 + j * s2 + h * s3);
+                const uint4* po = reinterpret_cast<const uint4*>(o + b * o0 + i * o1 + j * o2 + h * o3);
+                const uint4* pr = reinterpret_cast<const uint4*>(r + b * r0 + i * r1 + j * r2 + h * r3);
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-            const uint4 a = __ldg(pd + c), bo = __ldg(po + c);
-            uint4 br = make_uint4(0, 0, 0, 0);
-            if (use_resid) br = __ldg(pr + c);
-            const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, ow[4] = {bo.x, bo.y, bo.z, bo.w},
-                           rw[4] = {br.x, br.y, br.z, br.w};
+                for (int c = 0; c < D / 8; ++c) {
+                    const uint4 a = __ldg(pd + c), bo = __ldg(po + c);
+                    uint4 br = make_uint4(0, 0, 0, 0);
+                    if (use_resid) br = __ldg(pr + c);
+                    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, ow[4] = {bo.x, bo.y, bo.z, bo.w},
+                                   rw[4] = {br.x, br.y, br.z, br.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                acc = fmaf(bf16lo(aw[e]), bf16lo(ow[e]) + bf16lo(rw[e]), acc);
-                acc = fmaf(bf16hi(aw[e]), bf16hi(ow[e]) + bf16hi(rw[e]), acc);
+                    for (int e = 0; e < 4; ++e) {
+                        dsum = fmaf(bf16lo(aw[e]), bf16lo(ow[e]) + bf16lo(rw[e]), dsum);
+                        dsum = fmaf(bf16hi(aw[e]), bf16hi(ow[e]) + bf16hi(rw[e]), dsum);
+                    }
+                }
+                lv = __ldg(lse + ((static_cast<int64_t>(b) * H + h) * N + i) * N + j) * LOG2E;
             }
+            Dv[idx] = dsum;
+            Lv[idx] = lv;
+        } else if (idx < n1 + n2) {
+            const int64_t e = idx - n1;
+            const int k = static_cast<int>(e % Np);
+            const int64_t t = e / Np;
+            const int i = static_cast<int>(t % N);
+            const int b = static_cast<int>(t / N);
+            float mv = -INFINITY;
+            if (k < N) mv = mask ? __ldg(mask + b * m0 + i * m1 + k * m2) * LOG2E : 0.f;
+            Mv[e] = mv;
+        } else {
+            const int64_t e = idx - n1 - n2;
+            const int kt = static_cast<int>(e % 32);
+            const int64_t t = e / 32;
+            const int i = static_cast<int>(t % N);
+            const int b = static_cast<int>(t / N);
+            int f = 0;
+            if (kt < nt) {
+                if ((kt + 1) * 128 > N) f = 1;  // padded keys need the -inf
+                if (mask && !f)
+                    for (int k = kt * 128; k < (kt + 1) * 128; ++k)
+                        if (__ldg(mask + b * m0 + i * m1 + k * m2) != 0.f) { f = 1; break; }
+            }
+            Fv[e] = f;
         }
-        Dout[idx] = acc;
     }
 }
 
@@ -143,24 +193,26 @@ struct MainLayout {
     static constexpr int T_STAGE = 2 * QKV_TILE + BIAS_TILE;
     static constexpr int OFF_P = OFF_T + NS * T_STAGE;
     static constexpr int OFF_DS = OFF_P + PT_TILE;
-    // vectors
-    static constexpr int OFF_MASKV = OFF_DS + PT_TILE;      // [KVS][128] fp32
-    static constexpr int OFF_VEC = OFF_MASKV + KVS * 512;   // [NS][lse2 128, D 128] fp32
+    // vectors (bulk-copied from the pre-pass arrays)
+    static constexpr int OFF_MASKV = OFF_DS + PT_TILE;      // [KVS][128] fp32 mask*log2(e)
+    static constexpr int OFF_FLAGS = OFF_MASKV + KVS * 512; // [KVS][32] int: key tile needs the mask add
+    static constexpr int OFF_VEC = OFF_FLAGS + KVS * 128;   // [NS][lse*log2(e) 128, D 128] fp32
     static constexpr int OFF_BAR = OFF_VEC + NS * 1024;
     static constexpr int B_KVFULL = 0, B_KVEMPTY = KVS, B_TFULL = 2 * KVS, B_TEMPTY = 2 * KVS + NS,
                          B_SDPFULL = 2 * KVS + 2 * NS, B_SDPFREE = B_SDPFULL + 1, B_PDSFULL = B_SDPFULL + 2,
                          B_PDSFREE = B_SDPFULL + 3, B_DQFULL = B_SDPFULL + 4, B_DQFREE = B_SDPFULL + 5,
                          B_DKVFULL = B_SDPFULL + 6, B_DKVFREE = B_SDPFULL + 7, B_DRAIN = B_SDPFULL + 8,
                          NBAR = B_DRAIN + 1;
-    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag, mask flags[KVS]
-    static constexpr int SMEM = OFF_MISC + 16 + KVS * 4;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
+    static constexpr int SMEM = OFF_MISC + 16;
     static_assert(SMEM <= 232448, "shared memory budget");
-    // TMEM columns
+    // TMEM columns; dQ is one D-wide block per query tile when they all fit
+    // (256 + 2D + nt*D <= 512), else a single block drained every tile
     static constexpr int T_S = 0, T_DP = 128, T_DK = 256, T_DV = 256 + D, T_DQ = 256 + 2 * D;
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     tri_attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                              const __grid_constant__ CUtensorMap tm_bias, const BwdParams p) {
@@ -171,7 +223,6 @@ __global__ void __launch_bounds__(320, 1)
     auto BAR = [&](int idx) -> uint32_t { return sb + L::OFF_BAR + idx * 8; };
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
-    volatile int* mask_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 16);
 
     const int nt = p.nt;
     const int problems = p.B * p.N * p.H;
@@ -222,6 +273,7 @@ __global__ void __launch_bounds__(320, 1)
 
     if (warp == 8) {
         // =========================== producer ===============================
+        regs_shrink();
         int armed_kv[L::KVS], armed_t[L::NS];
 #pragma unroll
         for (int s = 0; s < L::KVS; ++s) armed_kv[s] = 0;
@@ -256,35 +308,23 @@ __global__ void __launch_bounds__(320, 1)
                     c[p.bpos_b] = b;
                     tma_load_4d(dst, &tm_bias, bar, c[0], c[1], c[2], c[3]);
                 };
+                const float* mrow = p.Mv + (static_cast<int64_t>(b) * p.N + i) * p.Np;
+                const int* frow = p.Fv + (static_cast<int64_t>(b) * p.N + i) * 32;
+                const int64_t vrow = ((static_cast<int64_t>(b) * p.H + h) * p.N + i) * p.Np;
                 for (int kt = 0; ok && kt < nt; ++kt) {
                     const int ks = gk % L::KVS;
                     if (gk >= L::KVS && !mbar_wait_warp(BAR(L::B_KVEMPTY + ks), ((gk / L::KVS) - 1) & 1, wc, 1)) {
                         ok = false;
                         break;
                     }
-                    {  // key mask row (user mask, -inf past N)
-                        float v[4];
-                        bool nz = false;
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int k = kt * 128 + lane * 4 + e;
-                            float x = -INFINITY;
-                            if (k < p.N) x = p.mask ? __ldg(p.mask + b * p.ms0 + i * p.ms1 + k * p.ms2) : 0.f;
-                            v[e] = x;
-                            nz |= (x != 0.f);
-                        }
-                        *reinterpret_cast<float4*>(smem + L::OFF_MASKV + ks * 512 + lane * 16) =
-                            make_float4(v[0], v[1], v[2], v[3]);
-                        const unsigned any = __any_sync(0xFFFFFFFFu, nz);
-                        if (lane == 0) mask_flag[ks] = any ? 1 : 0;
-                    }
-                    __syncwarp();
                     if (lane == 0) {
                         const uint32_t bar = BAR(L::B_KVFULL + ks);
                         const uint32_t base = sb + L::OFF_KV + ks * 2 * L::QKV_TILE;
-                        mbar_arrive_expect_tx(bar, 2 * L::QKV_TILE);
+                        mbar_arrive_expect_tx(bar, 2 * L::QKV_TILE + 512 + 128);
                         load_pair(base, &tm_k, bar, kt * 128);
                         load_pair(base + L::QKV_TILE, &tm_v, bar, kt * 128);
+                        bulk_load(sb + L::OFF_MASKV + ks * 512, mrow + kt * 128, 512, bar);
+                        bulk_load(sb + L::OFF_FLAGS + ks * 128, frow, 128, bar);
                     }
                     armed_kv[ks]++;
                     ++gk;
@@ -294,31 +334,16 @@ __global__ void __launch_bounds__(320, 1)
                             ok = false;
                             break;
                         }
-                        {  // lse (log2 units) and D rows for this query tile
-                            float* vec = reinterpret_cast<float*>(smem + L::OFF_VEC + ts * 1024);
-                            const int64_t rowbase = ((static_cast<int64_t>(b) * p.H + h) * p.N + i) * p.N;
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int jj = lane * 4 + e;
-                                const int j = jt * 128 + jj;
-                                float lv = INFINITY, dv = 0.f;
-                                if (j < p.N) {
-                                    lv = __ldg(p.lse + rowbase + j) * LOG2E;
-                                    dv = p.Dv[rowbase + j];
-                                }
-                                vec[jj] = lv;
-                                vec[128 + jj] = dv;
-                            }
-                        }
-                        __syncwarp();
                         if (lane == 0) {
                             const uint32_t bar = BAR(L::B_TFULL + ts);
                             const uint32_t base = sb + L::OFF_T + ts * L::T_STAGE;
-                            mbar_arrive_expect_tx(bar, 2 * L::QKV_TILE + L::BIAS_TILE);
+                            mbar_arrive_expect_tx(bar, 2 * L::QKV_TILE + L::BIAS_TILE + 1024);
                             load_pair(base, &tm_q, bar, jt * 128);
                             load_pair(base + L::QKV_TILE, &tm_do, bar, jt * 128);
                             load_bias(base + 2 * L::QKV_TILE, bar, kt * 128, jt * 128);
                             load_bias(base + 2 * L::QKV_TILE + L::BIAS_TILE / 2, bar, kt * 128 + 64, jt * 128);
+                            bulk_load(sb + L::OFF_VEC + ts * 1024, p.Lv + vrow + jt * 128, 512, bar);
+                            bulk_load(sb + L::OFF_VEC + ts * 1024 + 512, p.Dv + vrow + jt * 128, 512, bar);
                         }
                         armed_t[ts]++;
                         ++g;
@@ -336,6 +361,7 @@ __global__ void __launch_bounds__(320, 1)
         }
     } else if (warp == 9) {
         // =========================== MMA issuer =============================
+        regs_shrink();
         if (lane == 0 && !aborted_early) {
             constexpr uint32_t SW = (D == 32) ? SWZ_64B : SWZ_128B;
             constexpr uint32_t SBO = 8 * L::ROWB;
@@ -343,13 +369,20 @@ __global__ void __launch_bounds__(320, 1)
             constexpr uint32_t IDESC_G = idesc_bf16_f32(128, D, true, true);      // P^T dO, dS^T Q
             constexpr uint32_t IDESC_Q = idesc_bf16_f32(128, D, false, true);     // dS K
             struct Pending {
-                int g, ts, ks, jt, kcount;
+                int g, ts, ks, jt, kt, kcount;
                 bool valid;
-            } pend{0, 0, 0, 0, 0, false};
+            } pend{0, 0, 0, 0, 0, 0, false};
             bool ok = true;
+            int ep_count = 0;  // dQ epilogue tiles issued so far
             auto issue_grads = [&](const Pending& t) -> bool {
+                // a dQ epilogue tile: every tile (single block) or the last key tile of a query tile
+                const bool ep = !p.dq_tmem || t.kt == nt - 1;
                 if (!mbar_wait(BAR(L::B_PDSFULL), t.g & 1, wc, 3)) return false;
-                if (t.g > 0 && !mbar_wait(BAR(L::B_DQFREE), (t.g - 1) & 1, wc, 4)) return false;
+                // the previous epilogue has read its dQ block (keeps DQ_FULL at most one phase ahead,
+                // and before a new problem overwrites the last query tile's block)
+                const bool reuse = p.dq_tmem && t.kt == 0 && t.jt == nt - 1;
+                if ((ep || reuse) && ep_count > 0 && !mbar_wait(BAR(L::B_DQFREE), (ep_count - 1) & 1, wc, 4))
+                    return false;
                 if (t.jt == 0 && t.kcount > 0 && !mbar_wait(BAR(L::B_DKVFREE), (t.kcount - 1) & 1, wc, 5))
                     return false;
                 tc_fence_after();
@@ -369,16 +402,21 @@ __global__ void __launch_bounds__(320, 1)
                     mma_ss(tmem + L::T_DV, adp, bdo, IDESC_G, acc);
                     mma_ss(tmem + L::T_DK, ads, bq, IDESC_G, acc);
                 }
+                const uint32_t dq_col = p.dq_tmem ? L::T_DQ + t.jt * D : L::T_DQ;
+                const bool dq_acc = p.dq_tmem && t.kt > 0;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {  // contraction over 128 keys
                     // A = dS rows j: K-major, two 64-key halves 16 KB apart
                     const uint64_t a = smem_desc(dsa + (kk >> 2) * (L::PT_TILE / 2) + (kk & 3) * 32, 16, 1024, SWZ_128B);
                     const uint64_t bk = smem_desc(ka + kk * 16 * L::ROWB, L::QKV_TILE, SBO, SW);
-                    mma_ss(tmem + L::T_DQ, a, bk, IDESC_Q, kk > 0 ? 1u : 0u);
+                    mma_ss(tmem + dq_col, a, bk, IDESC_Q, (dq_acc || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(BAR(L::B_PDSFREE));
                 mma_commit(BAR(L::B_TEMPTY + t.ts));
-                mma_commit(BAR(L::B_DQFULL));
+                if (ep) {
+                    mma_commit(BAR(L::B_DQFULL));
+                    ++ep_count;
+                }
                 if (t.jt == nt - 1) {
                     mma_commit(BAR(L::B_DKVFULL));
                     mma_commit(BAR(L::B_KVEMPTY + t.ks));
@@ -414,7 +452,7 @@ __global__ void __launch_bounds__(320, 1)
                         if (pend.valid) {
                             if (!(ok = issue_grads(pend))) break;
                         }
-                        pend = Pending{g, ts, ks, jt, gk, true};
+                        pend = Pending{g, ts, ks, jt, kt, gk, true};
                         ++g;
                     }
                     ++gk;
@@ -425,74 +463,83 @@ __global__ void __launch_bounds__(320, 1)
             drain_wait(BAR(L::B_DRAIN), 0, 100000000ull);
         }
         __syncwarp();
-    } else if (!aborted_early) {
+    } else if (warp >= 10) {
+        regs_shrink();  // spare warps of the last warpgroup
+    } else {
+        regs_grow();
+        if (!aborted_early) {
         // =========================== softmax + epilogue warps ===============
         const int w = warp >> 2;  // column half of every tile handled by this warpgroup
         const int qd = warp & 3;
         const int row = qd * 32 + lane;
         const uint32_t tl = tmem + (static_cast<uint32_t>(qd * 32) << 16);
-        const float scale = p.scale, c2 = p.scale * LOG2E;
+        const float scale = p.scale;
         struct Done {
             int g, jt, kt, kcount, b, h, i;
             bool valid;
         } prev{0, 0, 0, 0, 0, 0, 0, false};
         bool ok = true;
 
+        int ep_count = 0;  // dQ epilogues done
         auto epilogue = [&](const Done& t) -> bool {
-            // ---- dQ tile: this warpgroup's D/2 columns, accumulated over kt in the slot ----
-            if (!mbar_wait_warp(BAR(L::B_DQFULL), t.g & 1, wc, 10)) return false;
-            tc_fence_after();
-            uint32_t dqr[D / 2];
-            if constexpr (D == 32) {
-                uint32_t x[16];
-                tmem_ld16(tl + L::T_DQ + w * 16, x);
-                tmem_wait_ld();
-                asm volatile("" : "+r"(x[0]), "+r"(x[1]), "+r"(x[2]), "+r"(x[3]), "+r"(x[4]), "+r"(x[5]),
-                             "+r"(x[6]), "+r"(x[7]), "+r"(x[8]), "+r"(x[9]), "+r"(x[10]), "+r"(x[11]),
-                             "+r"(x[12]), "+r"(x[13]), "+r"(x[14]), "+r"(x[15]));
+            // ---- dQ: this warpgroup's D/2 columns of the tile's block ----
+            if (!p.dq_tmem || t.kt == nt - 1) {
+                if (!mbar_wait_warp(BAR(L::B_DQFULL), ep_count & 1, wc, 10)) return false;
+                tc_fence_after();
+                const uint32_t dq_col = p.dq_tmem ? L::T_DQ + t.jt * D : L::T_DQ;
+                uint32_t dqr[D / 2];
+                if constexpr (D == 32) {
+                    uint32_t x[16];
+                    tmem_ld16(tl + dq_col + w * 16, x);
+                    tmem_wait_ld();
+                    asm volatile("" : "+r"(x[0]), "+r"(x[1]), "+r"(x[2]), "+r"(x[3]), "+r"(x[4]), "+r"(x[5]),
+                                 "+r"(x[6]), "+r"(x[7]), "+r"(x[8]), "+r"(x[9]), "+r"(x[10]), "+r"(x[11]),
+                                 "+r"(x[12]), "+r"(x[13]), "+r"(x[14]), "+r"(x[15]));
 #pragma unroll
-                for (int e = 0; e < 16; ++e) dqr[e] = x[e];
-            } else {
-                uint32_t x[32];
-                tmem_ld32(tl + L::T_DQ + w * 32, x);
-                tmem_wait_ld();
-                reg_fence32(x);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) dqr[e] = x[e];
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(BAR(L::B_DQFREE));
-            const int j = t.jt * 128 + row;
-            if (j < p.N) {
-                float* slot = p.dq_slots + (static_cast<int64_t>(blockIdx.x) * p.N + j) * D + w * (D / 2);
-                float acc[D / 2];
-#pragma unroll
-                for (int e = 0; e < D / 2; ++e) acc[e] = __uint_as_float(dqr[e]);
-                if (t.kt > 0) {
-#pragma unroll
-                    for (int e = 0; e < D / 2; e += 4) {
-                        const float4 v = *reinterpret_cast<const float4*>(slot + e);
-                        acc[e] += v.x;
-                        acc[e + 1] += v.y;
-                        acc[e + 2] += v.z;
-                        acc[e + 3] += v.w;
-                    }
-                }
-                if (t.kt < nt - 1) {
-#pragma unroll
-                    for (int e = 0; e < D / 2; e += 4)
-                        *reinterpret_cast<float4*>(slot + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+                    for (int e = 0; e < 16; ++e) dqr[e] = x[e];
                 } else {
-                    __nv_bfloat16* dst = p.dq + t.b * p.dqs[0] + t.i * p.dqs[1] + j * p.dqs[2] + t.h * p.dqs[3] + w * (D / 2);
+                    uint32_t x[32];
+                    tmem_ld32(tl + dq_col + w * 32, x);
+                    tmem_wait_ld();
+                    reg_fence32(x);
 #pragma unroll
-                    for (int e = 0; e < D / 2; e += 8) {
-                        uint4 v;
-                        v.x = pack_bf16(acc[e] * scale, acc[e + 1] * scale);
-                        v.y = pack_bf16(acc[e + 2] * scale, acc[e + 3] * scale);
-                        v.z = pack_bf16(acc[e + 4] * scale, acc[e + 5] * scale);
-                        v.w = pack_bf16(acc[e + 6] * scale, acc[e + 7] * scale);
-                        *reinterpret_cast<uint4*>(dst + e) = v;
+                    for (int e = 0; e < 32; ++e) dqr[e] = x[e];
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(BAR(L::B_DQFREE));
+                ++ep_count;
+                const int j = t.jt * 128 + row;
+                if (j < p.N) {
+                    float acc[D / 2];
+#pragma unroll
+                    for (int e = 0; e < D / 2; ++e) acc[e] = __uint_as_float(dqr[e]);
+                    float* slot = p.dq_slots + (static_cast<int64_t>(blockIdx.x) * p.N + j) * D + w * (D / 2);
+                    if (!p.dq_tmem && t.kt > 0) {
+#pragma unroll
+                        for (int e = 0; e < D / 2; e += 4) {
+                            const float4 v = *reinterpret_cast<const float4*>(slot + e);
+                            acc[e] += v.x;
+                            acc[e + 1] += v.y;
+                            acc[e + 2] += v.z;
+                            acc[e + 3] += v.w;
+                        }
+                    }
+                    if (!p.dq_tmem && t.kt < nt - 1) {
+#pragma unroll
+                        for (int e = 0; e < D / 2; e += 4)
+                            *reinterpret_cast<float4*>(slot + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+                    } else {
+                        __nv_bfloat16* dst = p.dq + t.b * p.dqs[0] + t.i * p.dqs[1] + j * p.dqs[2] + t.h * p.dqs[3] + w * (D / 2);
+#pragma unroll
+                        for (int e = 0; e < D / 2; e += 8) {
+                            uint4 v;
+                            v.x = pack_bf16(acc[e] * scale, acc[e + 1] * scale);
+                            v.y = pack_bf16(acc[e + 2] * scale, acc[e + 3] * scale);
+                            v.z = pack_bf16(acc[e + 4] * scale, acc[e + 5] * scale);
+                            v.w = pack_bf16(acc[e + 6] * scale, acc[e + 7] * scale);
+                            *reinterpret_cast<uint4*>(dst + e) = v;
+                        }
                     }
                 }
             }
@@ -540,7 +587,7 @@ __global__ void __launch_bounds__(320, 1)
             for (int kt = 0; ok && kt < nt; ++kt) {
                 const int ks = gk % L::KVS;
                 if (!mbar_wait_warp(BAR(L::B_KVFULL + ks), (gk / L::KVS) & 1, wc, 12)) { ok = false; break; }
-                const bool has_mask = mask_flag[ks] != 0;
+                const bool has_mask = reinterpret_cast<const int*>(smem + L::OFF_FLAGS + ks * 128)[kt] != 0;
                 const uint32_t maskv = sb + L::OFF_MASKV + ks * 512 + w * 256;
                 for (int jt = 0; jt < nt; ++jt) {
                     const int ts = g % L::NS;
@@ -570,40 +617,47 @@ __global__ void __launch_bounds__(320, 1)
                     if (g > 0 && !mbar_wait_warp(BAR(L::B_PDSFREE), (g - 1) & 1, wc, 15)) { ok = false; break; }
                     const uint32_t prow = sb + L::OFF_P + w * (L::PT_TILE / 2) + row * 128;
                     const uint32_t drow = sb + L::OFF_DS + w * (L::PT_TILE / 2) + row * 128;
+                    // p = 2^((S*scale + bias)*log2e [+ mask*log2e] - lse*log2e), ds = p (dP - D)
+                    const float2 sc2 = make_float2(scale, scale), l2e = make_float2(LOG2E, LOG2E);
+                    const float2 nl2 = make_float2(-lse2, -lse2), nD2 = make_float2(-Dj, -Dj);
+                    auto tile = [&](auto masked) {
+                        constexpr bool kMasked = decltype(masked)::value;
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint32_t off = (c ^ (row & 7)) << 4;
-                        const uint4 bb = lds128(brow + off);
-                        const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
-                        float mk[8];
-                        if (has_mask) {
-                            const float4 m0 = lds128f(maskv + c * 32), m1 = lds128f(maskv + c * 32 + 16);
-                            mk[0] = m0.x; mk[1] = m0.y; mk[2] = m0.z; mk[3] = m0.w;
-                            mk[4] = m1.x; mk[5] = m1.y; mk[6] = m1.z; mk[7] = m1.w;
-                        } else {
+                        for (int c = 0; c < 8; ++c) {
+                            const uint32_t off = (c ^ (row & 7)) << 4;
+                            const uint4 bb = lds128(brow + off);
+                            const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+                            float mk[8];
+                            if constexpr (kMasked) {
+                                const float4 m0 = lds128f(maskv + c * 32), m1 = lds128f(maskv + c * 32 + 16);
+                                mk[0] = m0.x; mk[1] = m0.y; mk[2] = m0.z; mk[3] = m0.w;
+                                mk[4] = m1.x; mk[5] = m1.y; mk[6] = m1.z; mk[7] = m1.w;
+                            }
+                            uint32_t pw[4], dw[4];
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) mk[e] = 0.f;
+                            for (int e = 0; e < 4; ++e) {
+                                const int x0 = c * 8 + 2 * e;
+                                const uint32_t sv0 = (x0 < 32) ? s0[x0] : s1[x0 - 32];
+                                const uint32_t sv1 = (x0 + 1 < 32) ? s0[x0 + 1] : s1[x0 + 1 - 32];
+                                const uint32_t dv0 = (x0 < 32) ? d0[x0] : d1[x0 - 32];
+                                const uint32_t dv1 = (x0 + 1 < 32) ? d0[x0 + 1] : d1[x0 + 1 - 32];
+                                const float2 t = ffma2(make_float2(__uint_as_float(sv0), __uint_as_float(sv1)), sc2,
+                                                       bf16x2_to_f2(bw[e]));
+                                float2 y = ffma2(t, l2e, nl2);
+                                if constexpr (kMasked) y = fadd2(y, make_float2(mk[2 * e], mk[2 * e + 1]));
+                                const float p0 = ex2(y.x), p1 = ex2(y.y);
+                                const float2 ds = fmul2(make_float2(p0, p1),
+                                                        fadd2(make_float2(__uint_as_float(dv0), __uint_as_float(dv1)), nD2));
+                                const float ds0 = ds.x, ds1 = ds.y;
+                                pw[e] = pack_bf16(p0, p1);
+                                dw[e] = pack_bf16(ds0, ds1);
+                            }
+                            sts128(prow + off, make_uint4(pw[0], pw[1], pw[2], pw[3]));
+                            sts128(drow + off, make_uint4(dw[0], dw[1], dw[2], dw[3]));
                         }
-                        uint32_t pw[4], dw[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int x0 = c * 8 + 2 * e;
-                            const uint32_t sv0 = (x0 < 32) ? s0[x0] : s1[x0 - 32];
-                            const uint32_t sv1 = (x0 + 1 < 32) ? s0[x0 + 1] : s1[x0 + 1 - 32];
-                            const uint32_t dv0 = (x0 < 32) ? d0[x0] : d1[x0 - 32];
-                            const uint32_t dv1 = (x0 + 1 < 32) ? d0[x0 + 1] : d1[x0 + 1 - 32];
-                            // y*log2e = S*scale*log2e + (bias + mask)*log2e
-                            const float y0 = fmaf(__uint_as_float(sv0), c2, (bf16lo(bw[e]) + mk[2 * e]) * LOG2E);
-                            const float y1 = fmaf(__uint_as_float(sv1), c2, (bf16hi(bw[e]) + mk[2 * e + 1]) * LOG2E);
-                            const float p0 = ex2(y0 - lse2), p1 = ex2(y1 - lse2);
-                            const float ds0 = p0 * (__uint_as_float(dv0) - Dj);
-                            const float ds1 = p1 * (__uint_as_float(dv1) - Dj);
-                            pw[e] = pack_bf16(p0, p1);
-                            dw[e] = pack_bf16(ds0, ds1);
-                        }
-                        sts128(prow + off, make_uint4(pw[0], pw[1], pw[2], pw[3]));
-                        sts128(drow + off, make_uint4(dw[0], dw[1], dw[2], dw[3]));
-                    }
+                    };
+                    if (has_mask) tile(std::true_type{});
+                    else tile(std::false_type{});
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
@@ -621,8 +675,10 @@ __global__ void __launch_bounds__(320, 1)
         if (ok && prev.valid) epilogue(prev);
     }
 
+    }
+
     tc_fence_before();
-    __syncthreads();
+    cta_end_barrier();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
@@ -639,18 +695,19 @@ struct DbLayout {
     static constexpr int QKV_TILE = 128 * ROWB;
     static constexpr int STAGE = 4 * QKV_TILE;  // Q, dO, K, V
     static constexpr int OFF_BIAS = NS * STAGE;  // [128 rows][128 keys] fp32, log2 units, swizzled
-    static constexpr int OFF_VEC = OFF_BIAS + 128 * 128 * 4;  // [NS][lse2 128, D 128, mask 128] fp32
-    static constexpr int VEC = 1536;
+    // [NS][lse*log2e 128, D 128, mask*log2e 128 (fp32), key-tile flags 32 (int)]
+    static constexpr int OFF_VEC = OFF_BIAS + 128 * 128 * 4;
+    static constexpr int VEC = 1664;
     static constexpr int OFF_BAR = OFF_VEC + NS * VEC;
     static constexpr int B_FULL = 0, B_EMPTY = NS, B_SDPFULL = 2 * NS, B_SDPFREE = 2 * NS + 2,
                          B_DRAIN = 2 * NS + 4, NBAR = B_DRAIN + 1;
-    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort, mask flags[NS]
-    static constexpr int SMEM = OFF_MISC + 16 + NS * 4;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort
+    static constexpr int SMEM = OFF_MISC + 16;
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     tri_attn_bwd_dbias_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                               const __nv_bfloat16* __restrict__ bias, int64_t bs0, int64_t bs1, int64_t bs2,
@@ -662,7 +719,6 @@ __global__ void __launch_bounds__(320, 1)
     auto BAR = [&](int idx) -> uint32_t { return sb + L::OFF_BAR + idx * 8; };
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
-    volatile int* mask_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 16);
 
     const int nt = p.nt;
     int item = blockIdx.x;
@@ -709,6 +765,7 @@ __global__ void __launch_bounds__(320, 1)
     constexpr float LOG2E = 1.4426950408889634f;
 
     if (warp == 8) {
+        regs_shrink();
         int armed[L::NS];
 #pragma unroll
         for (int s = 0; s < L::NS; ++s) armed[s] = 0;
@@ -723,33 +780,13 @@ __global__ void __launch_bounds__(320, 1)
                 const int i = i_begin + n;
                 const int s = n % L::NS;
                 if (n >= L::NS && !mbar_wait_warp(BAR(L::B_EMPTY + s), ((n / L::NS) - 1) & 1, wc, 1)) break;
-                float* vec = reinterpret_cast<float*>(smem + L::OFF_VEC + s * L::VEC);
-                const int64_t rowbase = ((static_cast<int64_t>(b) * p.H + h) * p.N + i) * p.N;
-                bool nz = false;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int jj = lane * 4 + e;
-                    const int j = jt * 128 + jj;
-                    float lv = INFINITY, dv = 0.f;
-                    if (j < p.N) {
-                        lv = __ldg(p.lse + rowbase + j) * LOG2E;
-                        dv = p.Dv[rowbase + j];
-                    }
-                    vec[jj] = lv;
-                    vec[128 + jj] = dv;
-                    const int k = kt * 128 + jj;
-                    float mv = -INFINITY;
-                    if (k < p.N) mv = p.mask ? __ldg(p.mask + b * p.ms0 + i * p.ms1 + k * p.ms2) : 0.f;
-                    vec[256 + jj] = mv * LOG2E;
-                    nz |= (mv != 0.f);
-                }
-                const unsigned any = __any_sync(0xFFFFFFFFu, nz);
-                if (lane == 0) mask_flag[s] = any ? 1 : 0;
-                __syncwarp();
                 if (lane == 0) {
                     const uint32_t bar = BAR(L::B_FULL + s);
                     const uint32_t base = sb + s * L::STAGE;
-                    mbar_arrive_expect_tx(bar, L::STAGE);
+                    const uint32_t vec = sb + L::OFF_VEC + s * L::VEC;
+                    const int64_t vrow = ((static_cast<int64_t>(b) * p.H + h) * p.N + i) * p.Np + jt * 128;
+                    const int64_t mrow = (static_cast<int64_t>(b) * p.N + i) * p.Np + kt * 128;
+                    mbar_arrive_expect_tx(bar, L::STAGE + L::VEC);
                     auto ld = [&](uint32_t dst, const CUtensorMap* m, int row0) {
                         int c[5] = {0, 0, 0, 0, 0};
                         c[p.qpos_h] = h;
@@ -762,6 +799,10 @@ __global__ void __launch_bounds__(320, 1)
                     ld(base + L::QKV_TILE, &tm_do, jt * 128);
                     ld(base + 2 * L::QKV_TILE, &tm_k, kt * 128);
                     ld(base + 3 * L::QKV_TILE, &tm_v, kt * 128);
+                    bulk_load(vec, p.Lv + vrow, 512, bar);
+                    bulk_load(vec + 512, p.Dv + vrow, 512, bar);
+                    bulk_load(vec + 1024, p.Mv + mrow, 512, bar);
+                    bulk_load(vec + 1536, p.Fv + (static_cast<int64_t>(b) * p.N + i) * 32, 128, bar);
                 }
                 armed[s]++;
             }
@@ -772,6 +813,7 @@ __global__ void __launch_bounds__(320, 1)
                 if (armed[s] > 0) drain_wait(BAR(L::B_FULL + s), (armed[s] - 1) & 1, 100000000ull);
         }
     } else if (warp == 9) {
+        regs_shrink();
         if (lane == 0 && !aborted_early) {
             constexpr uint32_t SW = (D == 32) ? SWZ_64B : SWZ_128B;
             constexpr uint32_t SBO = 8 * L::ROWB;
@@ -796,7 +838,11 @@ __global__ void __launch_bounds__(320, 1)
             drain_wait(BAR(L::B_DRAIN), 0, 100000000ull);
         }
         __syncwarp();
-    } else if (!aborted_early) {
+    } else if (warp >= 10) {
+        regs_shrink();  // spare warps of the last warpgroup
+    } else {
+        regs_grow();
+        if (!aborted_early) {
         const int w = warp >> 2;
         const int qd = warp & 3;
         const int row = qd * 32 + lane;
@@ -832,8 +878,9 @@ __global__ void __launch_bounds__(320, 1)
             const float* vec = reinterpret_cast<const float*>(smem + L::OFF_VEC + s * L::VEC);
             const float lse2 = vec[row];
             const float Dj = vec[128 + row];
-            const bool has_mask = mask_flag[s] != 0;
+            const bool has_mask = reinterpret_cast<const int*>(vec + 384)[kt] != 0;
             const uint32_t ma = sb + L::OFF_VEC + s * L::VEC + 1024 + w * 256;
+            const float2 c22 = make_float2(c2, c2), nl2 = make_float2(-lse2, -lse2), nD2 = make_float2(-Dj, -Dj);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t sv[32], dv[32];
@@ -851,14 +898,23 @@ __global__ void __launch_bounds__(320, 1)
                 for (int c = 0; c < 8; ++c) {
                     const int cc = half * 8 + c;
                     const float4 bq = lds128f(brow + ((cc ^ (row & 15)) << 4));
-                    float4 mq = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (has_mask) mq = lds128f(ma + cc * 16);
-                    const float bb[4] = {bq.x + mq.x, bq.y + mq.y, bq.z + mq.z, bq.w + mq.w};
+                    float2 b01 = make_float2(bq.x, bq.y), b23 = make_float2(bq.z, bq.w);
+                    if (has_mask) {
+                        const float4 mq = lds128f(ma + cc * 16);
+                        b01 = fadd2(b01, make_float2(mq.x, mq.y));
+                        b23 = fadd2(b23, make_float2(mq.z, mq.w));
+                    }
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int xl = 4 * c + e;
-                        const float pv = ex2(fmaf(__uint_as_float(sv[xl]), c2, bb[e]) - lse2);
-                        acc[32 * half + xl] = fmaf(pv, __uint_as_float(dv[xl]) - Dj, acc[32 * half + xl]);
+                    for (int e = 0; e < 2; ++e) {
+                        const int xl = 4 * c + 2 * e;
+                        const float2 t = ffma2(make_float2(__uint_as_float(sv[xl]), __uint_as_float(sv[xl + 1])), c22,
+                                               e ? b23 : b01);
+                        const float2 y = fadd2(t, nl2);
+                        const float2 pv = make_float2(ex2(y.x), ex2(y.y));
+                        const float2 dd = fadd2(make_float2(__uint_as_float(dv[xl]), __uint_as_float(dv[xl + 1])), nD2);
+                        const float2 a = ffma2(pv, dd, make_float2(acc[32 * half + xl], acc[32 * half + xl + 1]));
+                        acc[32 * half + xl] = a.x;
+                        acc[32 * half + xl + 1] = a.y;
                     }
                 }
             }
@@ -893,8 +949,10 @@ __global__ void __launch_bounds__(320, 1)
         }
     }
 
+    }
+
     tc_fence_before();
-    __syncthreads();
+    cta_end_barrier();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);

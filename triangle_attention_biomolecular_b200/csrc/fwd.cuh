@@ -13,8 +13,10 @@
 // backward.
 //
 // B200 mapping:
-//  * one CTA = 320 threads: warps 0-3 softmax for row i0, warps 4-7 softmax
-//    for row i1, warp 8 TMA producer, warp 9 MMA issuer (one thread);
+//  * one CTA = 384 threads: warps 0-3 softmax for row i0, warps 4-7 softmax
+//    for row i1, warp 8 TMA producer, warp 9 MMA issuer (one thread), warps
+//    10-11 idle; the last warpgroup hands most of its registers to the
+//    softmax warpgroups;
 //  * both rows share every bias tile (the bias is the same for all rows i),
 //    so each 32 KB bias tile crosses L2->SMEM once per two rows;
 //  * TMEM (512 columns): per warpgroup w, S at 256w, P (BF16 pairs) at
@@ -90,7 +92,7 @@ __device__ __forceinline__ void reg_fence32(uint32_t (&r)[32]) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     tri_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_bias,
                         const FwdParams p) {
@@ -149,6 +151,7 @@ __global__ void __launch_bounds__(320, 1)
 
     if (warp == 8) {
         // =========================== TMA producer ===========================
+        regs_shrink();
         int armed[L::NS];
 #pragma unroll
         for (int s = 0; s < L::NS; ++s) armed[s] = 0;
@@ -178,26 +181,34 @@ __global__ void __launch_bounds__(320, 1)
                 load_qkv(sb + L::OFF_Q, &tm_q, BAR(L::B_Q), i0, jt * 128);
                 load_qkv(sb + L::OFF_Q + L::QKV_TILE, &tm_q, BAR(L::B_Q), i1, jt * 128);
             }
-            for (int kt = 0; kt < nkt; ++kt) {
-                const int s = kt % L::NS;
-                if (kt >= L::NS && !mbar_wait_warp(BAR(L::B_EMPTY + s), ((kt / L::NS) - 1) & 1, wc, 1)) break;
-                const uint32_t st = sb + L::OFF_STAGES + s * L::STAGE;
-                // key-mask rows (user mask, -inf past N) for both rows i0, i1
+            // key-mask rows (user mask, -inf past N) are fetched one stage ahead so
+            // their latency overlaps the wait for a free stage
+            float mnext[2][4];
+            auto fetch_mask = [&](int kt) {
 #pragma unroll
                 for (int w = 0; w < 2; ++w) {
                     const int i = w ? i1 : i0;
-                    float v[4];
-                    bool nz = false;
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int k = kt * 128 + lane * 4 + e;
                         float x = -INFINITY;
                         if (k < p.N) x = p.mask ? __ldg(p.mask + b * p.ms0 + i * p.ms1 + k * p.ms2) : 0.f;
-                        v[e] = x;
-                        nz |= (x != 0.f);
+                        mnext[w][e] = x;
                     }
+                }
+            };
+            fetch_mask(0);
+            for (int kt = 0; kt < nkt; ++kt) {
+                const int s = kt % L::NS;
+                if (kt >= L::NS && !mbar_wait_warp(BAR(L::B_EMPTY + s), ((kt / L::NS) - 1) & 1, wc, 1)) break;
+                const uint32_t st = sb + L::OFF_STAGES + s * L::STAGE;
+#pragma unroll
+                for (int w = 0; w < 2; ++w) {
+                    bool nz = false;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) nz |= (mnext[w][e] != 0.f);
                     float4* dst = reinterpret_cast<float4*>(smem + (st - sb) + L::OFF_MASK + w * 512 + lane * 16);
-                    *dst = make_float4(v[0], v[1], v[2], v[3]);
+                    *dst = make_float4(mnext[w][0], mnext[w][1], mnext[w][2], mnext[w][3]);
                     const unsigned any = __any_sync(0xFFFFFFFFu, nz);
                     if (lane == 0) mask_flag[s * 2 + w] = any ? 1 : 0;
                 }
@@ -213,6 +224,7 @@ __global__ void __launch_bounds__(320, 1)
                     load_bias(st + L::OFF_BIAS + L::BIAS_TILE / 2, bar, kt * 128 + 64, jt * 128);
                 }
                 armed[s]++;
+                if (kt + 1 < nkt) fetch_mask(kt + 1);
             }
         }
         // never leave with bulk copies still writing into this CTA's shared memory
@@ -224,6 +236,7 @@ __global__ void __launch_bounds__(320, 1)
         }
     } else if (warp == 9) {
         // =========================== MMA issuer =============================
+        regs_shrink();
         if (lane == 0 && !aborted_early) {
             constexpr uint32_t SW = (D == 32) ? SWZ_64B : SWZ_128B;
             constexpr uint32_t SBO = 8 * L::ROWB;
@@ -290,7 +303,11 @@ __global__ void __launch_bounds__(320, 1)
             drain_wait(BAR(L::B_DRAIN), 0, 100000000ull);
         }
         __syncwarp();
-    } else if (!aborted_early) {
+    } else if (warp >= 10) {
+        regs_shrink();  // spare warps of the last warpgroup
+    } else {
+        regs_grow();
+        if (!aborted_early) {
         // =========================== softmax warpgroups =====================
         const int w = warp >> 2;
         const int qd = warp & 3;
@@ -331,37 +348,46 @@ __global__ void __launch_bounds__(320, 1)
                 x[64 + e] = __uint_as_float(r2[e]);
                 x[96 + e] = __uint_as_float(r3[e]);
             }
-            // y = scale * S + bias (+ mask)
+            // y = scale * S + bias (+ mask), two lanes per instruction
             const uint32_t brow = st + L::OFF_BIAS + row * 128;
+            const float2 sc2 = make_float2(scale, scale);
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
                 const uint4 bb = lds128(brow + (c >> 3) * (L::BIAS_TILE / 2) + (((c & 7) ^ (row & 7)) << 4));
-                const int x0 = c * 8;
-                x[x0 + 0] = fmaf(x[x0 + 0], scale, bf16lo(bb.x));
-                x[x0 + 1] = fmaf(x[x0 + 1], scale, bf16hi(bb.x));
-                x[x0 + 2] = fmaf(x[x0 + 2], scale, bf16lo(bb.y));
-                x[x0 + 3] = fmaf(x[x0 + 3], scale, bf16hi(bb.y));
-                x[x0 + 4] = fmaf(x[x0 + 4], scale, bf16lo(bb.z));
-                x[x0 + 5] = fmaf(x[x0 + 5], scale, bf16hi(bb.z));
-                x[x0 + 6] = fmaf(x[x0 + 6], scale, bf16lo(bb.w));
-                x[x0 + 7] = fmaf(x[x0 + 7], scale, bf16hi(bb.w));
+                const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int x0 = c * 8 + 2 * e;
+                    const float2 y = ffma2(make_float2(x[x0], x[x0 + 1]), sc2, bf16x2_to_f2(bw[e]));
+                    x[x0] = y.x;
+                    x[x0 + 1] = y.y;
+                }
             }
             if (mask_flag[s * 2 + w]) {
                 const uint32_t ma = st + L::OFF_MASK + w * 512;
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
                     const float4 mv = lds128f(ma + c * 16);
-                    x[4 * c + 0] += mv.x;
-                    x[4 * c + 1] += mv.y;
-                    x[4 * c + 2] += mv.z;
-                    x[4 * c + 3] += mv.w;
+                    const float2 y0 = fadd2(make_float2(x[4 * c], x[4 * c + 1]), make_float2(mv.x, mv.y));
+                    const float2 y1 = fadd2(make_float2(x[4 * c + 2], x[4 * c + 3]), make_float2(mv.z, mv.w));
+                    x[4 * c] = y0.x;
+                    x[4 * c + 1] = y0.y;
+                    x[4 * c + 2] = y1.x;
+                    x[4 * c + 3] = y1.y;
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(BAR(L::B_EMPTY + s));
-            float mt = x[0];
+            // row maximum: four independent chains of three-input maxima
+            float ma0 = x[0], ma1 = x[1], ma2 = x[2], ma3 = x[3];
 #pragma unroll
-            for (int e = 1; e < 128; ++e) mt = fmaxf(mt, x[e]);
+            for (int e = 4; e < 128; e += 8) {
+                ma0 = fmax3(ma0, x[e], x[e + 1]);
+                ma1 = fmax3(ma1, x[e + 2], x[e + 3]);
+                ma2 = fmax3(ma2, x[e + 4], x[e + 5]);
+                ma3 = fmax3(ma3, x[e + 6], x[e + 7]);
+            }
+            const float mt = fmaxf(fmaxf(ma0, ma1), fmaxf(ma2, ma3));
             bool need = false;
             float alpha = 1.f;
             if (kt == 0) {
@@ -378,19 +404,27 @@ __global__ void __launch_bounds__(320, 1)
                 if (!mbar_wait_warp(BAR(L::B_PVDONE + w), (kt - 1) & 1, wc, 8)) { ok = false; break; }
                 tc_fence_after();
             }
-            float ls = 0.f;
+            const float2 l2e = make_float2(LOG2E, LOG2E), nmb = make_float2(-mb, -mb);
+            float2 ls0 = make_float2(0.f, 0.f), ls1 = ls0, ls2 = ls0, ls3 = ls0;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {
-                    const float p0 = ex2(fmaf(x[32 * q + 2 * c], LOG2E, -mb));
-                    const float p1 = ex2(fmaf(x[32 * q + 2 * c + 1], LOG2E, -mb));
-                    ls += p0 + p1;
-                    pk[c] = pack_bf16(p0, p1);
+                    const float2 a2 = ffma2(make_float2(x[32 * q + 2 * c], x[32 * q + 2 * c + 1]), l2e, nmb);
+                    const float2 pp = make_float2(ex2(a2.x), ex2(a2.y));
+                    switch (c & 3) {
+                        case 0: ls0 = fadd2(ls0, pp); break;
+                        case 1: ls1 = fadd2(ls1, pp); break;
+                        case 2: ls2 = fadd2(ls2, pp); break;
+                        default: ls3 = fadd2(ls3, pp); break;
+                    }
+                    pk[c] = pack_bf16(pp.x, pp.y);
                 }
                 tmem_st16(tP + 16 * q, pk);
             }
+            const float2 lsum = fadd2(fadd2(ls0, ls1), fadd2(ls2, ls3));
+            const float ls = lsum.x + lsum.y;
             l += ls;
             if (kt > 0 && __any_sync(0xFFFFFFFFu, need)) {
                 // rare: the reference maximum moved, rescale this row of O before the next PV
@@ -446,8 +480,10 @@ __global__ void __launch_bounds__(320, 1)
         }
     }
 
+    }
+
     tc_fence_before();
-    __syncthreads();
+    cta_end_barrier();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
