@@ -134,40 +134,25 @@ tri_attn_status ensure_device() {
     return TRI_ATTN_OK;
 }
 
-// Outer (non-innermost) dimensions of a tensor map, sorted by increasing
-// byte stride so the descriptor always sees an ascending stride order.
-struct OuterDim {
-    uint64_t size, stride_bytes;
-    uint32_t box;
-    int tag;
-};
-
-// Encode a tiled BF16 map.  inner = innermost extent (contiguous), inner_box
-// its box; outer dims are sorted by stride and their final positions (1-based
-// in the map) are returned through pos[tag].
-bool encode_map(CUtensorMap* m, void* ptr, uint64_t inner, uint32_t inner_box, OuterDim* od, int nouter,
-                CUtensorMapSwizzle swz, int* pos) {
-    // size-1 dims may carry any stride; give them a harmless valid one
-    for (int a = 0; a < nouter; ++a)
-        if (od[a].size == 1 || od[a].stride_bytes == 0) od[a].stride_bytes = 0;
-    std::stable_sort(od, od + nouter, [](const OuterDim& x, const OuterDim& y) { return x.stride_bytes < y.stride_bytes; });
-    uint64_t prev = inner * 2;
-    for (int a = 0; a < nouter; ++a) {
-        if (od[a].stride_bytes == 0) od[a].stride_bytes = ((prev + 15) / 16) * 16;
-        prev = od[a].stride_bytes * od[a].size;
-    }
+// Encode a tiled BF16 map with the outer dimensions in the given (fixed) order.
+// Strides need not be monotonic (an ending-node view swaps the j and i
+// strides); a size-1 dimension's stride is irrelevant and is replaced by a
+// harmless 16-byte multiple.
+bool encode_map(CUtensorMap* m, void* ptr, uint64_t inner, uint32_t inner_box, const uint64_t* size,
+                const uint64_t* stride_bytes, const uint32_t* box, int nouter, CUtensorMapSwizzle swz) {
     cuuint64_t dims[5], strides[4];
-    cuuint32_t box[5], estr[5] = {1, 1, 1, 1, 1};
+    cuuint32_t boxd[5], estr[5] = {1, 1, 1, 1, 1};
     dims[0] = inner;
-    box[0] = inner_box;
+    boxd[0] = inner_box;
     for (int a = 0; a < nouter; ++a) {
-        dims[a + 1] = od[a].size;
-        strides[a] = od[a].stride_bytes;
-        box[a + 1] = od[a].box;
-        pos[od[a].tag] = a + 1;
-        if (od[a].stride_bytes % 16 || od[a].stride_bytes >= (1ull << 40)) return false;
+        dims[a + 1] = size[a];
+        boxd[a + 1] = box[a];
+        uint64_t st = stride_bytes[a];
+        if (size[a] == 1) st = 16;
+        if (st == 0 || st % 16 || st >= (1ull << 40)) return false;
+        strides[a] = st;
     }
-    CUresult r = encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 1 + nouter, ptr, dims, strides, box, estr,
+    CUresult r = encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 1 + nouter, ptr, dims, strides, boxd, estr,
                            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS && std::getenv("TRI_ATTN_DEBUG")) {
@@ -176,35 +161,28 @@ bool encode_map(CUtensorMap* m, void* ptr, uint64_t inner, uint32_t inner_box, O
         for (int a = 0; a <= nouter; ++a) std::fprintf(stderr, " %llu", static_cast<unsigned long long>(dims[a]));
         std::fprintf(stderr, " strides");
         for (int a = 0; a < nouter; ++a) std::fprintf(stderr, " %llu", static_cast<unsigned long long>(strides[a]));
-        std::fprintf(stderr, " box");
-        for (int a = 0; a <= nouter; ++a) std::fprintf(stderr, " %u", box[a]);
-        std::fprintf(stderr, " swizzle %d\n", static_cast<int>(swz));
+        std::fprintf(stderr, "\n");
     }
     return r == CUDA_SUCCESS;
 }
 
-// Pair tensor [B,N,N,H,d] map with a 128-row box along j (or along i when
-// `rows_along_i`): tags 0=h, 1=j, 2=i, 3=b.
-bool map_pair(CUtensorMap* m, const tri_attn_tensor5& t, int B, int N, int H, int d, bool rows_along_i,
-              int* pos) {
-    OuterDim od[4] = {
-        {static_cast<uint64_t>(H), static_cast<uint64_t>(t.stride[3]) * 2, 1, 0},
-        {static_cast<uint64_t>(N), static_cast<uint64_t>(t.stride[2]) * 2, rows_along_i ? 1u : 128u, 1},
-        {static_cast<uint64_t>(N), static_cast<uint64_t>(t.stride[1]) * 2, rows_along_i ? 128u : 1u, 2},
-        {static_cast<uint64_t>(B), static_cast<uint64_t>(t.stride[0]) * 2, 1, 3},
-    };
-    return encode_map(m, t.ptr, d, d, od, 4, d == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
-                      pos);
+// Pair tensor [B,N,N,H,d] map: coordinates (c, h, j, i, b), box d x 1 x 128 x 1 x 1.
+bool map_pair(CUtensorMap* m, const tri_attn_tensor5& t, int B, int N, int H, int d) {
+    const uint64_t size[4] = {static_cast<uint64_t>(H), static_cast<uint64_t>(N), static_cast<uint64_t>(N),
+                              static_cast<uint64_t>(B)};
+    const uint64_t st[4] = {static_cast<uint64_t>(t.stride[3]) * 2, static_cast<uint64_t>(t.stride[2]) * 2,
+                            static_cast<uint64_t>(t.stride[1]) * 2, static_cast<uint64_t>(t.stride[0]) * 2};
+    const uint32_t box[4] = {1, 128, 1, 1};
+    return encode_map(m, t.ptr, d, d, size, st, box, 4, d == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// Bias [B,H,N,N] map: box 64 keys x 128 query rows, 128-byte swizzle; tags 0=j, 1=h, 2=b.
-bool map_bias(CUtensorMap* m, const tri_attn_tensor4& t, int B, int N, int H, int* pos) {
-    OuterDim od[3] = {
-        {static_cast<uint64_t>(N), static_cast<uint64_t>(t.stride[2]) * 2, 128, 0},
-        {static_cast<uint64_t>(H), static_cast<uint64_t>(t.stride[1]) * 2, 1, 1},
-        {static_cast<uint64_t>(B), static_cast<uint64_t>(t.stride[0]) * 2, 1, 2},
-    };
-    return encode_map(m, t.ptr, N, 64, od, 3, CU_TENSOR_MAP_SWIZZLE_128B, pos);
+// Bias [B,H,N,N] map: coordinates (k, j, h, b), box 64 keys x 128 rows, 128-byte swizzle.
+bool map_bias(CUtensorMap* m, const tri_attn_tensor4& t, int B, int N, int H) {
+    const uint64_t size[3] = {static_cast<uint64_t>(N), static_cast<uint64_t>(H), static_cast<uint64_t>(B)};
+    const uint64_t st[3] = {static_cast<uint64_t>(t.stride[2]) * 2, static_cast<uint64_t>(t.stride[1]) * 2,
+                            static_cast<uint64_t>(t.stride[0]) * 2};
+    const uint32_t box[3] = {128, 1, 1};
+    return encode_map(m, t.ptr, N, 64, size, st, box, 3, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 float eff_scale(float s, int d) { return s == 0.f ? 1.0f / std::sqrt(static_cast<float>(d)) : s; }
@@ -236,13 +214,9 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, f
     };
     const tri_attn_fwd_args& f = a->f;
     const int B = f.B, N = f.N, H = f.H, d = f.d;
-    CUtensorMap mq, mk, mv, mdo, mb;
-    int pq[4], pk[4], pv[4], pdo[4], pb[3];
-    if (!map_pair(&mq, f.q, B, N, H, d, false, pq) || !map_pair(&mk, f.k, B, N, H, d, false, pk) ||
-        !map_pair(&mv, f.v, B, N, H, d, false, pv) || !map_pair(&mdo, a->dout, B, N, H, d, false, pdo) ||
-        !map_bias(&mb, f.bias, B, N, H, pb))
-        return TRI_ATTN_ERR_STRIDE;
-    if (std::memcmp(pq, pk, sizeof pq) || std::memcmp(pq, pv, sizeof pq) || std::memcmp(pq, pdo, sizeof pq))
+    CUtensorMap mq, mk, mv, mdo;
+    if (!map_pair(&mq, f.q, B, N, H, d) || !map_pair(&mk, f.k, B, N, H, d) || !map_pair(&mv, f.v, B, N, H, d) ||
+        !map_pair(&mdo, a->dout, B, N, H, d))
         return TRI_ATTN_ERR_STRIDE;
     uint8_t* wsb = static_cast<uint8_t*>(a->workspace);
     BwdParams p{};
@@ -251,13 +225,13 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, f
     p.Np = ws.Np;
     p.dq_tmem = (256 + 2 * d + p.nt * d <= 512) ? 1 : 0;
     p.scale = scale;
-    p.qpos_h = pq[0]; p.qpos_j = pq[1]; p.qpos_i = pq[2]; p.qpos_b = pq[3];
-    p.bpos_j = pb[0]; p.bpos_h = pb[1]; p.bpos_b = pb[2];
     float* Dv = reinterpret_cast<float*>(wsb + ws.off_D);
     float* Lv = reinterpret_cast<float*>(wsb + ws.off_L);
     float* Mv = reinterpret_cast<float*>(wsb + ws.off_M);
     int* Fv = reinterpret_cast<int*>(wsb + ws.off_F);
     p.Dv = Dv; p.Lv = Lv; p.Mv = Mv; p.Fv = Fv;
+    p.bias = static_cast<const __nv_bfloat16*>(f.bias.ptr);
+    p.bs0 = f.bias.stride[0]; p.bs1 = f.bias.stride[1]; p.bs2 = f.bias.stride[2];
     p.dq_slots = reinterpret_cast<float*>(wsb + ws.off_dq);
     p.part = reinterpret_cast<float*>(wsb + ws.off_part);
     p.chunks = ws.chunks;
@@ -286,7 +260,7 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, f
             static_cast<const __nv_bfloat16*>(f.resid.ptr), sr[0], sr[1], sr[2], sr[3], use_resid, f.lse, f.mask.ptr,
             sm[0], sm[1], sm[2], Dv, Lv, Mv, Fv, B, N, H, ws.Np, p.nt);
         mark(1);
-        tri_attn_bwd_main_kernel<32><<<ws.grid_main, 384, MainLayout<32>::SMEM, stream>>>(mq, mk, mv, mdo, mb, p);
+        tri_attn_bwd_main_kernel<32><<<ws.grid_main, 384, MainLayout<32>::SMEM, stream>>>(mq, mk, mv, mdo, p);
         mark(2);
         tri_attn_bwd_dbias_kernel<32><<<db_grid, 384, DbLayout<32>::SMEM, stream>>>(
             mq, mk, mv, mdo, bias, f.bias.stride[0], f.bias.stride[1], f.bias.stride[2], p);
@@ -297,7 +271,7 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, f
             static_cast<const __nv_bfloat16*>(f.resid.ptr), sr[0], sr[1], sr[2], sr[3], use_resid, f.lse, f.mask.ptr,
             sm[0], sm[1], sm[2], Dv, Lv, Mv, Fv, B, N, H, ws.Np, p.nt);
         mark(1);
-        tri_attn_bwd_main_kernel<64><<<ws.grid_main, 384, MainLayout<64>::SMEM, stream>>>(mq, mk, mv, mdo, mb, p);
+        tri_attn_bwd_main_kernel<64><<<ws.grid_main, 384, MainLayout<64>::SMEM, stream>>>(mq, mk, mv, mdo, p);
         mark(2);
         tri_attn_bwd_dbias_kernel<64><<<db_grid, 384, DbLayout<64>::SMEM, stream>>>(
             mq, mk, mv, mdo, bias, f.bias.stride[0], f.bias.stride[1], f.bias.stride[2], p);
@@ -320,6 +294,11 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, f
 extern "C" {
 
 int tri_attn_abi_version(void) { return TRI_ATTN_ABI_VERSION; }
+
+#ifdef TRI_TRACE
+// instrumentation builds only: where the kernels write their phase cycles
+int tri_attn_trace_set(void* p) { return cudaMemcpyToSymbol(tri::g_trace, &p, sizeof(p)) == cudaSuccess ? 0 : 1; }
+#endif
 
 const char* tri_attn_strerror(tri_attn_status s) {
     switch (s) {
@@ -346,18 +325,14 @@ tri_attn_status tri_attn_fwd(const tri_attn_fwd_args* a, tri_attn_stream_t strea
     if ((st = ensure_device())) return st;
     const int B = a->B, N = a->N, H = a->H, d = a->d;
     CUtensorMap mq, mk, mv, mb;
-    int pq[4], pk[4], pv[4], pb[3];
-    if (!map_pair(&mq, a->q, B, N, H, d, false, pq) || !map_pair(&mk, a->k, B, N, H, d, false, pk) ||
-        !map_pair(&mv, a->v, B, N, H, d, false, pv) || !map_bias(&mb, a->bias, B, N, H, pb))
+    if (!map_pair(&mq, a->q, B, N, H, d) || !map_pair(&mk, a->k, B, N, H, d) || !map_pair(&mv, a->v, B, N, H, d) ||
+        !map_bias(&mb, a->bias, B, N, H))
         return TRI_ATTN_ERR_STRIDE;
-    if (std::memcmp(pq, pk, sizeof pq) || std::memcmp(pq, pv, sizeof pq)) return TRI_ATTN_ERR_STRIDE;
     tri::FwdParams p{};
     p.B = B; p.N = N; p.H = H;
     p.nt = (N + 127) / 128;
     p.npairs = (N + 1) / 2;
     p.scale = eff_scale(a->scale, d);
-    p.qpos_h = pq[0]; p.qpos_j = pq[1]; p.qpos_i = pq[2]; p.qpos_b = pq[3];
-    p.bpos_j = pb[0]; p.bpos_h = pb[1]; p.bpos_b = pb[2];
     p.mask = a->mask.ptr;
     p.ms0 = a->mask.stride[0]; p.ms1 = a->mask.stride[1]; p.ms2 = a->mask.stride[2];
     p.o = static_cast<__nv_bfloat16*>(a->o.ptr);

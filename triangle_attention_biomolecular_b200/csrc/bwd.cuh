@@ -81,12 +81,12 @@ inline BwdWorkspace bwd_workspace_layout(int B, int N, int H, int d) {
 struct BwdParams {
     int B, N, H, nt, Np;
     float scale;
-    int qpos_h, qpos_j, qpos_i, qpos_b;  // tensor-map coordinate positions (pair tensors)
-    int bpos_j, bpos_h, bpos_b;          // bias tensor map
     const float* Lv;  // [B,H,N,Np] lse * log2(e); +inf past N
     const float* Dv;  // [B,H,N,Np] D; 0 past N
     const float* Mv;  // [B,N,Np]   mask * log2(e); -inf past N
     const int* Fv;    // [B,N,32]   1 where a key tile needs the mask add
+    const __nv_bfloat16* bias;  // [B,H,N,N] (read directly by the softmax warps of the main kernel)
+    int64_t bs0, bs1, bs2;
     float* dq_slots;  // [kDqSlots][N][d] (used when dq_tmem == 0)
     int dq_tmem;      // 1: dQ for every query tile stays in TMEM across key tiles
     float* part;      // [chunks][B,H,N,N] (chunks > 1)
@@ -182,26 +182,25 @@ __global__ void __launch_bounds__(256) tri_attn_bwd_prep_kernel(
 template <int D>
 struct MainLayout {
     static constexpr int KVS = (D == 32) ? 2 : 1;  // K/V buffers
-    static constexpr int NS = 2;                   // per-tile stages (Q, dO, bias, vectors)
+    static constexpr int NS = 2;                   // per-tile stages (Q, dO, vectors)
     static constexpr int ROWB = D * 2;
     static constexpr int QKV_TILE = 128 * ROWB;
-    static constexpr int BIAS_TILE = 128 * 128 * 2;
     static constexpr int PT_TILE = 128 * 128 * 2;  // P or dS, BF16, two 64-column SW128 halves
     // 1 KB aligned tiles
-    static constexpr int OFF_KV = 0;  // [KVS][K, V]
-    static constexpr int OFF_T = OFF_KV + KVS * 2 * QKV_TILE;  // [NS][Q, dO, bias]
-    static constexpr int T_STAGE = 2 * QKV_TILE + BIAS_TILE;
-    static constexpr int OFF_P = OFF_T + NS * T_STAGE;
-    static constexpr int OFF_DS = OFF_P + PT_TILE;
+    static constexpr int OFF_KV = 0;                           // [KVS][K, V]
+    static constexpr int OFF_T = OFF_KV + KVS * 2 * QKV_TILE;  // [NS][Q, dO]
+    static constexpr int T_STAGE = 2 * QKV_TILE;
+    static constexpr int OFF_PDS = OFF_T + NS * T_STAGE;       // [2 buffers][P, dS]
+    static constexpr int PDS_BUF = 2 * PT_TILE;
     // vectors (bulk-copied from the pre-pass arrays)
-    static constexpr int OFF_MASKV = OFF_DS + PT_TILE;      // [KVS][128] fp32 mask*log2(e)
-    static constexpr int OFF_FLAGS = OFF_MASKV + KVS * 512; // [KVS][32] int: key tile needs the mask add
-    static constexpr int OFF_VEC = OFF_FLAGS + KVS * 128;   // [NS][lse*log2(e) 128, D 128] fp32
+    static constexpr int OFF_MASKV = OFF_PDS + 2 * PDS_BUF;  // [KVS][128] fp32 mask*log2(e)
+    static constexpr int OFF_FLAGS = OFF_MASKV + KVS * 512;  // [KVS][32] int: key tile needs the mask add
+    static constexpr int OFF_VEC = OFF_FLAGS + KVS * 128;    // [NS][lse*log2(e) 128, D 128] fp32
     static constexpr int OFF_BAR = OFF_VEC + NS * 1024;
     static constexpr int B_KVFULL = 0, B_KVEMPTY = KVS, B_TFULL = 2 * KVS, B_TEMPTY = 2 * KVS + NS,
                          B_SDPFULL = 2 * KVS + 2 * NS, B_SDPFREE = B_SDPFULL + 1, B_PDSFULL = B_SDPFULL + 2,
-                         B_PDSFREE = B_SDPFULL + 3, B_DQFULL = B_SDPFULL + 4, B_DQFREE = B_SDPFULL + 5,
-                         B_DKVFULL = B_SDPFULL + 6, B_DKVFREE = B_SDPFULL + 7, B_DRAIN = B_SDPFULL + 8,
+                         B_PDSFREE = B_SDPFULL + 4, B_DQFULL = B_SDPFULL + 6, B_DQFREE = B_SDPFULL + 7,
+                         B_DKVFULL = B_SDPFULL + 8, B_DKVFREE = B_SDPFULL + 9, B_DRAIN = B_SDPFULL + 10,
                          NBAR = B_DRAIN + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
     static constexpr int SMEM = OFF_MISC + 16;
@@ -215,7 +214,7 @@ template <int D>
 __global__ void __launch_bounds__(384, 1)
     tri_attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                             const __grid_constant__ CUtensorMap tm_bias, const BwdParams p) {
+                             const BwdParams p) {
     using L = MainLayout<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sb = smem_addr(smem);
@@ -250,8 +249,10 @@ __global__ void __launch_bounds__(384, 1)
         }
         mbar_init(BAR(L::B_SDPFULL), 1);
         mbar_init(BAR(L::B_SDPFREE), 8);
-        mbar_init(BAR(L::B_PDSFULL), 8);
-        mbar_init(BAR(L::B_PDSFREE), 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(BAR(L::B_PDSFULL + x), 8);
+            mbar_init(BAR(L::B_PDSFREE + x), 1);
+        }
         mbar_init(BAR(L::B_DQFULL), 1);
         mbar_init(BAR(L::B_DQFREE), 8);
         mbar_init(BAR(L::B_DKVFULL), 1);
@@ -285,7 +286,6 @@ __global__ void __launch_bounds__(384, 1)
                 tma_prefetch_map(&tm_k);
                 tma_prefetch_map(&tm_v);
                 tma_prefetch_map(&tm_do);
-                tma_prefetch_map(&tm_bias);
             }
             int gk = 0, g = 0;
             bool ok = true;
@@ -293,20 +293,7 @@ __global__ void __launch_bounds__(384, 1)
                 int b, h, i;
                 decode(pr, b, h, i);
                 auto load_pair = [&](uint32_t dst, const CUtensorMap* m, uint32_t bar, int row0) {
-                    int c[5] = {0, 0, 0, 0, 0};
-                    c[p.qpos_h] = h;
-                    c[p.qpos_j] = row0;
-                    c[p.qpos_i] = i;
-                    c[p.qpos_b] = b;
-                    tma_load_5d(dst, m, bar, c[0], c[1], c[2], c[3], c[4]);
-                };
-                auto load_bias = [&](uint32_t dst, uint32_t bar, int k0, int j0) {
-                    int c[4] = {0, 0, 0, 0};
-                    c[0] = k0;
-                    c[p.bpos_j] = j0;
-                    c[p.bpos_h] = h;
-                    c[p.bpos_b] = b;
-                    tma_load_4d(dst, &tm_bias, bar, c[0], c[1], c[2], c[3]);
+                    tma_load_5d(dst, m, bar, 0, h, row0, i, b);
                 };
                 const float* mrow = p.Mv + (static_cast<int64_t>(b) * p.N + i) * p.Np;
                 const int* frow = p.Fv + (static_cast<int64_t>(b) * p.N + i) * 32;
@@ -337,11 +324,9 @@ __global__ void __launch_bounds__(384, 1)
                         if (lane == 0) {
                             const uint32_t bar = BAR(L::B_TFULL + ts);
                             const uint32_t base = sb + L::OFF_T + ts * L::T_STAGE;
-                            mbar_arrive_expect_tx(bar, 2 * L::QKV_TILE + L::BIAS_TILE + 1024);
+                            mbar_arrive_expect_tx(bar, 2 * L::QKV_TILE + 1024);
                             load_pair(base, &tm_q, bar, jt * 128);
                             load_pair(base + L::QKV_TILE, &tm_do, bar, jt * 128);
-                            load_bias(base + 2 * L::QKV_TILE, bar, kt * 128, jt * 128);
-                            load_bias(base + 2 * L::QKV_TILE + L::BIAS_TILE / 2, bar, kt * 128 + 64, jt * 128);
                             bulk_load(sb + L::OFF_VEC + ts * 1024, p.Lv + vrow + jt * 128, 512, bar);
                             bulk_load(sb + L::OFF_VEC + ts * 1024 + 512, p.Dv + vrow + jt * 128, 512, bar);
                         }
@@ -368,6 +353,15 @@ __global__ void __launch_bounds__(384, 1)
             constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);  // Q K^T, dO V^T
             constexpr uint32_t IDESC_G = idesc_bf16_f32(128, D, true, true);      // P^T dO, dS^T Q
             constexpr uint32_t IDESC_Q = idesc_bf16_f32(128, D, false, true);     // dS K
+            // descriptors built once; per-stage / per-step variants are constant adds
+            const uint64_t d_tk = smem_desc(sb + L::OFF_T, 16, SBO, SW);            // Q / dO rows, K-major
+            const uint64_t d_tmn = smem_desc(sb + L::OFF_T, L::QKV_TILE, SBO, SW);  // Q / dO rows, MN-major
+            const uint64_t d_kvk = smem_desc(sb + L::OFF_KV, 16, SBO, SW);          // K / V rows, K-major
+            const uint64_t d_kvmn = smem_desc(sb + L::OFF_KV, L::QKV_TILE, SBO, SW);
+            const uint64_t d_pmn = smem_desc(sb + L::OFF_PDS, L::PT_TILE / 2, 1024, SWZ_128B);
+            const uint64_t d_dsmn = smem_desc(sb + L::OFF_PDS + L::PT_TILE, L::PT_TILE / 2, 1024, SWZ_128B);
+            const uint64_t d_dsk = smem_desc(sb + L::OFF_PDS + L::PT_TILE, 16, 1024, SWZ_128B);
+            TRI_TRACE_DECL
             struct Pending {
                 int g, ts, ks, jt, kt, kcount;
                 bool valid;
@@ -377,41 +371,39 @@ __global__ void __launch_bounds__(384, 1)
             auto issue_grads = [&](const Pending& t) -> bool {
                 // a dQ epilogue tile: every tile (single block) or the last key tile of a query tile
                 const bool ep = !p.dq_tmem || t.kt == nt - 1;
-                if (!mbar_wait(BAR(L::B_PDSFULL), t.g & 1, wc, 3)) return false;
+                TRI_TP(7)
+                const int pb = t.g & 1;  // P/dS buffer of this tile
+                if (!mbar_wait(BAR(L::B_PDSFULL + pb), (t.g >> 1) & 1, wc, 3)) return false;
+                TRI_TP(4)
                 // the previous epilogue has read its dQ block (keeps DQ_FULL at most one phase ahead,
                 // and before a new problem overwrites the last query tile's block)
                 const bool reuse = p.dq_tmem && t.kt == 0 && t.jt == nt - 1;
                 if ((ep || reuse) && ep_count > 0 && !mbar_wait(BAR(L::B_DQFREE), (ep_count - 1) & 1, wc, 4))
                     return false;
+                TRI_TP(5)
                 if (t.jt == 0 && t.kcount > 0 && !mbar_wait(BAR(L::B_DKVFREE), (t.kcount - 1) & 1, wc, 5))
                     return false;
+                TRI_TP(6)
                 tc_fence_after();
-                const uint32_t tb = sb + L::OFF_T + t.ts * L::T_STAGE;
-                const uint32_t qa = tb, doa = tb + L::QKV_TILE;
-                const uint32_t ka = sb + L::OFF_KV + t.ks * 2 * L::QKV_TILE;
-                const uint32_t pa = sb + L::OFF_P, dsa = sb + L::OFF_DS;
+                const uint32_t toff = t.ts * L::T_STAGE;
+                const uint64_t bdo = desc_add(d_tmn, toff + L::QKV_TILE), bq = desc_add(d_tmn, toff);
+                const uint64_t bk = desc_add(d_kvmn, t.ks * 2 * L::QKV_TILE);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {  // contraction over 128 queries
                     const uint32_t acc = (t.jt > 0 || kk > 0) ? 1u : 0u;
                     // A = P^T / dS^T: MN-major, 64-element chunks 16 KB apart, 8-row groups 1 KB apart
-                    const uint64_t adp = smem_desc(pa + kk * 2048, L::PT_TILE / 2, 1024, SWZ_128B);
-                    const uint64_t ads = smem_desc(dsa + kk * 2048, L::PT_TILE / 2, 1024, SWZ_128B);
-                    // B = dO / Q rows j: MN-major over channels
-                    const uint64_t bdo = smem_desc(doa + kk * 16 * L::ROWB, L::QKV_TILE, SBO, SW);
-                    const uint64_t bq = smem_desc(qa + kk * 16 * L::ROWB, L::QKV_TILE, SBO, SW);
-                    mma_ss(tmem + L::T_DV, adp, bdo, IDESC_G, acc);
-                    mma_ss(tmem + L::T_DK, ads, bq, IDESC_G, acc);
+                    mma_ss(tmem + L::T_DV, desc_add(d_pmn, pb * L::PDS_BUF + kk * 2048), desc_add(bdo, kk * 16 * L::ROWB),
+                           IDESC_G, acc);
+                    mma_ss(tmem + L::T_DK, desc_add(d_dsmn, pb * L::PDS_BUF + kk * 2048), desc_add(bq, kk * 16 * L::ROWB),
+                           IDESC_G, acc);
                 }
                 const uint32_t dq_col = p.dq_tmem ? L::T_DQ + t.jt * D : L::T_DQ;
                 const bool dq_acc = p.dq_tmem && t.kt > 0;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {  // contraction over 128 keys
-                    // A = dS rows j: K-major, two 64-key halves 16 KB apart
-                    const uint64_t a = smem_desc(dsa + (kk >> 2) * (L::PT_TILE / 2) + (kk & 3) * 32, 16, 1024, SWZ_128B);
-                    const uint64_t bk = smem_desc(ka + kk * 16 * L::ROWB, L::QKV_TILE, SBO, SW);
-                    mma_ss(tmem + dq_col, a, bk, IDESC_Q, (dq_acc || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(BAR(L::B_PDSFREE));
+                for (int kk = 0; kk < 8; ++kk)  // contraction over 128 keys; A = dS rows j, K-major halves 16 KB apart
+                    mma_ss(tmem + dq_col, desc_add(d_dsk, pb * L::PDS_BUF + (kk >> 2) * (L::PT_TILE / 2) + (kk & 3) * 32),
+                           desc_add(bk, kk * 16 * L::ROWB), IDESC_Q, (dq_acc || kk > 0) ? 1u : 0u);
+                mma_commit(BAR(L::B_PDSFREE + pb));
                 mma_commit(BAR(L::B_TEMPTY + t.ts));
                 if (ep) {
                     mma_commit(BAR(L::B_DQFULL));
@@ -432,23 +424,27 @@ __global__ void __launch_bounds__(384, 1)
                         if (!(ok = issue_grads(pend))) break;
                         pend.valid = false;
                     }
+                    TRI_TP(7)
                     if (!mbar_wait(BAR(L::B_KVFULL + ks), (gk / L::KVS) & 1, wc, 6)) { ok = false; break; }
-                    const uint32_t ka = sb + L::OFF_KV + ks * 2 * L::QKV_TILE;
-                    const uint32_t va = ka + L::QKV_TILE;
+                    TRI_TP(0)
+                    const uint64_t kd = desc_add(d_kvk, ks * 2 * L::QKV_TILE);
+                    const uint64_t vd = desc_add(kd, L::QKV_TILE);
                     for (int jt = 0; jt < nt; ++jt) {
                         const int ts = g % L::NS;
+                        TRI_TP(7)
                         if (!mbar_wait(BAR(L::B_TFULL + ts), (g / L::NS) & 1, wc, 7)) { ok = false; break; }
+                        TRI_TP(1)
                         if (g > 0 && !mbar_wait(BAR(L::B_SDPFREE), (g - 1) & 1, wc, 8)) { ok = false; break; }
+                        TRI_TP(2)
                         tc_fence_after();
-                        const uint32_t tb = sb + L::OFF_T + ts * L::T_STAGE;
+                        const uint64_t qd = desc_add(d_tk, ts * L::T_STAGE), dod = desc_add(qd, L::QKV_TILE);
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
-                            mma_ss(tmem + L::T_S, smem_desc(tb + kk * 32, 16, SBO, SW),
-                                   smem_desc(ka + kk * 32, 16, SBO, SW), IDESC_S, kk > 0 ? 1u : 0u);
-                            mma_ss(tmem + L::T_DP, smem_desc(tb + L::QKV_TILE + kk * 32, 16, SBO, SW),
-                                   smem_desc(va + kk * 32, 16, SBO, SW), IDESC_S, kk > 0 ? 1u : 0u);
+                            mma_ss(tmem + L::T_S, desc_add(qd, kk * 32), desc_add(kd, kk * 32), IDESC_S, kk > 0 ? 1u : 0u);
+                            mma_ss(tmem + L::T_DP, desc_add(dod, kk * 32), desc_add(vd, kk * 32), IDESC_S, kk > 0 ? 1u : 0u);
                         }
                         mma_commit(BAR(L::B_SDPFULL));
+                        TRI_TP(3)
                         if (pend.valid) {
                             if (!(ok = issue_grads(pend))) break;
                         }
@@ -459,6 +455,8 @@ __global__ void __launch_bounds__(384, 1)
                 }
             }
             if (ok && pend.valid) ok = issue_grads(pend);
+            TRI_TP(7)
+            TRI_TRACE_FLUSH_AT(20000)
             mma_commit(BAR(L::B_DRAIN));
             drain_wait(BAR(L::B_DRAIN), 0, 100000000ull);
         }
@@ -581,17 +579,48 @@ __global__ void __launch_bounds__(384, 1)
         };
 
         int gk = 0, g = 0;
+        TRI_TRACE_DECL
         for (int pr = blockIdx.x; ok && pr < problems; pr += gridDim.x) {
             int b, h, i;
             decode(pr, b, h, i);
             for (int kt = 0; ok && kt < nt; ++kt) {
                 const int ks = gk % L::KVS;
                 if (!mbar_wait_warp(BAR(L::B_KVFULL + ks), (gk / L::KVS) & 1, wc, 12)) { ok = false; break; }
+                TRI_TP(9)
                 const bool has_mask = reinterpret_cast<const int*>(smem + L::OFF_FLAGS + ks * 128)[kt] != 0;
                 const uint32_t maskv = sb + L::OFF_MASKV + ks * 512 + w * 256;
                 for (int jt = 0; jt < nt; ++jt) {
                     const int ts = g % L::NS;
+                    // this thread's 64 bias values (row j, keys kt*128 + 64w ..), straight from global
+                    // memory (L2-resident: shared by every row i); issued before the waits below
+                    uint32_t bw[32];
+                    {
+                        const int j = jt * 128 + row;
+                        const int k0 = kt * 128 + w * 64;
+                        const __nv_bfloat16* bp = p.bias + b * p.bs0 + h * p.bs1 + static_cast<int64_t>(j) * p.bs2 + k0;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            uint4 v = make_uint4(0, 0, 0, 0);
+                            if (j < p.N) {
+                                if (k0 + 8 * c + 8 <= p.N) {
+                                    v = __ldg(reinterpret_cast<const uint4*>(bp + 8 * c));
+                                } else if (k0 + 8 * c < p.N) {  // ragged key tail: element loads, zeros past N
+                                    uint16_t e8[8];
+#pragma unroll
+                                    for (int u = 0; u < 8; ++u)
+                                        e8[u] = (k0 + 8 * c + u < p.N) ? __bfloat16_as_ushort(bp[8 * c + u]) : 0;
+                                    v = make_uint4(e8[0] | (e8[1] << 16), e8[2] | (e8[3] << 16), e8[4] | (e8[5] << 16),
+                                                   e8[6] | (static_cast<uint32_t>(e8[7]) << 16));
+                                }
+                            }
+                            bw[4 * c] = v.x;
+                            bw[4 * c + 1] = v.y;
+                            bw[4 * c + 2] = v.z;
+                            bw[4 * c + 3] = v.w;
+                        }
+                    }
                     if (!mbar_wait_warp(BAR(L::B_SDPFULL), g & 1, wc, 13)) { ok = false; break; }
+                    TRI_TP(0)
                     tc_fence_after();
                     uint32_t s0[32], s1[32], d0[32], d1[32];
                     tmem_ld32(tl + L::T_S + w * 64, s0);
@@ -603,37 +632,30 @@ __global__ void __launch_bounds__(384, 1)
                     reg_fence32(s1);
                     reg_fence32(d0);
                     reg_fence32(d1);
+                    TRI_TP(1)
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(BAR(L::B_SDPFREE));
                     if (!mbar_wait_warp(BAR(L::B_TFULL + ts), (g / L::NS) & 1, wc, 14)) { ok = false; break; }
-                    const uint32_t tb = sb + L::OFF_T + ts * L::T_STAGE;
+                    TRI_TP(2)
                     const float* vec = reinterpret_cast<const float*>(smem + L::OFF_VEC + ts * 1024);
                     const float lse2 = vec[row];
                     const float Dj = vec[128 + row];
-                    // bias row j, this warpgroup's 64-key half
-                    const uint32_t brow = tb + 2 * L::QKV_TILE + w * (L::BIAS_TILE / 2) + row * 128;
-                    // P and dS rows go straight into the SW128 K-major tiles (this warpgroup's half)
-                    if (g > 0 && !mbar_wait_warp(BAR(L::B_PDSFREE), (g - 1) & 1, wc, 15)) { ok = false; break; }
-                    const uint32_t prow = sb + L::OFF_P + w * (L::PT_TILE / 2) + row * 128;
-                    const uint32_t drow = sb + L::OFF_DS + w * (L::PT_TILE / 2) + row * 128;
-                    // p = 2^((S*scale + bias)*log2e [+ mask*log2e] - lse*log2e), ds = p (dP - D)
+                    // P and dS of this warpgroup's 64 keys, packed BF16 pairs, computed while the
+                    // previous tile's gradient MMAs still read the shared-memory tiles
+                    uint32_t pw[32], dw[32];
                     const float2 sc2 = make_float2(scale, scale), l2e = make_float2(LOG2E, LOG2E);
                     const float2 nl2 = make_float2(-lse2, -lse2), nD2 = make_float2(-Dj, -Dj);
                     auto tile = [&](auto masked) {
                         constexpr bool kMasked = decltype(masked)::value;
 #pragma unroll
                         for (int c = 0; c < 8; ++c) {
-                            const uint32_t off = (c ^ (row & 7)) << 4;
-                            const uint4 bb = lds128(brow + off);
-                            const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
                             float mk[8];
                             if constexpr (kMasked) {
                                 const float4 m0 = lds128f(maskv + c * 32), m1 = lds128f(maskv + c * 32 + 16);
                                 mk[0] = m0.x; mk[1] = m0.y; mk[2] = m0.z; mk[3] = m0.w;
                                 mk[4] = m1.x; mk[5] = m1.y; mk[6] = m1.z; mk[7] = m1.w;
                             }
-                            uint32_t pw[4], dw[4];
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
                                 const int x0 = c * 8 + 2 * e;
@@ -642,30 +664,42 @@ __global__ void __launch_bounds__(384, 1)
                                 const uint32_t dv0 = (x0 < 32) ? d0[x0] : d1[x0 - 32];
                                 const uint32_t dv1 = (x0 + 1 < 32) ? d0[x0 + 1] : d1[x0 + 1 - 32];
                                 const float2 t = ffma2(make_float2(__uint_as_float(sv0), __uint_as_float(sv1)), sc2,
-                                                       bf16x2_to_f2(bw[e]));
+                                                       bf16x2_to_f2(bw[c * 4 + e]));
                                 float2 y = ffma2(t, l2e, nl2);
                                 if constexpr (kMasked) y = fadd2(y, make_float2(mk[2 * e], mk[2 * e + 1]));
                                 const float p0 = ex2(y.x), p1 = ex2(y.y);
                                 const float2 ds = fmul2(make_float2(p0, p1),
                                                         fadd2(make_float2(__uint_as_float(dv0), __uint_as_float(dv1)), nD2));
-                                const float ds0 = ds.x, ds1 = ds.y;
-                                pw[e] = pack_bf16(p0, p1);
-                                dw[e] = pack_bf16(ds0, ds1);
+                                pw[c * 4 + e] = pack_bf16(p0, p1);
+                                dw[c * 4 + e] = pack_bf16(ds.x, ds.y);
                             }
-                            sts128(prow + off, make_uint4(pw[0], pw[1], pw[2], pw[3]));
-                            sts128(drow + off, make_uint4(dw[0], dw[1], dw[2], dw[3]));
                         }
                     };
                     if (has_mask) tile(std::true_type{});
                     else tile(std::false_type{});
+                    TRI_TP(4)
+                    // the previous tile's gradient MMAs have finished reading P and dS
+                    const int pb = g & 1;  // P/dS buffer of this tile (the other one may still be read)
+                    if (g >= 2 && !mbar_wait_warp(BAR(L::B_PDSFREE + pb), ((g >> 1) - 1) & 1, wc, 15)) { ok = false; break; }
+                    TRI_TP(3)
+                    const uint32_t prow = sb + L::OFF_PDS + pb * L::PDS_BUF + w * (L::PT_TILE / 2) + row * 128;
+                    const uint32_t drow = prow + L::PT_TILE;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint32_t off = (c ^ (row & 7)) << 4;
+                        sts128(prow + off, make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]));
+                        sts128(drow + off, make_uint4(dw[4 * c], dw[4 * c + 1], dw[4 * c + 2], dw[4 * c + 3]));
+                    }
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        mbar_arrive(BAR(L::B_PDSFULL));
+                        mbar_arrive(BAR(L::B_PDSFULL + pb));
                         mbar_arrive(BAR(L::B_TEMPTY + ts));
                         if (jt == nt - 1) mbar_arrive(BAR(L::B_KVEMPTY + ks));
                     }
+                    TRI_TP(5)
                     if (prev.valid && !(ok = epilogue(prev))) break;
+                    TRI_TP(6)
                     prev = Done{g, jt, kt, gk, b, h, i, true};
                     ++g;
                 }
@@ -673,6 +707,8 @@ __global__ void __launch_bounds__(384, 1)
             }
         }
         if (ok && prev.valid) epilogue(prev);
+        TRI_TP(8)
+        TRI_TRACE_FLUSH_AT(20000)
     }
 
     }
@@ -788,12 +824,7 @@ __global__ void __launch_bounds__(384, 1)
                     const int64_t mrow = (static_cast<int64_t>(b) * p.N + i) * p.Np + kt * 128;
                     mbar_arrive_expect_tx(bar, L::STAGE + L::VEC);
                     auto ld = [&](uint32_t dst, const CUtensorMap* m, int row0) {
-                        int c[5] = {0, 0, 0, 0, 0};
-                        c[p.qpos_h] = h;
-                        c[p.qpos_j] = row0;
-                        c[p.qpos_i] = i;
-                        c[p.qpos_b] = b;
-                        tma_load_5d(dst, m, bar, c[0], c[1], c[2], c[3], c[4]);
+                        tma_load_5d(dst, m, bar, 0, h, row0, i, b);
                     };
                     ld(base, &tm_q, jt * 128);
                     ld(base + L::QKV_TILE, &tm_do, jt * 128);
@@ -818,22 +849,29 @@ __global__ void __launch_bounds__(384, 1)
             constexpr uint32_t SW = (D == 32) ? SWZ_64B : SWZ_128B;
             constexpr uint32_t SBO = 8 * L::ROWB;
             constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
+            const uint64_t d0 = smem_desc(sb, 16, SBO, SW);
+            TRI_TRACE_DECL
             for (int n = 0; n < nrows; ++n) {
                 const int s = n % L::NS, x = n & 1;
+                TRI_TP(2)
                 if (!mbar_wait(BAR(L::B_FULL + s), (n / L::NS) & 1, wc, 2)) break;
+                TRI_TP(0)
                 if (n >= 2 && !mbar_wait(BAR(L::B_SDPFREE + x), ((n >> 1) - 1) & 1, wc, 3)) break;
+                TRI_TP(1)
                 tc_fence_after();
-                const uint32_t base = sb + s * L::STAGE;
+                const uint64_t qd = desc_add(d0, s * L::STAGE);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    mma_ss(tmem + x * 256, smem_desc(base + kk * 32, 16, SBO, SW),
-                           smem_desc(base + 2 * L::QKV_TILE + kk * 32, 16, SBO, SW), IDESC_S, kk > 0 ? 1u : 0u);
-                    mma_ss(tmem + x * 256 + 128, smem_desc(base + L::QKV_TILE + kk * 32, 16, SBO, SW),
-                           smem_desc(base + 3 * L::QKV_TILE + kk * 32, 16, SBO, SW), IDESC_S, kk > 0 ? 1u : 0u);
+                    mma_ss(tmem + x * 256, desc_add(qd, kk * 32), desc_add(qd, 2 * L::QKV_TILE + kk * 32), IDESC_S,
+                           kk > 0 ? 1u : 0u);
+                    mma_ss(tmem + x * 256 + 128, desc_add(qd, L::QKV_TILE + kk * 32),
+                           desc_add(qd, 3 * L::QKV_TILE + kk * 32), IDESC_S, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(BAR(L::B_SDPFULL + x));
                 mma_commit(BAR(L::B_EMPTY + s));
             }
+            TRI_TP(2)
+            TRI_TRACE_FLUSH_AT(30000)
             mma_commit(BAR(L::B_DRAIN));
             drain_wait(BAR(L::B_DRAIN), 0, 100000000ull);
         }
@@ -870,9 +908,11 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int e = 0; e < 64; ++e) acc[e] = 0.f;
         bool ok = true;
+        TRI_TRACE_DECL
         for (int n = 0; n < nrows; ++n) {
             const int x = n & 1, s = n % L::NS;
             if (!mbar_wait_warp(BAR(L::B_SDPFULL + x), (n >> 1) & 1, wc, 4)) { ok = false; break; }
+            TRI_TP(0)
             tc_fence_after();
             if (!mbar_wait_warp(BAR(L::B_FULL + s), (n / L::NS) & 1, wc, 5)) { ok = false; break; }
             const float* vec = reinterpret_cast<const float*>(smem + L::OFF_VEC + s * L::VEC);
@@ -881,6 +921,7 @@ __global__ void __launch_bounds__(384, 1)
             const bool has_mask = reinterpret_cast<const int*>(vec + 384)[kt] != 0;
             const uint32_t ma = sb + L::OFF_VEC + s * L::VEC + 1024 + w * 256;
             const float2 c22 = make_float2(c2, c2), nl2 = make_float2(-lse2, -lse2), nD2 = make_float2(-Dj, -Dj);
+            TRI_TP(1)
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t sv[32], dv[32];
@@ -918,9 +959,11 @@ __global__ void __launch_bounds__(384, 1)
                     }
                 }
             }
+            TRI_TP(2)
             __syncwarp();
             if (lane == 0) mbar_arrive(BAR(L::B_EMPTY + s));
         }
+        TRI_TP(3)
         if (ok && j < p.N) {
             const int k0 = kt * 128 + w * 64;
             if (p.chunks == 1) {
@@ -947,6 +990,8 @@ __global__ void __launch_bounds__(384, 1)
                     if (k0 + e < p.N) dst[e] = acc[e];
             }
         }
+        TRI_TP(4)
+        TRI_TRACE_FLUSH_AT(30000)
     }
 
     }

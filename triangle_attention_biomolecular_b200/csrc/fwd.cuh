@@ -36,10 +36,6 @@ namespace tri {
 struct FwdParams {
     int B, N, H, nt, npairs;
     float scale;
-    // positions (1..4) of the h, j, i, b coordinates in the Q/K/V tensor maps
-    int qpos_h, qpos_j, qpos_i, qpos_b;
-    // positions (1..3) of the j, h, b coordinates in the bias tensor map
-    int bpos_j, bpos_h, bpos_b;
     const float* mask;
     int64_t ms0, ms1, ms2;
     __nv_bfloat16* o;
@@ -156,20 +152,10 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int s = 0; s < L::NS; ++s) armed[s] = 0;
         auto load_qkv = [&](uint32_t dst, const CUtensorMap* m, uint32_t bar, int i, int j0) {
-            int c[5] = {0, 0, 0, 0, 0};
-            c[p.qpos_h] = h;
-            c[p.qpos_j] = j0;
-            c[p.qpos_i] = i;
-            c[p.qpos_b] = b;
-            tma_load_5d(dst, m, bar, c[0], c[1], c[2], c[3], c[4]);
+            tma_load_5d(dst, m, bar, 0, h, j0, i, b);
         };
         auto load_bias = [&](uint32_t dst, uint32_t bar, int k0, int j0) {
-            int c[4] = {0, 0, 0, 0};
-            c[0] = k0;
-            c[p.bpos_j] = j0;
-            c[p.bpos_h] = h;
-            c[p.bpos_b] = b;
-            tma_load_4d(dst, &tm_bias, bar, c[0], c[1], c[2], c[3]);
+            tma_load_4d(dst, &tm_bias, bar, k0, j0, h, b);
         };
         if (!aborted_early) {
             if (lane == 0) {
@@ -197,10 +183,13 @@ __global__ void __launch_bounds__(384, 1)
                     }
                 }
             };
+            TRI_TRACE_DECL
             fetch_mask(0);
             for (int kt = 0; kt < nkt; ++kt) {
                 const int s = kt % L::NS;
+                TRI_TP(1)
                 if (kt >= L::NS && !mbar_wait_warp(BAR(L::B_EMPTY + s), ((kt / L::NS) - 1) & 1, wc, 1)) break;
+                TRI_TP(0)
                 const uint32_t st = sb + L::OFF_STAGES + s * L::STAGE;
 #pragma unroll
                 for (int w = 0; w < 2; ++w) {
@@ -226,6 +215,8 @@ __global__ void __launch_bounds__(384, 1)
                 armed[s]++;
                 if (kt + 1 < nkt) fetch_mask(kt + 1);
             }
+            TRI_TP(1)
+            TRI_TRACE_FLUSH_AT(0)
         }
         // never leave with bulk copies still writing into this CTA's shared memory
         if (lane == 0) {
@@ -242,43 +233,52 @@ __global__ void __launch_bounds__(384, 1)
             constexpr uint32_t SBO = 8 * L::ROWB;
             constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false, false);
             constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
-            auto issue_pv = [&](int w, uint32_t stage, int ktile) {
-                const uint32_t va = stage + (w ? L::OFF_V1 : L::OFF_V0);
+            // descriptors built once; per-stage / per-step variants are constant adds
+            const uint64_t dq0 = smem_desc(sb + L::OFF_Q, 16, SBO, SW);
+            const uint64_t dst0 = smem_desc(sb + L::OFF_STAGES, 16, SBO, SW);          // K-major rows
+            const uint64_t dvt0 = smem_desc(sb + L::OFF_STAGES, L::QKV_TILE, SBO, SW);  // MN-major rows
+            auto issue_pv = [&](int w, int s, int ktile) {
+                const uint64_t vd = desc_add(dvt0, s * L::STAGE + (w ? L::OFF_V1 : L::OFF_V0));
                 const uint32_t tS = tmem + w * 256;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tS + 192, tS + 128 + kk * 8, smem_desc(va + kk * 16 * L::ROWB, L::QKV_TILE, SBO, SW),
-                           IDESC_PV, (ktile > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts(tS + 192, tS + 128 + kk * 8, desc_add(vd, kk * 16 * L::ROWB), IDESC_PV,
+                           (ktile > 0 || kk > 0) ? 1u : 0u);
             };
+            TRI_TRACE_DECL
             bool ok = mbar_wait(BAR(L::B_Q), 0, wc, 2);
+            TRI_TP(9)
             for (int kt = 0; ok && kt < nkt; ++kt) {
                 const int s = kt % L::NS;
+                TRI_TP(4)
                 if (!mbar_wait(BAR(L::B_FULL + s), (kt / L::NS) & 1, wc, 3)) { ok = false; break; }
+                TRI_TP(0)
                 tc_fence_after();
-                const uint32_t st = sb + L::OFF_STAGES + s * L::STAGE;
 #pragma unroll
                 for (int w = 0; w < 2; ++w) {
                     if (kt > 0) {
+                        TRI_TP(4)
                         if (!mbar_wait(BAR(L::B_SFREE + w), (kt - 1) & 1, wc, 4)) { ok = false; break; }
+                        TRI_TP(1)
                         tc_fence_after();
                     }
-                    const uint32_t qa = sb + L::OFF_Q + w * L::QKV_TILE;
-                    const uint32_t ka = st + (w ? L::OFF_K1 : L::OFF_K0);
+                    const uint64_t qd = desc_add(dq0, w * L::QKV_TILE);
+                    const uint64_t kd = desc_add(dst0, s * L::STAGE + (w ? L::OFF_K1 : L::OFF_K0));
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk)
-                        mma_ss(tmem + w * 256, smem_desc(qa + kk * 32, 16, SBO, SW),
-                               smem_desc(ka + kk * 32, 16, SBO, SW), IDESC_QK, kk > 0 ? 1u : 0u);
+                        mma_ss(tmem + w * 256, desc_add(qd, kk * 32), desc_add(kd, kk * 32), IDESC_QK, kk > 0 ? 1u : 0u);
                     mma_commit(BAR(L::B_SFULL + w));
                 }
                 if (!ok) break;
                 if (kt > 0) {
                     const int sp = (kt - 1) % L::NS;
-                    const uint32_t pst = sb + L::OFF_STAGES + sp * L::STAGE;
 #pragma unroll
                     for (int w = 0; w < 2; ++w) {
+                        TRI_TP(4)
                         if (!mbar_wait(BAR(L::B_PFULL + w), (kt - 1) & 1, wc, 5)) { ok = false; break; }
+                        TRI_TP(2)
                         tc_fence_after();
-                        issue_pv(w, pst, kt - 1);
+                        issue_pv(w, sp, kt - 1);
                         mma_commit(BAR(L::B_PVDONE + w));
                     }
                     if (!ok) break;
@@ -288,16 +288,17 @@ __global__ void __launch_bounds__(384, 1)
             if (ok) {
                 const int kl = nkt - 1;
                 const int sp = kl % L::NS;
-                const uint32_t pst = sb + L::OFF_STAGES + sp * L::STAGE;
 #pragma unroll
                 for (int w = 0; w < 2; ++w) {
                     if (!mbar_wait(BAR(L::B_PFULL + w), kl & 1, wc, 5)) { ok = false; break; }
                     tc_fence_after();
-                    issue_pv(w, pst, kl);
+                    issue_pv(w, sp, kl);
                     mma_commit(BAR(L::B_PVDONE + w));
                 }
                 if (ok) mma_commit(BAR(L::B_EMPTY + sp));
             }
+            TRI_TP(5)
+            TRI_TRACE_FLUSH_AT(0)
             // every MMA this thread issued has completed before the CTA leaves
             mma_commit(BAR(L::B_DRAIN));
             drain_wait(BAR(L::B_DRAIN), 0, 100000000ull);
@@ -321,9 +322,11 @@ __global__ void __launch_bounds__(384, 1)
         constexpr float RESCALE_AT = 5.545177444479562f;  // 8 * ln 2
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
+        TRI_TRACE_DECL
         for (int kt = 0; kt < nkt; ++kt) {
             const int s = kt % L::NS;
             if (!mbar_wait_warp(BAR(L::B_SFULL + w), kt & 1, wc, 6)) { ok = false; break; }
+            if (kt == 0) { TRI_TP(9) } else { TRI_TP(0) }
             tc_fence_after();
             uint32_t r0[32], r1[32], r2[32], r3[32];
             tmem_ld32(tS + 0, r0);
@@ -335,10 +338,12 @@ __global__ void __launch_bounds__(384, 1)
             reg_fence32(r1);
             reg_fence32(r2);
             reg_fence32(r3);
+            TRI_TP(1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(BAR(L::B_SFREE + w));
             if (!mbar_wait_warp(BAR(L::B_FULL + s), (kt / L::NS) & 1, wc, 7)) { ok = false; break; }
+            TRI_TP(2)
             const uint32_t st = sb + L::OFF_STAGES + s * L::STAGE;
             float x[128];
 #pragma unroll
@@ -388,6 +393,7 @@ __global__ void __launch_bounds__(384, 1)
                 ma3 = fmax3(ma3, x[e + 6], x[e + 7]);
             }
             const float mt = fmaxf(fmaxf(ma0, ma1), fmaxf(ma2, ma3));
+            TRI_TP(3)
             bool need = false;
             float alpha = 1.f;
             if (kt == 0) {
@@ -399,32 +405,39 @@ __global__ void __launch_bounds__(384, 1)
                 l *= alpha;
             }
             const float mb = fmaxf(m_ref, -3.0e38f) * LOG2E;
+            // probabilities into packed BF16 registers first; the previous PV may still be
+            // reading the P columns
+            const float2 l2e = make_float2(LOG2E, LOG2E), nmb = make_float2(-mb, -mb);
+            float2 ls0 = make_float2(0.f, 0.f), ls1 = ls0, ls2 = ls0, ls3 = ls0;
+            uint32_t pk[64];
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                const float2 a2 = ffma2(make_float2(x[2 * c], x[2 * c + 1]), l2e, nmb);
+                const float2 pp = make_float2(ex2(a2.x), ex2(a2.y));
+                switch (c & 3) {
+                    case 0: ls0 = fadd2(ls0, pp); break;
+                    case 1: ls1 = fadd2(ls1, pp); break;
+                    case 2: ls2 = fadd2(ls2, pp); break;
+                    default: ls3 = fadd2(ls3, pp); break;
+                }
+                pk[c] = pack_bf16(pp.x, pp.y);
+            }
+            const float2 lsum = fadd2(fadd2(ls0, ls1), fadd2(ls2, ls3));
+            const float ls = lsum.x + lsum.y;
+            TRI_TP(5)
             if (kt > 0) {
                 // PV of the previous tile has finished: the P columns are free and O is stable
                 if (!mbar_wait_warp(BAR(L::B_PVDONE + w), (kt - 1) & 1, wc, 8)) { ok = false; break; }
                 tc_fence_after();
             }
-            const float2 l2e = make_float2(LOG2E, LOG2E), nmb = make_float2(-mb, -mb);
-            float2 ls0 = make_float2(0.f, 0.f), ls1 = ls0, ls2 = ls0, ls3 = ls0;
+            TRI_TP(4)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                uint32_t pk[16];
+                uint32_t pq[16];
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    const float2 a2 = ffma2(make_float2(x[32 * q + 2 * c], x[32 * q + 2 * c + 1]), l2e, nmb);
-                    const float2 pp = make_float2(ex2(a2.x), ex2(a2.y));
-                    switch (c & 3) {
-                        case 0: ls0 = fadd2(ls0, pp); break;
-                        case 1: ls1 = fadd2(ls1, pp); break;
-                        case 2: ls2 = fadd2(ls2, pp); break;
-                        default: ls3 = fadd2(ls3, pp); break;
-                    }
-                    pk[c] = pack_bf16(pp.x, pp.y);
-                }
-                tmem_st16(tP + 16 * q, pk);
+                for (int c = 0; c < 16; ++c) pq[c] = pk[16 * q + c];
+                tmem_st16(tP + 16 * q, pq);
             }
-            const float2 lsum = fadd2(fadd2(ls0, ls1), fadd2(ls2, ls3));
-            const float ls = lsum.x + lsum.y;
             l += ls;
             if (kt > 0 && __any_sync(0xFFFFFFFFu, need)) {
                 // rare: the reference maximum moved, rescale this row of O before the next PV
@@ -443,6 +456,7 @@ __global__ void __launch_bounds__(384, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(BAR(L::B_PFULL + w));
+            TRI_TP(7)
         }
         if (ok && mbar_wait_warp(BAR(L::B_PVDONE + w), (nkt - 1) & 1, wc, 9)) {
             tc_fence_after();
@@ -478,6 +492,8 @@ __global__ void __launch_bounds__(384, 1)
                     m_ref + lg2(l) * 0.6931471805599453f;
             }
         }
+        TRI_TP(8)
+        TRI_TRACE_FLUSH_AT(0)
     }
 
     }

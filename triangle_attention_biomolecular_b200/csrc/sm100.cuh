@@ -19,6 +19,34 @@ namespace tri {
 // ---------------------------------------------------------------------------
 __device__ uint32_t g_error_word;
 
+// Optional phase timing (instrumentation only; compiled out unless TRI_TRACE is
+// defined): each warp accumulates clock64() cycles per phase and lane 0 writes
+// them to a buffer of [blocks][12 warps][16 phases].
+#ifdef TRI_TRACE
+__device__ unsigned long long* g_trace;
+#define TRI_TRACE_DECL                                  \
+    unsigned long long tri_acc_[16];                    \
+    for (int tri_q_ = 0; tri_q_ < 16; ++tri_q_) tri_acc_[tri_q_] = 0; \
+    unsigned long long tri_last_ = clock64();
+#define TRI_TP(p)                                       \
+    {                                                   \
+        const unsigned long long tri_t_ = clock64();    \
+        tri_acc_[p] += tri_t_ - tri_last_;              \
+        tri_last_ = tri_t_;                             \
+    }
+#define TRI_TRACE_FLUSH_AT(base)                                                                          \
+    {                                                                                                     \
+        if (g_trace && (threadIdx.x & 31) == 0)                                                           \
+            for (int tri_q_ = 0; tri_q_ < 16; ++tri_q_)                                                   \
+                g_trace[(static_cast<size_t>(blockIdx.x + (base)) * 12 + (threadIdx.x >> 5)) * 16 + tri_q_] =  \
+                    tri_acc_[tri_q_];                                                                     \
+    }
+#else
+#define TRI_TRACE_DECL
+#define TRI_TP(p)
+#define TRI_TRACE_FLUSH_AT(base)
+#endif
+
 // site codes: high byte = kernel, low bits = wait site
 enum : uint32_t {
     ERR_TIMEOUT_BIT = 0x80000000u,
@@ -212,6 +240,10 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
            (static_cast<uint64_t>(swizzle) << 61);
 }
 
+// A descriptor advanced by a byte offset (start-address field, 16-byte units; the
+// field never carries because shared-memory addresses stay below 256 KB).
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t byte_offset) { return desc + (byte_offset >> 4); }
+
 // TMEM loads/stores, shape 32x32b: each thread of the warp moves consecutive
 // 32-bit columns of its own TMEM lane.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
@@ -261,9 +293,10 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 // Register rebalancing between warpgroups.  Kernels launch 384 threads
 // (168 registers each, 64512 total); the producer/MMA warpgroup gives up
 // registers and the two softmax warpgroups take them:
-// 128 * 56 + 256 * 224 = 64512, exactly the launch total.
-constexpr int kRegsLaunch = 168, kRegsSmall = 56, kRegsLarge = 224;
-static_assert(128 * kRegsSmall + 256 * kRegsLarge == 384 * kRegsLaunch, "register split must match the launch");
+// 128 * 88 + 256 * 208 = 64512, exactly the launch total.
+constexpr int kRegsLaunch = 168, kRegsSmall = 88, kRegsLarge = 208;
+static_assert(128 * kRegsSmall + 256 * kRegsLarge <= 384 * kRegsLaunch && kRegsSmall % 8 == 0 && kRegsLarge % 8 == 0,
+              "register split must fit the launch total");
 __device__ __forceinline__ void regs_shrink() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSmall)); }
 __device__ __forceinline__ void regs_grow() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsLarge)); }
 // every role of the CTA meets here before tensor memory is released
