@@ -76,8 +76,11 @@ typedef enum {
     TRI_ATTN_ERR_WORKSPACE = 7,      /* workspace NULL or smaller than required        */
     TRI_ATTN_ERR_ARCH = 8,           /* current device is not sm_100                   */
     TRI_ATTN_ERR_CUDA = 9,           /* a CUDA runtime/driver call failed              */
-    TRI_ATTN_ERR_DEVICE_TIMEOUT = 10 /* a kernel's bounded wait expired (see
+    TRI_ATTN_ERR_DEVICE_TIMEOUT = 10, /* a kernel's bounded wait expired (see
                                         tri_attn_device_error)                        */
+    TRI_ATTN_ERR_SCRATCH_LIMIT = 11  /* the sizes need more scratch than
+                                        TRI_ATTN_STATIC_SCRATCH_BYTES (only from
+                                        tri_attn_bwd_static_scratch)                 */
 } tri_attn_status;
 
 /* BF16 pair tensor [B,N,N,H,d]; stride[] = element strides of (b,i,j,h,c), c-stride 1. */
@@ -164,6 +167,39 @@ tri_attn_status tri_attn_bwd(const tri_attn_bwd_args *args, tri_attn_stream_t st
  * owns.  Otherwise identical to tri_attn_bwd. */
 tri_attn_status tri_attn_bwd_marked(const tri_attn_bwd_args *args, tri_attn_stream_t stream,
                                     void *const *markers);
+
+/* Size of the static scratch area of tri_attn_bwd_static_scratch, per device:
+ * 64 MiB, enough for every size whose tri_attn_bwd_workspace_bytes is at most
+ * that (for example B=1, N=768, H=4 at d=32 or d=64). */
+#define TRI_ATTN_STATIC_SCRATCH_BYTES (64ull << 20)
+
+/*
+ * The backward without any device allocation.  The method's pages have no
+ * counterpart to this: it is a service of the library, for callers that must
+ * not allocate device memory on the path where the backward runs (an
+ * application whose allocator owns all device memory, or a latency-critical
+ * loop where cudaMalloc / cudaFree, which can synchronise the device, are not
+ * allowed).  It runs exactly the kernels of tri_attn_bwd and returns the same
+ * results, but its scratch is a fixed array of TRI_ATTN_STATIC_SCRATCH_BYTES
+ * in the library's own device memory, reserved when the library's module for
+ * it is loaded onto a device; args->workspace and args->workspace_bytes are
+ * ignored.
+ *   - Limit: sizes whose tri_attn_bwd_workspace_bytes(B,N,H,d) exceeds
+ *     TRI_ATTN_STATIC_SCRATCH_BYTES are rejected with
+ *     TRI_ATTN_ERR_SCRATCH_LIMIT before anything is enqueued.
+ *   - Set-up: the first call on each device (the current device at the call)
+ *     looks up the array's device address, which loads the module there; call
+ *     it once on each device before any stream capture begins, so that this
+ *     set-up happens outside a capture.
+ *   - Initial contents: nothing in the scratch has to start at zero; every
+ *     word the kernels read is written earlier in the same call.
+ *   - Races: all calls on one device share the one array.  Two calls whose
+ *     work can overlap on the device (different streams without an ordering
+ *     event between them, or several host threads) race on it and produce
+ *     wrong gradients; order them, for example on one stream.
+ * Otherwise the same arguments and error rules as tri_attn_bwd.
+ */
+tri_attn_status tri_attn_bwd_static_scratch(const tri_attn_bwd_args *args, tri_attn_stream_t stream);
 
 /* Static, NUL-terminated description of a status code. */
 const char *tri_attn_strerror(tri_attn_status status);

@@ -26,6 +26,8 @@ TRI_ATTN_ERR_WORKSPACE = 7
 TRI_ATTN_ERR_ARCH = 8
 TRI_ATTN_ERR_CUDA = 9
 TRI_ATTN_ERR_DEVICE_TIMEOUT = 10
+TRI_ATTN_ERR_SCRATCH_LIMIT = 11
+TRI_ATTN_STATIC_SCRATCH_BYTES = 64 << 20
 TRI_ATTN_BWD_NO_RESIDUAL = 1
 
 
@@ -82,6 +84,8 @@ def load() -> ctypes.CDLL:
             lib.tri_attn_bwd_marked.argtypes = [ctypes.POINTER(BwdArgs), ctypes.c_void_p,
                                                 ctypes.POINTER(ctypes.c_void_p)]
             lib.tri_attn_bwd_marked.restype = ctypes.c_int
+            lib.tri_attn_bwd_static_scratch.argtypes = [ctypes.POINTER(BwdArgs), ctypes.c_void_p]
+            lib.tri_attn_bwd_static_scratch.restype = ctypes.c_int
             lib.tri_attn_bwd_workspace_bytes.argtypes = [ctypes.c_int] * 4
             lib.tri_attn_bwd_workspace_bytes.restype = ctypes.c_size_t
             lib.tri_attn_strerror.argtypes = [ctypes.c_int]
@@ -241,6 +245,17 @@ def tri_attn_bwd_marked(q, k, v, bias, mask, o, resid, lse, dout, dq, dk, dv, db
     st = load().tri_attn_bwd_marked(ctypes.byref(a), _stream_handle(stream), arr)
     if st != TRI_ATTN_OK:
         raise TriAttnError(st, "tri_attn_bwd_marked")
+
+
+def tri_attn_bwd_static_scratch(q, k, v, bias, mask, o, resid, lse, dout, dq, dk, dv, dbias,
+                                scale: float = 0.0, flags: int = 0, stream=None) -> None:
+    """tri_attn_bwd without a workspace argument: the library's fixed per-device
+    scratch array is used instead, so nothing is allocated.  Calls on one device
+    share that array and must not overlap on the device."""
+    a = bwd_args(q, k, v, bias, mask, o, resid, lse, dout, dq, dk, dv, dbias, None, scale, flags)
+    st = load().tri_attn_bwd_static_scratch(ctypes.byref(a), _stream_handle(stream))
+    if st != TRI_ATTN_OK:
+        raise TriAttnError(st, "tri_attn_bwd_static_scratch")
 
 
 def tri_attn_device_error(clear: bool = True):

@@ -313,6 +313,7 @@ const char* tri_attn_strerror(tri_attn_status s) {
         case TRI_ATTN_ERR_ARCH: return "current device is not compute capability 10.0 (sm_100)";
         case TRI_ATTN_ERR_CUDA: return "a CUDA call failed";
         case TRI_ATTN_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel expired";
+        case TRI_ATTN_ERR_SCRATCH_LIMIT: return "sizes need more scratch than the 64 MiB static scratch area holds";
     }
     return "unknown status";
 }
