@@ -280,8 +280,9 @@ __global__ void __launch_bounds__(384, 1)
         for (int s = 0; s < L::KVS; ++s) armed_kv[s] = 0;
 #pragma unroll
         for (int s = 0; s < L::NS; ++s) armed_t[s] = 0;
+        const bool leader = elect_one();
         if (!aborted_early) {
-            if (lane == 0) {
+            if (leader) {
                 tma_prefetch_map(&tm_q);
                 tma_prefetch_map(&tm_k);
                 tma_prefetch_map(&tm_v);
@@ -304,7 +305,7 @@ __global__ void __launch_bounds__(384, 1)
                         ok = false;
                         break;
                     }
-                    if (lane == 0) {
+                    if (leader) {
                         const uint32_t bar = BAR(L::B_KVFULL + ks);
                         const uint32_t base = sb + L::OFF_KV + ks * 2 * L::QKV_TILE;
                         mbar_arrive_expect_tx(bar, 2 * L::QKV_TILE + 512 + 128);
@@ -321,7 +322,7 @@ __global__ void __launch_bounds__(384, 1)
                             ok = false;
                             break;
                         }
-                        if (lane == 0) {
+                        if (leader) {
                             const uint32_t bar = BAR(L::B_TFULL + ts);
                             const uint32_t base = sb + L::OFF_T + ts * L::T_STAGE;
                             mbar_arrive_expect_tx(bar, 2 * L::QKV_TILE + 1024);
@@ -336,7 +337,7 @@ __global__ void __launch_bounds__(384, 1)
                 }
             }
         }
-        if (lane == 0) {
+        if (leader) {
 #pragma unroll
             for (int s = 0; s < L::KVS; ++s)
                 if (armed_kv[s] > 0) drain_wait(BAR(L::B_KVFULL + s), (armed_kv[s] - 1) & 1, 100000000ull);
@@ -347,7 +348,8 @@ __global__ void __launch_bounds__(384, 1)
     } else if (warp == 9) {
         // =========================== MMA issuer =============================
         regs_shrink();
-        if (lane == 0 && !aborted_early) {
+        const bool leader = elect_one();
+        if (!aborted_early) {
             constexpr uint32_t SW = (D == 32) ? SWZ_64B : SWZ_128B;
             constexpr uint32_t SBO = 8 * L::ROWB;
             constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);  // Q K^T, dO V^T
@@ -373,21 +375,24 @@ __global__ void __launch_bounds__(384, 1)
                 const bool ep = !p.dq_tmem || t.kt == nt - 1;
                 TRI_TP(7)
                 const int pb = t.g & 1;  // P/dS buffer of this tile
-                if (!mbar_wait(BAR(L::B_PDSFULL + pb), (t.g >> 1) & 1, wc, 3)) return false;
+                if (!mbar_wait_warp(BAR(L::B_PDSFULL + pb), (t.g >> 1) & 1, wc, 3)) return false;
                 TRI_TP(4)
                 // the previous epilogue has read its dQ block (keeps DQ_FULL at most one phase ahead,
                 // and before a new problem overwrites the last query tile's block)
                 const bool reuse = p.dq_tmem && t.kt == 0 && t.jt == nt - 1;
-                if ((ep || reuse) && ep_count > 0 && !mbar_wait(BAR(L::B_DQFREE), (ep_count - 1) & 1, wc, 4))
+                if ((ep || reuse) && ep_count > 0 && !mbar_wait_warp(BAR(L::B_DQFREE), (ep_count - 1) & 1, wc, 4))
                     return false;
                 TRI_TP(5)
-                if (t.jt == 0 && t.kcount > 0 && !mbar_wait(BAR(L::B_DKVFREE), (t.kcount - 1) & 1, wc, 5))
+                if (t.jt == 0 && t.kcount > 0 && !mbar_wait_warp(BAR(L::B_DKVFREE), (t.kcount - 1) & 1, wc, 5))
                     return false;
                 TRI_TP(6)
                 tc_fence_after();
                 const uint32_t toff = t.ts * L::T_STAGE;
                 const uint64_t bdo = desc_add(d_tmn, toff + L::QKV_TILE), bq = desc_add(d_tmn, toff);
                 const uint64_t bk = desc_add(d_kvmn, t.ks * 2 * L::QKV_TILE);
+                const uint32_t dq_col = p.dq_tmem ? L::T_DQ + t.jt * D : L::T_DQ;
+                const bool dq_acc = p.dq_tmem && t.kt > 0;
+                if (leader) {
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {  // contraction over 128 queries
                     const uint32_t acc = (t.jt > 0 || kk > 0) ? 1u : 0u;
@@ -397,22 +402,20 @@ __global__ void __launch_bounds__(384, 1)
                     mma_ss(tmem + L::T_DK, desc_add(d_dsmn, pb * L::PDS_BUF + kk * 2048), desc_add(bq, kk * 16 * L::ROWB),
                            IDESC_G, acc);
                 }
-                const uint32_t dq_col = p.dq_tmem ? L::T_DQ + t.jt * D : L::T_DQ;
-                const bool dq_acc = p.dq_tmem && t.kt > 0;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)  // contraction over 128 keys; A = dS rows j, K-major halves 16 KB apart
                     mma_ss(tmem + dq_col, desc_add(d_dsk, pb * L::PDS_BUF + (kk >> 2) * (L::PT_TILE / 2) + (kk & 3) * 32),
                            desc_add(bk, kk * 16 * L::ROWB), IDESC_Q, (dq_acc || kk > 0) ? 1u : 0u);
                 mma_commit(BAR(L::B_PDSFREE + pb));
                 mma_commit(BAR(L::B_TEMPTY + t.ts));
-                if (ep) {
-                    mma_commit(BAR(L::B_DQFULL));
-                    ++ep_count;
-                }
+                if (ep) mma_commit(BAR(L::B_DQFULL));
                 if (t.jt == nt - 1) {
                     mma_commit(BAR(L::B_DKVFULL));
                     mma_commit(BAR(L::B_KVEMPTY + t.ks));
                 }
+                }
+                __syncwarp();
+                if (ep) ++ep_count;
                 return true;
             };
             int gk = 0, g = 0;
@@ -425,25 +428,28 @@ __global__ void __launch_bounds__(384, 1)
                         pend.valid = false;
                     }
                     TRI_TP(7)
-                    if (!mbar_wait(BAR(L::B_KVFULL + ks), (gk / L::KVS) & 1, wc, 6)) { ok = false; break; }
+                    if (!mbar_wait_warp(BAR(L::B_KVFULL + ks), (gk / L::KVS) & 1, wc, 6)) { ok = false; break; }
                     TRI_TP(0)
                     const uint64_t kd = desc_add(d_kvk, ks * 2 * L::QKV_TILE);
                     const uint64_t vd = desc_add(kd, L::QKV_TILE);
                     for (int jt = 0; jt < nt; ++jt) {
                         const int ts = g % L::NS;
                         TRI_TP(7)
-                        if (!mbar_wait(BAR(L::B_TFULL + ts), (g / L::NS) & 1, wc, 7)) { ok = false; break; }
+                        if (!mbar_wait_warp(BAR(L::B_TFULL + ts), (g / L::NS) & 1, wc, 7)) { ok = false; break; }
                         TRI_TP(1)
-                        if (g > 0 && !mbar_wait(BAR(L::B_SDPFREE), (g - 1) & 1, wc, 8)) { ok = false; break; }
+                        if (g > 0 && !mbar_wait_warp(BAR(L::B_SDPFREE), (g - 1) & 1, wc, 8)) { ok = false; break; }
                         TRI_TP(2)
                         tc_fence_after();
                         const uint64_t qd = desc_add(d_tk, ts * L::T_STAGE), dod = desc_add(qd, L::QKV_TILE);
+                        if (leader) {
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            mma_ss(tmem + L::T_S, desc_add(qd, kk * 32), desc_add(kd, kk * 32), IDESC_S, kk > 0 ? 1u : 0u);
-                            mma_ss(tmem + L::T_DP, desc_add(dod, kk * 32), desc_add(vd, kk * 32), IDESC_S, kk > 0 ? 1u : 0u);
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                mma_ss(tmem + L::T_S, desc_add(qd, kk * 32), desc_add(kd, kk * 32), IDESC_S, kk > 0 ? 1u : 0u);
+                                mma_ss(tmem + L::T_DP, desc_add(dod, kk * 32), desc_add(vd, kk * 32), IDESC_S, kk > 0 ? 1u : 0u);
+                            }
+                            mma_commit(BAR(L::B_SDPFULL));
                         }
-                        mma_commit(BAR(L::B_SDPFULL));
+                        __syncwarp();
                         TRI_TP(3)
                         if (pend.valid) {
                             if (!(ok = issue_grads(pend))) break;
@@ -457,7 +463,8 @@ __global__ void __launch_bounds__(384, 1)
             if (ok && pend.valid) ok = issue_grads(pend);
             TRI_TP(7)
             TRI_TRACE_FLUSH_AT(20000)
-            mma_commit(BAR(L::B_DRAIN));
+            if (leader) mma_commit(BAR(L::B_DRAIN));
+            __syncwarp();
             drain_wait(BAR(L::B_DRAIN), 0, 100000000ull);
         }
         __syncwarp();
@@ -805,8 +812,9 @@ __global__ void __launch_bounds__(384, 1)
         int armed[L::NS];
 #pragma unroll
         for (int s = 0; s < L::NS; ++s) armed[s] = 0;
+        const bool leader = elect_one();
         if (!aborted_early) {
-            if (lane == 0) {
+            if (leader) {
                 tma_prefetch_map(&tm_q);
                 tma_prefetch_map(&tm_k);
                 tma_prefetch_map(&tm_v);
@@ -816,7 +824,7 @@ __global__ void __launch_bounds__(384, 1)
                 const int i = i_begin + n;
                 const int s = n % L::NS;
                 if (n >= L::NS && !mbar_wait_warp(BAR(L::B_EMPTY + s), ((n / L::NS) - 1) & 1, wc, 1)) break;
-                if (lane == 0) {
+                if (leader) {
                     const uint32_t bar = BAR(L::B_FULL + s);
                     const uint32_t base = sb + s * L::STAGE;
                     const uint32_t vec = sb + L::OFF_VEC + s * L::VEC;
@@ -838,14 +846,15 @@ __global__ void __launch_bounds__(384, 1)
                 armed[s]++;
             }
         }
-        if (lane == 0) {
+        if (leader) {
 #pragma unroll
             for (int s = 0; s < L::NS; ++s)
                 if (armed[s] > 0) drain_wait(BAR(L::B_FULL + s), (armed[s] - 1) & 1, 100000000ull);
         }
     } else if (warp == 9) {
         regs_shrink();
-        if (lane == 0 && !aborted_early) {
+        const bool leader = elect_one();
+        if (!aborted_early) {
             constexpr uint32_t SW = (D == 32) ? SWZ_64B : SWZ_128B;
             constexpr uint32_t SBO = 8 * L::ROWB;
             constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
@@ -854,25 +863,29 @@ __global__ void __launch_bounds__(384, 1)
             for (int n = 0; n < nrows; ++n) {
                 const int s = n % L::NS, x = n & 1;
                 TRI_TP(2)
-                if (!mbar_wait(BAR(L::B_FULL + s), (n / L::NS) & 1, wc, 2)) break;
+                if (!mbar_wait_warp(BAR(L::B_FULL + s), (n / L::NS) & 1, wc, 2)) break;
                 TRI_TP(0)
-                if (n >= 2 && !mbar_wait(BAR(L::B_SDPFREE + x), ((n >> 1) - 1) & 1, wc, 3)) break;
+                if (n >= 2 && !mbar_wait_warp(BAR(L::B_SDPFREE + x), ((n >> 1) - 1) & 1, wc, 3)) break;
                 TRI_TP(1)
                 tc_fence_after();
                 const uint64_t qd = desc_add(d0, s * L::STAGE);
+                if (leader) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    mma_ss(tmem + x * 256, desc_add(qd, kk * 32), desc_add(qd, 2 * L::QKV_TILE + kk * 32), IDESC_S,
-                           kk > 0 ? 1u : 0u);
-                    mma_ss(tmem + x * 256 + 128, desc_add(qd, L::QKV_TILE + kk * 32),
-                           desc_add(qd, 3 * L::QKV_TILE + kk * 32), IDESC_S, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        mma_ss(tmem + x * 256, desc_add(qd, kk * 32), desc_add(qd, 2 * L::QKV_TILE + kk * 32), IDESC_S,
+                               kk > 0 ? 1u : 0u);
+                        mma_ss(tmem + x * 256 + 128, desc_add(qd, L::QKV_TILE + kk * 32),
+                               desc_add(qd, 3 * L::QKV_TILE + kk * 32), IDESC_S, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(BAR(L::B_SDPFULL + x));
+                    mma_commit(BAR(L::B_EMPTY + s));
                 }
-                mma_commit(BAR(L::B_SDPFULL + x));
-                mma_commit(BAR(L::B_EMPTY + s));
+                __syncwarp();
             }
             TRI_TP(2)
             TRI_TRACE_FLUSH_AT(30000)
-            mma_commit(BAR(L::B_DRAIN));
+            if (leader) mma_commit(BAR(L::B_DRAIN));
+            __syncwarp();
             drain_wait(BAR(L::B_DRAIN), 0, 100000000ull);
         }
         __syncwarp();

@@ -62,7 +62,7 @@ struct FwdLayout {
     // barrier indices
     static constexpr int B_Q = 0, B_FULL = 1, B_EMPTY = 1 + NS, B_SFULL = 1 + 2 * NS,
                          B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2, B_PVDONE = B_PFULL + 2,
-                         B_DRAIN = B_PVDONE + 2, NBAR = B_DRAIN + 1;
+                         B_EXPD = B_PVDONE + 2, B_DRAIN = B_EXPD + 2, NBAR = B_DRAIN + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag, mask flags[NS][2]
     static constexpr int SMEM = OFF_MISC + 16 + NS * 2 * 4;
     static_assert(SMEM <= 232448, "shared memory budget");
@@ -130,6 +130,7 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(BAR(L::B_SFREE + w), 4);
             mbar_init(BAR(L::B_PFULL + w), 4);
             mbar_init(BAR(L::B_PVDONE + w), 1);
+            mbar_init(BAR(L::B_EXPD + w), 4);
         }
         mbar_init(BAR(L::B_DRAIN), 1);
         fence_mbar_init();
@@ -157,8 +158,9 @@ __global__ void __launch_bounds__(384, 1)
         auto load_bias = [&](uint32_t dst, uint32_t bar, int k0, int j0) {
             tma_load_4d(dst, &tm_bias, bar, k0, j0, h, b);
         };
+        const bool leader = elect_one();
         if (!aborted_early) {
-            if (lane == 0) {
+            if (leader) {
                 tma_prefetch_map(&tm_q);
                 tma_prefetch_map(&tm_k);
                 tma_prefetch_map(&tm_v);
@@ -202,7 +204,7 @@ __global__ void __launch_bounds__(384, 1)
                     if (lane == 0) mask_flag[s * 2 + w] = any ? 1 : 0;
                 }
                 __syncwarp();
-                if (lane == 0) {
+                if (leader) {
                     const uint32_t bar = BAR(L::B_FULL + s);
                     mbar_arrive_expect_tx(bar, 4 * L::QKV_TILE + L::BIAS_TILE);
                     load_qkv(st + L::OFF_K0, &tm_k, bar, i0, kt * 128);
@@ -219,7 +221,7 @@ __global__ void __launch_bounds__(384, 1)
             TRI_TRACE_FLUSH_AT(0)
         }
         // never leave with bulk copies still writing into this CTA's shared memory
-        if (lane == 0) {
+        if (leader) {
             if (!aborted_early) drain_wait(BAR(L::B_Q), 0, 100000000ull);
 #pragma unroll
             for (int s = 0; s < L::NS; ++s)
@@ -228,7 +230,8 @@ __global__ void __launch_bounds__(384, 1)
     } else if (warp == 9) {
         // =========================== MMA issuer =============================
         regs_shrink();
-        if (lane == 0 && !aborted_early) {
+        const bool leader = elect_one();
+        if (!aborted_early) {
             constexpr uint32_t SW = (D == 32) ? SWZ_64B : SWZ_128B;
             constexpr uint32_t SBO = 8 * L::ROWB;
             constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false, false);
@@ -240,34 +243,42 @@ __global__ void __launch_bounds__(384, 1)
             auto issue_pv = [&](int w, int s, int ktile) {
                 const uint64_t vd = desc_add(dvt0, s * L::STAGE + (w ? L::OFF_V1 : L::OFF_V0));
                 const uint32_t tS = tmem + w * 256;
+                if (leader) {
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tS + 192, tS + 128 + kk * 8, desc_add(vd, kk * 16 * L::ROWB), IDESC_PV,
-                           (ktile > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(tS + 192, tS + 128 + kk * 8, desc_add(vd, kk * 16 * L::ROWB), IDESC_PV,
+                               (ktile > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(BAR(L::B_PVDONE + w));
+                }
+                __syncwarp();
             };
             TRI_TRACE_DECL
-            bool ok = mbar_wait(BAR(L::B_Q), 0, wc, 2);
+            bool ok = mbar_wait_warp(BAR(L::B_Q), 0, wc, 2);
             TRI_TP(9)
             for (int kt = 0; ok && kt < nkt; ++kt) {
                 const int s = kt % L::NS;
                 TRI_TP(4)
-                if (!mbar_wait(BAR(L::B_FULL + s), (kt / L::NS) & 1, wc, 3)) { ok = false; break; }
+                if (!mbar_wait_warp(BAR(L::B_FULL + s), (kt / L::NS) & 1, wc, 3)) { ok = false; break; }
                 TRI_TP(0)
                 tc_fence_after();
 #pragma unroll
                 for (int w = 0; w < 2; ++w) {
                     if (kt > 0) {
                         TRI_TP(4)
-                        if (!mbar_wait(BAR(L::B_SFREE + w), (kt - 1) & 1, wc, 4)) { ok = false; break; }
+                        if (!mbar_wait_warp(BAR(L::B_SFREE + w), (kt - 1) & 1, wc, 4)) { ok = false; break; }
                         TRI_TP(1)
                         tc_fence_after();
                     }
                     const uint64_t qd = desc_add(dq0, w * L::QKV_TILE);
                     const uint64_t kd = desc_add(dst0, s * L::STAGE + (w ? L::OFF_K1 : L::OFF_K0));
+                    if (leader) {
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        mma_ss(tmem + w * 256, desc_add(qd, kk * 32), desc_add(kd, kk * 32), IDESC_QK, kk > 0 ? 1u : 0u);
-                    mma_commit(BAR(L::B_SFULL + w));
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            mma_ss(tmem + w * 256, desc_add(qd, kk * 32), desc_add(kd, kk * 32), IDESC_QK,
+                                   kk > 0 ? 1u : 0u);
+                        mma_commit(BAR(L::B_SFULL + w));
+                    }
+                    __syncwarp();
                 }
                 if (!ok) break;
                 if (kt > 0) {
@@ -275,14 +286,14 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                     for (int w = 0; w < 2; ++w) {
                         TRI_TP(4)
-                        if (!mbar_wait(BAR(L::B_PFULL + w), (kt - 1) & 1, wc, 5)) { ok = false; break; }
+                        if (!mbar_wait_warp(BAR(L::B_PFULL + w), (kt - 1) & 1, wc, 5)) { ok = false; break; }
                         TRI_TP(2)
                         tc_fence_after();
                         issue_pv(w, sp, kt - 1);
-                        mma_commit(BAR(L::B_PVDONE + w));
                     }
                     if (!ok) break;
-                    mma_commit(BAR(L::B_EMPTY + sp));
+                    if (leader) mma_commit(BAR(L::B_EMPTY + sp));
+                    __syncwarp();
                 }
             }
             if (ok) {
@@ -290,17 +301,18 @@ __global__ void __launch_bounds__(384, 1)
                 const int sp = kl % L::NS;
 #pragma unroll
                 for (int w = 0; w < 2; ++w) {
-                    if (!mbar_wait(BAR(L::B_PFULL + w), kl & 1, wc, 5)) { ok = false; break; }
+                    if (!mbar_wait_warp(BAR(L::B_PFULL + w), kl & 1, wc, 5)) { ok = false; break; }
                     tc_fence_after();
                     issue_pv(w, sp, kl);
-                    mma_commit(BAR(L::B_PVDONE + w));
                 }
-                if (ok) mma_commit(BAR(L::B_EMPTY + sp));
+                if (ok && leader) mma_commit(BAR(L::B_EMPTY + sp));
+                __syncwarp();
             }
             TRI_TP(5)
             TRI_TRACE_FLUSH_AT(0)
-            // every MMA this thread issued has completed before the CTA leaves
-            mma_commit(BAR(L::B_DRAIN));
+            // every MMA the leader issued has completed before the CTA leaves
+            if (leader) mma_commit(BAR(L::B_DRAIN));
+            __syncwarp();
             drain_wait(BAR(L::B_DRAIN), 0, 100000000ull);
         }
         __syncwarp();
@@ -405,6 +417,13 @@ __global__ void __launch_bounds__(384, 1)
                 l *= alpha;
             }
             const float mb = fmaxf(m_ref, -3.0e38f) * LOG2E;
+            // Ping-pong on the exponential unit: the two warpgroups take turns
+            // (WG0 tile kt, WG1 tile kt, WG0 tile kt+1, ...), so one runs its
+            // exponentials while the other loads, biases and reduces its next tile.
+            if (w == 1 || kt > 0) {
+                const int turn = w == 1 ? kt : kt - 1;
+                if (!mbar_wait_warp(BAR(L::B_EXPD + (1 - w)), turn & 1, wc, 10)) { ok = false; break; }
+            }
             // probabilities into packed BF16 registers first; the previous PV may still be
             // reading the P columns
             const float2 l2e = make_float2(LOG2E, LOG2E), nmb = make_float2(-mb, -mb);
@@ -424,6 +443,8 @@ __global__ void __launch_bounds__(384, 1)
             }
             const float2 lsum = fadd2(fadd2(ls0, ls1), fadd2(ls2, ls3));
             const float ls = lsum.x + lsum.y;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(BAR(L::B_EXPD + w));
             TRI_TP(5)
             if (kt > 0) {
                 // PV of the previous tile has finished: the P columns are free and O is stable
