@@ -262,7 +262,7 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, f
         mark(1);
         tri_attn_bwd_main_kernel<32><<<ws.grid_main, 384, MainLayout<32>::SMEM, stream>>>(mq, mk, mv, mdo, p);
         mark(2);
-        tri_attn_bwd_dbias_kernel<32><<<db_grid, 384, DbLayout<32>::SMEM, stream>>>(
+        tri_attn_bwd_dbias_kernel<32><<<db_grid, DbLayout<32>::THREADS, DbLayout<32>::SMEM, stream>>>(
             mq, mk, mv, mdo, bias, f.bias.stride[0], f.bias.stride[1], f.bias.stride[2], p);
     } else {
         tri_attn_bwd_prep_kernel<64><<<prep_grid, 256, 0, stream>>>(
@@ -273,7 +273,7 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, f
         mark(1);
         tri_attn_bwd_main_kernel<64><<<ws.grid_main, 384, MainLayout<64>::SMEM, stream>>>(mq, mk, mv, mdo, p);
         mark(2);
-        tri_attn_bwd_dbias_kernel<64><<<db_grid, 384, DbLayout<64>::SMEM, stream>>>(
+        tri_attn_bwd_dbias_kernel<64><<<db_grid, DbLayout<64>::THREADS, DbLayout<64>::SMEM, stream>>>(
             mq, mk, mv, mdo, bias, f.bias.stride[0], f.bias.stride[1], f.bias.stride[2], p);
     }
     if (ws.chunks > 1) {

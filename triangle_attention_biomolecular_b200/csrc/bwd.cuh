@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(256) tri_attn_bwd_prep_kernel(
 template <int D>
 struct MainLayout {
     static constexpr int KVS = (D == 32) ? 2 : 1;  // K/V buffers
-    static constexpr int NS = 2;                   // per-tile stages (Q, dO, vectors)
+    static constexpr int NS = (D == 32) ? 3 : 2;   // per-tile stages (Q, dO, vectors)
     static constexpr int ROWB = D * 2;
     static constexpr int QKV_TILE = 128 * ROWB;
     static constexpr int PT_TILE = 128 * 128 * 2;  // P or dS, BF16, two 64-column SW128 halves
@@ -733,10 +733,13 @@ __global__ void __launch_bounds__(384, 1)
 // ===========================================================================
 template <int D>
 struct DbLayout {
-    static constexpr int NS = (D == 32) ? 3 : 2;
+    static constexpr int NS = (D == 32) ? 4 : 2;
     static constexpr int ROWB = D * 2;
     static constexpr int QKV_TILE = 128 * ROWB;
     static constexpr int STAGE = 4 * QKV_TILE;  // Q, dO, K, V
+    // warps 0-15: four softmax warpgroups, warpgroup w owns keys 32w..32w+31 of the
+    // tile; warp 16 producer, warp 17 MMA, 18-19 spare
+    static constexpr int THREADS = 640, SOFTMAX_WARPS = 16, W_PRODUCER = 16, W_MMA = 17;
     static constexpr int OFF_BIAS = NS * STAGE;  // [128 rows][128 keys] fp32, log2 units, swizzled
     // [NS][lse*log2e 128, D 128, mask*log2e 128 (fp32), key-tile flags 32 (int)]
     static constexpr int OFF_VEC = OFF_BIAS + 128 * 128 * 4;
@@ -750,7 +753,7 @@ struct DbLayout {
 };
 
 template <int D>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(640, 1)
     tri_attn_bwd_dbias_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                               const __nv_bfloat16* __restrict__ bias, int64_t bs0, int64_t bs1, int64_t bs2,
@@ -786,11 +789,11 @@ __global__ void __launch_bounds__(384, 1)
         }
         for (int s = 0; s < L::NS; ++s) {
             mbar_init(BAR(L::B_FULL + s), 1);
-            mbar_init(BAR(L::B_EMPTY + s), 1 + 8);
+            mbar_init(BAR(L::B_EMPTY + s), 1 + L::SOFTMAX_WARPS);
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(BAR(L::B_SDPFULL + x), 1);
-            mbar_init(BAR(L::B_SDPFREE + x), 8);
+            mbar_init(BAR(L::B_SDPFREE + x), L::SOFTMAX_WARPS);
         }
         mbar_init(BAR(L::B_DRAIN), 1);
         fence_mbar_init();
@@ -807,8 +810,8 @@ __global__ void __launch_bounds__(384, 1)
     const bool aborted_early = *abort_flag != 0;
     constexpr float LOG2E = 1.4426950408889634f;
 
-    if (warp == 8) {
-        regs_shrink();
+    if (warp == L::W_PRODUCER) {
+        regs_shrink640();
         int armed[L::NS];
 #pragma unroll
         for (int s = 0; s < L::NS; ++s) armed[s] = 0;
@@ -851,8 +854,8 @@ __global__ void __launch_bounds__(384, 1)
             for (int s = 0; s < L::NS; ++s)
                 if (armed[s] > 0) drain_wait(BAR(L::B_FULL + s), (armed[s] - 1) & 1, 100000000ull);
         }
-    } else if (warp == 9) {
-        regs_shrink();
+    } else if (warp == L::W_MMA) {
+        regs_shrink640();
         const bool leader = elect_one();
         if (!aborted_early) {
             constexpr uint32_t SW = (D == 32) ? SWZ_64B : SWZ_128B;
@@ -889,37 +892,38 @@ __global__ void __launch_bounds__(384, 1)
             drain_wait(BAR(L::B_DRAIN), 0, 100000000ull);
         }
         __syncwarp();
-    } else if (warp >= 10) {
-        regs_shrink();  // spare warps of the last warpgroup
+    } else if (warp >= L::SOFTMAX_WARPS) {
+        regs_shrink640();  // spare warps of the control warpgroup
     } else {
-        regs_grow();
+        regs_grow640();
         if (!aborted_early) {
-        const int w = warp >> 2;
-        const int qd = warp & 3;
+        const int w = warp >> 2;  // key quarter of the tile
+        const int qd = warp & 3;  // TMEM lane quarter = query rows 32qd..32qd+31
         const int row = qd * 32 + lane;
         const uint32_t tl = tmem + (static_cast<uint32_t>(qd * 32) << 16);
         const int j = jt * 128 + row;
         const float c2 = p.scale * LOG2E;
-        // this thread's 64 bias values (row j, keys kt*128 + 64w ..), log2 units, kept in
-        // shared memory (row = 256 B = 16 chunks, chunk index xor (row & 15))
-        const uint32_t brow = sb + L::OFF_BIAS + row * 512 + w * 256;
+        // this thread's 32 bias values (row j, keys kt*128 + 32w ..), log2 units, kept in
+        // shared memory: a row is 512 B = 32 chunks of 16 B; chunk w*8+c sits at
+        // w*8 + (c xor (row & 7)), so eight consecutive rows hit eight different bank groups
+        const uint32_t brow = sb + L::OFF_BIAS + row * 512 + w * 128;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
+        for (int c = 0; c < 8; ++c) {
             float v[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int k = kt * 128 + w * 64 + 4 * c + e;
+                const int k = kt * 128 + w * 32 + 4 * c + e;
                 float bv = 0.f;
                 if (j < p.N && k < p.N)
                     bv = __bfloat162float(bias[b * bs0 + h * bs1 + static_cast<int64_t>(j) * bs2 + k]);
                 v[e] = bv * LOG2E;
             }
-            sts128(brow + ((c ^ (row & 15)) << 4),
+            sts128(brow + ((c ^ (row & 7)) << 4),
                    make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]), __float_as_uint(v[3])));
         }
-        float acc[64];
+        float acc[32];
 #pragma unroll
-        for (int e = 0; e < 64; ++e) acc[e] = 0.f;
+        for (int e = 0; e < 32; ++e) acc[e] = 0.f;
         bool ok = true;
         TRI_TRACE_DECL
         for (int n = 0; n < nrows; ++n) {
@@ -932,26 +936,26 @@ __global__ void __launch_bounds__(384, 1)
             const float lse2 = vec[row];
             const float Dj = vec[128 + row];
             const bool has_mask = reinterpret_cast<const int*>(vec + 384)[kt] != 0;
-            const uint32_t ma = sb + L::OFF_VEC + s * L::VEC + 1024 + w * 256;
+            const uint32_t ma = sb + L::OFF_VEC + s * L::VEC + 1024 + w * 128;
             const float2 c22 = make_float2(c2, c2), nl2 = make_float2(-lse2, -lse2), nD2 = make_float2(-Dj, -Dj);
             TRI_TP(1)
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                uint32_t sv[32], dv[32];
-                tmem_ld32(tl + x * 256 + w * 64 + half * 32, sv);
-                tmem_ld32(tl + x * 256 + 128 + w * 64 + half * 32, dv);
+                uint32_t sv[16], dv[16];
+                tmem_ld16(tl + x * 256 + w * 32 + half * 16, sv);
+                tmem_ld16(tl + x * 256 + 128 + w * 32 + half * 16, dv);
                 tmem_wait_ld();
-                reg_fence32(sv);
-                reg_fence32(dv);
+                reg_fence16(sv);
+                reg_fence16(dv);
                 if (half == 1) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(BAR(L::B_SDPFREE + x));
                 }
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const int cc = half * 8 + c;
-                    const float4 bq = lds128f(brow + ((cc ^ (row & 15)) << 4));
+                for (int c = 0; c < 4; ++c) {
+                    const int cc = half * 4 + c;
+                    const float4 bq = lds128f(brow + ((cc ^ (row & 7)) << 4));
                     float2 b01 = make_float2(bq.x, bq.y), b23 = make_float2(bq.z, bq.w);
                     if (has_mask) {
                         const float4 mq = lds128f(ma + cc * 16);
@@ -966,9 +970,9 @@ __global__ void __launch_bounds__(384, 1)
                         const float2 y = fadd2(t, nl2);
                         const float2 pv = make_float2(ex2(y.x), ex2(y.y));
                         const float2 dd = fadd2(make_float2(__uint_as_float(dv[xl]), __uint_as_float(dv[xl + 1])), nD2);
-                        const float2 a = ffma2(pv, dd, make_float2(acc[32 * half + xl], acc[32 * half + xl + 1]));
-                        acc[32 * half + xl] = a.x;
-                        acc[32 * half + xl + 1] = a.y;
+                        const float2 a = ffma2(pv, dd, make_float2(acc[16 * half + xl], acc[16 * half + xl + 1]));
+                        acc[16 * half + xl] = a.x;
+                        acc[16 * half + xl + 1] = a.y;
                     }
                 }
             }
@@ -978,11 +982,11 @@ __global__ void __launch_bounds__(384, 1)
         }
         TRI_TP(3)
         if (ok && j < p.N) {
-            const int k0 = kt * 128 + w * 64;
+            const int k0 = kt * 128 + w * 32;
             if (p.chunks == 1) {
                 __nv_bfloat16* dst = p.dbias + b * p.dbs[0] + h * p.dbs[1] + static_cast<int64_t>(j) * p.dbs[2] + k0;
 #pragma unroll
-                for (int e = 0; e < 64; e += 8) {
+                for (int e = 0; e < 32; e += 8) {
                     if (k0 + e + 8 <= p.N) {
                         uint4 v;
                         v.x = pack_bf16(acc[e], acc[e + 1]);
@@ -999,7 +1003,7 @@ __global__ void __launch_bounds__(384, 1)
             } else {
                 float* dst = p.part + (((static_cast<int64_t>(chunk) * p.B + b) * p.H + h) * p.N + j) * p.N + k0;
 #pragma unroll
-                for (int e = 0; e < 64; ++e)
+                for (int e = 0; e < 32; ++e)
                     if (k0 + e < p.N) dst[e] = acc[e];
             }
         }
@@ -1010,7 +1014,7 @@ __global__ void __launch_bounds__(384, 1)
     }
 
     tc_fence_before();
-    cta_end_barrier();
+    cta_end_barrier640();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);

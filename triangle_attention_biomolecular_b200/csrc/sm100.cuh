@@ -38,7 +38,7 @@ __device__ unsigned long long* g_trace;
     {                                                                                                     \
         if (g_trace && (threadIdx.x & 31) == 0)                                                           \
             for (int tri_q_ = 0; tri_q_ < 16; ++tri_q_)                                                   \
-                g_trace[(static_cast<size_t>(blockIdx.x + (base)) * 12 + (threadIdx.x >> 5)) * 16 + tri_q_] =  \
+                g_trace[(static_cast<size_t>(blockIdx.x + (base)) * 32 + (threadIdx.x >> 5)) * 16 + tri_q_] =  \
                     tri_acc_[tri_q_];                                                                     \
     }
 #else
@@ -312,9 +312,20 @@ constexpr int kRegsLaunch = 168, kRegsSmall = 88, kRegsLarge = 208;
 static_assert(128 * kRegsSmall + 256 * kRegsLarge <= 384 * kRegsLaunch && kRegsSmall % 8 == 0 && kRegsLarge % 8 == 0,
               "register split must fit the launch total");
 __device__ __forceinline__ void regs_shrink() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSmall)); }
+// The same for 640-thread kernels (four softmax warpgroups and one control
+// warpgroup, 96 registers each at launch, 61440 total): 512 * 104 + 128 * 56 = 60416.
+constexpr int kRegsLaunch640 = 96, kRegsSmall640 = 56, kRegsLarge640 = 104;
+static_assert(128 * kRegsSmall640 + 512 * kRegsLarge640 <= 640 * kRegsLaunch640 && kRegsSmall640 % 8 == 0 &&
+                  kRegsLarge640 % 8 == 0,
+              "register split must fit the launch allocation");
+__device__ __forceinline__ void regs_shrink640() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSmall640));
+}
+__device__ __forceinline__ void regs_grow640() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsLarge640)); }
 __device__ __forceinline__ void regs_grow() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsLarge)); }
 // every role of the CTA meets here before tensor memory is released
 __device__ __forceinline__ void cta_end_barrier() { asm volatile("bar.sync 1, 384;" ::: "memory"); }
+__device__ __forceinline__ void cta_end_barrier640() { asm volatile("bar.sync 1, 640;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // arithmetic helpers
