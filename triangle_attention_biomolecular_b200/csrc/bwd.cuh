@@ -674,7 +674,9 @@ __global__ void __launch_bounds__(384, 1)
                                                        bf16x2_to_f2(bw[c * 4 + e]));
                                 float2 y = ffma2(t, l2e, nl2);
                                 if constexpr (kMasked) y = fadd2(y, make_float2(mk[2 * e], mk[2 * e + 1]));
-                                const float p0 = ex2(y.x), p1 = ex2(y.y);
+                                // in key tiles without a mask, one pair in four takes the FMA-pipe exponential
+                                const float2 pp = (!kMasked && e == 3) ? ex2_fma2(y) : make_float2(ex2(y.x), ex2(y.y));
+                                const float p0 = pp.x, p1 = pp.y;
                                 const float2 ds = fmul2(make_float2(p0, p1),
                                                         fadd2(make_float2(__uint_as_float(dv0), __uint_as_float(dv1)), nD2));
                                 pw[c * 4 + e] = pack_bf16(p0, p1);
@@ -939,43 +941,51 @@ __global__ void __launch_bounds__(640, 1)
             const uint32_t ma = sb + L::OFF_VEC + s * L::VEC + 1024 + w * 128;
             const float2 c22 = make_float2(c2, c2), nl2 = make_float2(-lse2, -lse2), nD2 = make_float2(-Dj, -Dj);
             TRI_TP(1)
+            // dS = P (dP - D) accumulated over rows; in key tiles without a mask a quarter of
+            // the exponentials run on the FMA pipe (ex2_fma2) beside the MUFU unit
+            auto row_step = [&](auto masked) {
+                constexpr bool kMasked = decltype(masked)::value;
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t sv[16], dv[16];
-                tmem_ld16(tl + x * 256 + w * 32 + half * 16, sv);
-                tmem_ld16(tl + x * 256 + 128 + w * 32 + half * 16, dv);
-                tmem_wait_ld();
-                reg_fence16(sv);
-                reg_fence16(dv);
-                if (half == 1) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(BAR(L::B_SDPFREE + x));
-                }
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int cc = half * 4 + c;
-                    const float4 bq = lds128f(brow + ((cc ^ (row & 7)) << 4));
-                    float2 b01 = make_float2(bq.x, bq.y), b23 = make_float2(bq.z, bq.w);
-                    if (has_mask) {
-                        const float4 mq = lds128f(ma + cc * 16);
-                        b01 = fadd2(b01, make_float2(mq.x, mq.y));
-                        b23 = fadd2(b23, make_float2(mq.z, mq.w));
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t sv[16], dv[16];
+                    tmem_ld16(tl + x * 256 + w * 32 + half * 16, sv);
+                    tmem_ld16(tl + x * 256 + 128 + w * 32 + half * 16, dv);
+                    tmem_wait_ld();
+                    reg_fence16(sv);
+                    reg_fence16(dv);
+                    if (half == 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(BAR(L::B_SDPFREE + x));
                     }
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int xl = 4 * c + 2 * e;
-                        const float2 t = ffma2(make_float2(__uint_as_float(sv[xl]), __uint_as_float(sv[xl + 1])), c22,
-                                               e ? b23 : b01);
-                        const float2 y = fadd2(t, nl2);
-                        const float2 pv = make_float2(ex2(y.x), ex2(y.y));
-                        const float2 dd = fadd2(make_float2(__uint_as_float(dv[xl]), __uint_as_float(dv[xl + 1])), nD2);
-                        const float2 a = ffma2(pv, dd, make_float2(acc[16 * half + xl], acc[16 * half + xl + 1]));
-                        acc[16 * half + xl] = a.x;
-                        acc[16 * half + xl + 1] = a.y;
+                    for (int c = 0; c < 4; ++c) {
+                        const int cc = half * 4 + c;
+                        const float4 bq = lds128f(brow + ((cc ^ (row & 7)) << 4));
+                        float2 b01 = make_float2(bq.x, bq.y), b23 = make_float2(bq.z, bq.w);
+                        if constexpr (kMasked) {
+                            const float4 mq = lds128f(ma + cc * 16);
+                            b01 = fadd2(b01, make_float2(mq.x, mq.y));
+                            b23 = fadd2(b23, make_float2(mq.z, mq.w));
+                        }
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int xl = 4 * c + 2 * e;
+                            const float2 t = ffma2(make_float2(__uint_as_float(sv[xl]), __uint_as_float(sv[xl + 1])),
+                                                   c22, e ? b23 : b01);
+                            const float2 y = fadd2(t, nl2);
+                            const float2 pv = (!kMasked && (xl & 6) == 6) ? ex2_fma2(y) : make_float2(ex2(y.x), ex2(y.y));
+                            const float2 dd =
+                                fadd2(make_float2(__uint_as_float(dv[xl]), __uint_as_float(dv[xl + 1])), nD2);
+                            const float2 a = ffma2(pv, dd, make_float2(acc[16 * half + xl], acc[16 * half + xl + 1]));
+                            acc[16 * half + xl] = a.x;
+                            acc[16 * half + xl + 1] = a.y;
+                        }
                     }
                 }
-            }
+            };
+            if (has_mask) row_step(std::true_type{});
+            else row_step(std::false_type{});
             TRI_TP(2)
             __syncwarp();
             if (lane == 0) mbar_arrive(BAR(L::B_EMPTY + s));

@@ -29,6 +29,8 @@
 //    flagged so the add is skipped.
 #pragma once
 
+#include <type_traits>
+
 #include "sm100.cuh"
 
 namespace tri {
@@ -387,7 +389,8 @@ __global__ void __launch_bounds__(384, 1)
                     x[x0 + 1] = y.y;
                 }
             }
-            if (mask_flag[s * 2 + w]) {
+            const bool tile_masked = mask_flag[s * 2 + w] != 0;
+            if (tile_masked) {
                 const uint32_t ma = st + L::OFF_MASK + w * 512;
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
@@ -436,18 +439,24 @@ __global__ void __launch_bounds__(384, 1)
             const float2 l2e = make_float2(LOG2E, LOG2E), nmb = make_float2(-mb, -mb);
             float2 ls0 = make_float2(0.f, 0.f), ls1 = ls0, ls2 = ls0, ls3 = ls0;
             uint32_t pk[64];
+            // in key tiles without a mask, one pair in four takes the FMA-pipe exponential
+            auto exps = [&](auto mixed) {
+                constexpr bool kMixed = decltype(mixed)::value;
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                const float2 a2 = ffma2(make_float2(x[2 * c], x[2 * c + 1]), l2e, nmb);
-                const float2 pp = make_float2(ex2(a2.x), ex2(a2.y));
-                switch (c & 3) {
-                    case 0: ls0 = fadd2(ls0, pp); break;
-                    case 1: ls1 = fadd2(ls1, pp); break;
-                    case 2: ls2 = fadd2(ls2, pp); break;
-                    default: ls3 = fadd2(ls3, pp); break;
+                for (int c = 0; c < 64; ++c) {
+                    const float2 a2 = ffma2(make_float2(x[2 * c], x[2 * c + 1]), l2e, nmb);
+                    const float2 pp = (kMixed && (c & 3) == 3) ? ex2_fma2(a2) : make_float2(ex2(a2.x), ex2(a2.y));
+                    switch (c & 3) {
+                        case 0: ls0 = fadd2(ls0, pp); break;
+                        case 1: ls1 = fadd2(ls1, pp); break;
+                        case 2: ls2 = fadd2(ls2, pp); break;
+                        default: ls3 = fadd2(ls3, pp); break;
+                    }
+                    pk[c] = pack_bf16(pp.x, pp.y);
                 }
-                pk[c] = pack_bf16(pp.x, pp.y);
-            }
+            };
+            if (tile_masked) exps(std::false_type{});
+            else exps(std::true_type{});
             const float2 lsum = fadd2(fadd2(ls0, ls1), fadd2(ls2, ls3));
             const float ls = lsum.x + lsum.y;
             __syncwarp();

@@ -369,6 +369,15 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
     return d;
 }
+__device__ __forceinline__ float2 fadd2_rm(float2 a, float2 b) {  // rounded toward minus infinity
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rm.ftz.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
 __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
     float2 d;
     asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
@@ -377,6 +386,34 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
         : "=f"(d.x), "=f"(d.y)
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
     return d;
+}
+
+// 2^x for a pair of arguments on the FMA pipe, leaving the MUFU unit free: the
+// kernels route a fixed share of their exponentials here so that both pipes work.
+// Method (range reduction + polynomial): x = n + f with n = floor(x), taken from the
+// low mantissa bits of x + 1.5*2^23 added with rounding toward minus infinity;
+// 2^f on [0, 1) by the cubic c0 + c1 f + c2 f^2 + c3 f^3, whose coefficients were
+// fitted for least maximum relative error by Lawson's iterated weighted least
+// squares (7.5e-5 in exact arithmetic, 1.4e-4 with float32 evaluation); n is then
+// added into the exponent field.  Arguments are clamped to >= -125, so anything
+// below gives 2^-125 (about 2.4e-38) rather than 0: callers use it only where a
+// masked key (which must give exactly 0) cannot occur.
+constexpr float kEx2C0 = 0.9999251365661621f, kEx2C1 = 0.6958339810371399f, kEx2C2 = 0.22606706619262695f,
+                kEx2C3 = 0.07802402973175049f;
+__device__ __forceinline__ float2 ex2_fma2(float2 x) {
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const float2 t = fadd2_rm(x, make_float2(kMagic, kMagic));      // 1.5*2^23 + floor(x)
+    const float2 n = fadd2(t, make_float2(-kMagic, -kMagic));       // floor(x), exact
+    const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);          // x - floor(x), exact
+    float2 q = ffma2(make_float2(kEx2C3, kEx2C3), f, make_float2(kEx2C2, kEx2C2));
+    q = ffma2(q, f, make_float2(kEx2C1, kEx2C1));
+    q = ffma2(q, f, make_float2(kEx2C0, kEx2C0));
+    // floor(x) sits in the low mantissa bits of t; shifting t left by 23 moves it into the
+    // exponent field (the constant high bits shift out)
+    return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 // max of three
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
