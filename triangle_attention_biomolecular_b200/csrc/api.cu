@@ -260,7 +260,7 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, f
             static_cast<const __nv_bfloat16*>(f.resid.ptr), sr[0], sr[1], sr[2], sr[3], use_resid, f.lse, f.mask.ptr,
             sm[0], sm[1], sm[2], Dv, Lv, Mv, Fv, B, N, H, ws.Np, p.nt);
         mark(1);
-        tri_attn_bwd_main_kernel<32><<<ws.grid_main, 384, MainLayout<32>::SMEM, stream>>>(mq, mk, mv, mdo, p);
+        tri_attn_bwd_main_kernel<32><<<ws.grid_main, MainLayout<32>::THREADS, MainLayout<32>::SMEM, stream>>>(mq, mk, mv, mdo, p);
         mark(2);
         tri_attn_bwd_dbias_kernel<32><<<db_grid, DbLayout<32>::THREADS, DbLayout<32>::SMEM, stream>>>(
             mq, mk, mv, mdo, bias, f.bias.stride[0], f.bias.stride[1], f.bias.stride[2], p);
@@ -271,7 +271,7 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, f
             static_cast<const __nv_bfloat16*>(f.resid.ptr), sr[0], sr[1], sr[2], sr[3], use_resid, f.lse, f.mask.ptr,
             sm[0], sm[1], sm[2], Dv, Lv, Mv, Fv, B, N, H, ws.Np, p.nt);
         mark(1);
-        tri_attn_bwd_main_kernel<64><<<ws.grid_main, 384, MainLayout<64>::SMEM, stream>>>(mq, mk, mv, mdo, p);
+        tri_attn_bwd_main_kernel<64><<<ws.grid_main, MainLayout<64>::THREADS, MainLayout<64>::SMEM, stream>>>(mq, mk, mv, mdo, p);
         mark(2);
         tri_attn_bwd_dbias_kernel<64><<<db_grid, DbLayout<64>::THREADS, DbLayout<64>::SMEM, stream>>>(
             mq, mk, mv, mdo, bias, f.bias.stride[0], f.bias.stride[1], f.bias.stride[2], p);

@@ -181,6 +181,9 @@ __global__ void __launch_bounds__(256) tri_attn_bwd_prep_kernel(
 // ===========================================================================
 template <int D>
 struct MainLayout {
+    // warps 0-15: four softmax warpgroups, warpgroup w owns keys 32w..32w+31 of every
+    // tile; warp 16 producer, warp 17 MMA, 18-19 spare
+    static constexpr int THREADS = 640, SOFTMAX_WARPS = 16, W_PRODUCER = 16, W_MMA = 17;
     static constexpr int KVS = (D == 32) ? 2 : 1;  // K/V buffers
     static constexpr int NS = (D == 32) ? 3 : 2;   // per-tile stages (Q, dO, vectors)
     static constexpr int ROWB = D * 2;
@@ -211,7 +214,7 @@ struct MainLayout {
 };
 
 template <int D>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(640, 1)
     tri_attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                              const BwdParams p) {
@@ -241,22 +244,22 @@ __global__ void __launch_bounds__(384, 1)
         }
         for (int s = 0; s < L::KVS; ++s) {
             mbar_init(BAR(L::B_KVFULL + s), 1);
-            mbar_init(BAR(L::B_KVEMPTY + s), 1 + 8);
+            mbar_init(BAR(L::B_KVEMPTY + s), 1 + L::SOFTMAX_WARPS);
         }
         for (int s = 0; s < L::NS; ++s) {
             mbar_init(BAR(L::B_TFULL + s), 1);
-            mbar_init(BAR(L::B_TEMPTY + s), 1 + 8);
+            mbar_init(BAR(L::B_TEMPTY + s), 1 + L::SOFTMAX_WARPS);
         }
         mbar_init(BAR(L::B_SDPFULL), 1);
-        mbar_init(BAR(L::B_SDPFREE), 8);
+        mbar_init(BAR(L::B_SDPFREE), L::SOFTMAX_WARPS);
         for (int x = 0; x < 2; ++x) {
-            mbar_init(BAR(L::B_PDSFULL + x), 8);
+            mbar_init(BAR(L::B_PDSFULL + x), L::SOFTMAX_WARPS);
             mbar_init(BAR(L::B_PDSFREE + x), 1);
         }
         mbar_init(BAR(L::B_DQFULL), 1);
-        mbar_init(BAR(L::B_DQFREE), 8);
+        mbar_init(BAR(L::B_DQFREE), L::SOFTMAX_WARPS);
         mbar_init(BAR(L::B_DKVFULL), 1);
-        mbar_init(BAR(L::B_DKVFREE), 8);
+        mbar_init(BAR(L::B_DKVFREE), L::SOFTMAX_WARPS);
         mbar_init(BAR(L::B_DRAIN), 1);
         fence_mbar_init();
     }
@@ -272,9 +275,9 @@ __global__ void __launch_bounds__(384, 1)
     const bool aborted_early = *abort_flag != 0;
     constexpr float LOG2E = 1.4426950408889634f;
 
-    if (warp == 8) {
+    if (warp == L::W_PRODUCER) {
         // =========================== producer ===============================
-        regs_shrink();
+        regs_shrink640();
         int armed_kv[L::KVS], armed_t[L::NS];
 #pragma unroll
         for (int s = 0; s < L::KVS; ++s) armed_kv[s] = 0;
@@ -345,9 +348,9 @@ __global__ void __launch_bounds__(384, 1)
             for (int s = 0; s < L::NS; ++s)
                 if (armed_t[s] > 0) drain_wait(BAR(L::B_TFULL + s), (armed_t[s] - 1) & 1, 100000000ull);
         }
-    } else if (warp == 9) {
+    } else if (warp == L::W_MMA) {
         // =========================== MMA issuer =============================
-        regs_shrink();
+        regs_shrink640();
         const bool leader = elect_one();
         if (!aborted_early) {
             constexpr uint32_t SW = (D == 32) ? SWZ_64B : SWZ_128B;
@@ -468,13 +471,13 @@ __global__ void __launch_bounds__(384, 1)
             drain_wait(BAR(L::B_DRAIN), 0, 100000000ull);
         }
         __syncwarp();
-    } else if (warp >= 10) {
-        regs_shrink();  // spare warps of the last warpgroup
+    } else if (warp >= L::SOFTMAX_WARPS) {
+        regs_shrink640();  // spare warps of the control warpgroup
     } else {
-        regs_grow();
+        regs_grow640();
         if (!aborted_early) {
         // =========================== softmax + epilogue warps ===============
-        const int w = warp >> 2;  // column half of every tile handled by this warpgroup
+        const int w = warp >> 2;  // key quarter of every tile handled by this warpgroup
         const int qd = warp & 3;
         const int row = qd * 32 + lane;
         const uint32_t tl = tmem + (static_cast<uint32_t>(qd * 32) << 16);
@@ -487,28 +490,27 @@ __global__ void __launch_bounds__(384, 1)
 
         int ep_count = 0;  // dQ epilogues done
         auto epilogue = [&](const Done& t) -> bool {
-            // ---- dQ: this warpgroup's D/2 columns of the tile's block ----
+            // ---- dQ: this warpgroup's D/4 columns of the tile's block ----
             if (!p.dq_tmem || t.kt == nt - 1) {
                 if (!mbar_wait_warp(BAR(L::B_DQFULL), ep_count & 1, wc, 10)) return false;
                 tc_fence_after();
                 const uint32_t dq_col = p.dq_tmem ? L::T_DQ + t.jt * D : L::T_DQ;
-                uint32_t dqr[D / 2];
+                uint32_t dqr[D / 4];
                 if constexpr (D == 32) {
+                    uint32_t x[8];
+                    tmem_ld8(tl + dq_col + w * 8, x);
+                    tmem_wait_ld();
+                    asm volatile("" : "+r"(x[0]), "+r"(x[1]), "+r"(x[2]), "+r"(x[3]), "+r"(x[4]), "+r"(x[5]),
+                                 "+r"(x[6]), "+r"(x[7]));
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) dqr[e] = x[e];
+                } else {
                     uint32_t x[16];
                     tmem_ld16(tl + dq_col + w * 16, x);
                     tmem_wait_ld();
-                    asm volatile("" : "+r"(x[0]), "+r"(x[1]), "+r"(x[2]), "+r"(x[3]), "+r"(x[4]), "+r"(x[5]),
-                                 "+r"(x[6]), "+r"(x[7]), "+r"(x[8]), "+r"(x[9]), "+r"(x[10]), "+r"(x[11]),
-                                 "+r"(x[12]), "+r"(x[13]), "+r"(x[14]), "+r"(x[15]));
+                    reg_fence16(x);
 #pragma unroll
                     for (int e = 0; e < 16; ++e) dqr[e] = x[e];
-                } else {
-                    uint32_t x[32];
-                    tmem_ld32(tl + dq_col + w * 32, x);
-                    tmem_wait_ld();
-                    reg_fence32(x);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) dqr[e] = x[e];
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -516,13 +518,13 @@ __global__ void __launch_bounds__(384, 1)
                 ++ep_count;
                 const int j = t.jt * 128 + row;
                 if (j < p.N) {
-                    float acc[D / 2];
+                    float acc[D / 4];
 #pragma unroll
-                    for (int e = 0; e < D / 2; ++e) acc[e] = __uint_as_float(dqr[e]);
-                    float* slot = p.dq_slots + (static_cast<int64_t>(blockIdx.x) * p.N + j) * D + w * (D / 2);
+                    for (int e = 0; e < D / 4; ++e) acc[e] = __uint_as_float(dqr[e]);
+                    float* slot = p.dq_slots + (static_cast<int64_t>(blockIdx.x) * p.N + j) * D + w * (D / 4);
                     if (!p.dq_tmem && t.kt > 0) {
 #pragma unroll
-                        for (int e = 0; e < D / 2; e += 4) {
+                        for (int e = 0; e < D / 4; e += 4) {
                             const float4 v = *reinterpret_cast<const float4*>(slot + e);
                             acc[e] += v.x;
                             acc[e + 1] += v.y;
@@ -532,12 +534,12 @@ __global__ void __launch_bounds__(384, 1)
                     }
                     if (!p.dq_tmem && t.kt < nt - 1) {
 #pragma unroll
-                        for (int e = 0; e < D / 2; e += 4)
+                        for (int e = 0; e < D / 4; e += 4)
                             *reinterpret_cast<float4*>(slot + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
                     } else {
-                        __nv_bfloat16* dst = p.dq + t.b * p.dqs[0] + t.i * p.dqs[1] + j * p.dqs[2] + t.h * p.dqs[3] + w * (D / 2);
+                        __nv_bfloat16* dst = p.dq + t.b * p.dqs[0] + t.i * p.dqs[1] + j * p.dqs[2] + t.h * p.dqs[3] + w * (D / 4);
 #pragma unroll
-                        for (int e = 0; e < D / 2; e += 8) {
+                        for (int e = 0; e < D / 4; e += 8) {
                             uint4 v;
                             v.x = pack_bf16(acc[e] * scale, acc[e + 1] * scale);
                             v.y = pack_bf16(acc[e + 2] * scale, acc[e + 3] * scale);
@@ -548,31 +550,39 @@ __global__ void __launch_bounds__(384, 1)
                     }
                 }
             }
-            // ---- dK (warpgroup 0) or dV (warpgroup 1) of a finished key tile ----
+            // ---- dK (warpgroups 0, 1) or dV (2, 3), D/2 columns each, of a finished key tile ----
             if (t.jt == nt - 1) {
                 if (!mbar_wait_warp(BAR(L::B_DKVFULL), t.kcount & 1, wc, 11)) return false;
                 tc_fence_after();
-                uint32_t g16[D];
+                const bool is_dk = w < 2;
+                const int c_off = (w & 1) * (D / 2);
+                uint32_t g16[D / 2];
+                if constexpr (D == 32) {
+                    uint32_t x[16];
+                    tmem_ld16(tl + (is_dk ? L::T_DK : L::T_DV) + c_off, x);
+                    tmem_wait_ld();
+                    reg_fence16(x);
 #pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
+                    for (int e = 0; e < 16; ++e) g16[e] = x[e];
+                } else {
                     uint32_t x[32];
-                    tmem_ld32(tl + (w == 0 ? L::T_DK : L::T_DV) + c0, x);
+                    tmem_ld32(tl + (is_dk ? L::T_DK : L::T_DV) + c_off, x);
                     tmem_wait_ld();
                     reg_fence32(x);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) g16[c0 + e] = x[e];
+                    for (int e = 0; e < 32; ++e) g16[e] = x[e];
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(BAR(L::B_DKVFREE));
                 const int k = t.kt * 128 + row;
                 if (k < p.N) {
-                    const float f = (w == 0) ? scale : 1.f;
-                    __nv_bfloat16* dst = (w == 0)
+                    const float f = is_dk ? scale : 1.f;
+                    __nv_bfloat16* dst = (is_dk
                         ? p.dk + t.b * p.dks[0] + t.i * p.dks[1] + k * p.dks[2] + t.h * p.dks[3]
-                        : p.dv + t.b * p.dvs[0] + t.i * p.dvs[1] + k * p.dvs[2] + t.h * p.dvs[3];
+                        : p.dv + t.b * p.dvs[0] + t.i * p.dvs[1] + k * p.dvs[2] + t.h * p.dvs[3]) + c_off;
 #pragma unroll
-                    for (int e = 0; e < D; e += 8) {
+                    for (int e = 0; e < D / 2; e += 8) {
                         uint4 v;
                         v.x = pack_bf16(__uint_as_float(g16[e]) * f, __uint_as_float(g16[e + 1]) * f);
                         v.y = pack_bf16(__uint_as_float(g16[e + 2]) * f, __uint_as_float(g16[e + 3]) * f);
@@ -595,18 +605,18 @@ __global__ void __launch_bounds__(384, 1)
                 if (!mbar_wait_warp(BAR(L::B_KVFULL + ks), (gk / L::KVS) & 1, wc, 12)) { ok = false; break; }
                 TRI_TP(9)
                 const bool has_mask = reinterpret_cast<const int*>(smem + L::OFF_FLAGS + ks * 128)[kt] != 0;
-                const uint32_t maskv = sb + L::OFF_MASKV + ks * 512 + w * 256;
+                const uint32_t maskv = sb + L::OFF_MASKV + ks * 512 + w * 128;
                 for (int jt = 0; jt < nt; ++jt) {
                     const int ts = g % L::NS;
-                    // this thread's 64 bias values (row j, keys kt*128 + 64w ..), straight from global
+                    // this thread's 32 bias values (row j, keys kt*128 + 32w ..), straight from global
                     // memory (L2-resident: shared by every row i); issued before the waits below
-                    uint32_t bw[32];
+                    uint32_t bw[16];
                     {
                         const int j = jt * 128 + row;
-                        const int k0 = kt * 128 + w * 64;
+                        const int k0 = kt * 128 + w * 32;
                         const __nv_bfloat16* bp = p.bias + b * p.bs0 + h * p.bs1 + static_cast<int64_t>(j) * p.bs2 + k0;
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) {
+                        for (int c = 0; c < 4; ++c) {
                             uint4 v = make_uint4(0, 0, 0, 0);
                             if (j < p.N) {
                                 if (k0 + 8 * c + 8 <= p.N) {
@@ -629,73 +639,72 @@ __global__ void __launch_bounds__(384, 1)
                     if (!mbar_wait_warp(BAR(L::B_SDPFULL), g & 1, wc, 13)) { ok = false; break; }
                     TRI_TP(0)
                     tc_fence_after();
-                    uint32_t s0[32], s1[32], d0[32], d1[32];
-                    tmem_ld32(tl + L::T_S + w * 64, s0);
-                    tmem_ld32(tl + L::T_S + w * 64 + 32, s1);
-                    tmem_ld32(tl + L::T_DP + w * 64, d0);
-                    tmem_ld32(tl + L::T_DP + w * 64 + 32, d1);
-                    tmem_wait_ld();
-                    reg_fence32(s0);
-                    reg_fence32(s1);
-                    reg_fence32(d0);
-                    reg_fence32(d1);
-                    TRI_TP(1)
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(BAR(L::B_SDPFREE));
                     if (!mbar_wait_warp(BAR(L::B_TFULL + ts), (g / L::NS) & 1, wc, 14)) { ok = false; break; }
                     TRI_TP(2)
                     const float* vec = reinterpret_cast<const float*>(smem + L::OFF_VEC + ts * 1024);
                     const float lse2 = vec[row];
                     const float Dj = vec[128 + row];
-                    // P and dS of this warpgroup's 64 keys, packed BF16 pairs, computed while the
-                    // previous tile's gradient MMAs still read the shared-memory tiles
-                    uint32_t pw[32], dw[32];
+                    // P and dS of this warpgroup's 32 keys, packed BF16 pairs, computed in two
+                    // 16-key halves while the previous tile's gradient MMAs still read the
+                    // shared-memory tiles
+                    uint32_t pw[16], dw[16];
                     const float2 sc2 = make_float2(scale, scale), l2e = make_float2(LOG2E, LOG2E);
                     const float2 nl2 = make_float2(-lse2, -lse2), nD2 = make_float2(-Dj, -Dj);
                     auto tile = [&](auto masked) {
                         constexpr bool kMasked = decltype(masked)::value;
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            float mk[8];
-                            if constexpr (kMasked) {
-                                const float4 m0 = lds128f(maskv + c * 32), m1 = lds128f(maskv + c * 32 + 16);
-                                mk[0] = m0.x; mk[1] = m0.y; mk[2] = m0.z; mk[3] = m0.w;
-                                mk[4] = m1.x; mk[5] = m1.y; mk[6] = m1.z; mk[7] = m1.w;
+                        for (int hh = 0; hh < 2; ++hh) {
+                            uint32_t sv[16], dv[16];
+                            tmem_ld16(tl + L::T_S + w * 32 + hh * 16, sv);
+                            tmem_ld16(tl + L::T_DP + w * 32 + hh * 16, dv);
+                            tmem_wait_ld();
+                            reg_fence16(sv);
+                            reg_fence16(dv);
+                            if (hh == 1) {
+                                TRI_TP(1)
+                                tc_fence_before();
+                                __syncwarp();
+                                if (lane == 0) mbar_arrive(BAR(L::B_SDPFREE));
                             }
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int x0 = c * 8 + 2 * e;
-                                const uint32_t sv0 = (x0 < 32) ? s0[x0] : s1[x0 - 32];
-                                const uint32_t sv1 = (x0 + 1 < 32) ? s0[x0 + 1] : s1[x0 + 1 - 32];
-                                const uint32_t dv0 = (x0 < 32) ? d0[x0] : d1[x0 - 32];
-                                const uint32_t dv1 = (x0 + 1 < 32) ? d0[x0 + 1] : d1[x0 + 1 - 32];
-                                const float2 t = ffma2(make_float2(__uint_as_float(sv0), __uint_as_float(sv1)), sc2,
-                                                       bf16x2_to_f2(bw[c * 4 + e]));
-                                float2 y = ffma2(t, l2e, nl2);
-                                if constexpr (kMasked) y = fadd2(y, make_float2(mk[2 * e], mk[2 * e + 1]));
-                                // in key tiles without a mask, one pair in four takes the FMA-pipe exponential
-                                const float2 pp = (!kMasked && e == 3) ? ex2_fma2(y) : make_float2(ex2(y.x), ex2(y.y));
-                                const float p0 = pp.x, p1 = pp.y;
-                                const float2 ds = fmul2(make_float2(p0, p1),
-                                                        fadd2(make_float2(__uint_as_float(dv0), __uint_as_float(dv1)), nD2));
-                                pw[c * 4 + e] = pack_bf16(p0, p1);
-                                dw[c * 4 + e] = pack_bf16(ds.x, ds.y);
+                            for (int c = 0; c < 2; ++c) {
+                                const int cc = hh * 2 + c;  // 8-key chunk of this warpgroup's 32 keys
+                                float mk[8];
+                                if constexpr (kMasked) {
+                                    const float4 m0 = lds128f(maskv + cc * 32), m1 = lds128f(maskv + cc * 32 + 16);
+                                    mk[0] = m0.x; mk[1] = m0.y; mk[2] = m0.z; mk[3] = m0.w;
+                                    mk[4] = m1.x; mk[5] = m1.y; mk[6] = m1.z; mk[7] = m1.w;
+                                }
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const int xl = c * 8 + 2 * e;
+                                    const float2 t = ffma2(make_float2(__uint_as_float(sv[xl]), __uint_as_float(sv[xl + 1])),
+                                                           sc2, bf16x2_to_f2(bw[cc * 4 + e]));
+                                    float2 y = ffma2(t, l2e, nl2);
+                                    if constexpr (kMasked) y = fadd2(y, make_float2(mk[2 * e], mk[2 * e + 1]));
+                                    // in key tiles without a mask, one pair in four takes the FMA-pipe exponential
+                                    const float2 pp = (!kMasked && e == 3) ? ex2_fma2(y) : make_float2(ex2(y.x), ex2(y.y));
+                                    const float2 ds = fmul2(pp, fadd2(make_float2(__uint_as_float(dv[xl]),
+                                                                                  __uint_as_float(dv[xl + 1])), nD2));
+                                    pw[cc * 4 + e] = pack_bf16(pp.x, pp.y);
+                                    dw[cc * 4 + e] = pack_bf16(ds.x, ds.y);
+                                }
                             }
                         }
                     };
                     if (has_mask) tile(std::true_type{});
                     else tile(std::false_type{});
                     TRI_TP(4)
-                    // the previous tile's gradient MMAs have finished reading P and dS
+                    // the gradient MMAs of two tiles ago have finished reading this P/dS buffer
                     const int pb = g & 1;  // P/dS buffer of this tile (the other one may still be read)
                     if (g >= 2 && !mbar_wait_warp(BAR(L::B_PDSFREE + pb), ((g >> 1) - 1) & 1, wc, 15)) { ok = false; break; }
                     TRI_TP(3)
-                    const uint32_t prow = sb + L::OFF_PDS + pb * L::PDS_BUF + w * (L::PT_TILE / 2) + row * 128;
+                    // this warpgroup's 32 keys = four 16-byte chunks of one 64-key SW128 half
+                    const uint32_t prow = sb + L::OFF_PDS + pb * L::PDS_BUF + (w >> 1) * (L::PT_TILE / 2) + row * 128;
                     const uint32_t drow = prow + L::PT_TILE;
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint32_t off = (c ^ (row & 7)) << 4;
+                    for (int c = 0; c < 4; ++c) {
+                        const uint32_t off = ((((w & 1) * 4) + c) ^ (row & 7)) << 4;
                         sts128(prow + off, make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]));
                         sts128(drow + off, make_uint4(dw[4 * c], dw[4 * c + 1], dw[4 * c + 2], dw[4 * c + 3]));
                     }
@@ -723,7 +732,7 @@ __global__ void __launch_bounds__(384, 1)
     }
 
     tc_fence_before();
-    cta_end_barrier();
+    cta_end_barrier640();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
