@@ -650,45 +650,41 @@ __global__ void __launch_bounds__(640, 1)
                     uint32_t pw[16], dw[16];
                     const float2 sc2 = make_float2(scale, scale), l2e = make_float2(LOG2E, LOG2E);
                     const float2 nl2 = make_float2(-lse2, -lse2), nD2 = make_float2(-Dj, -Dj);
+                    // all 32 keys of S and dP first, so the S/dP columns are released to the MMA
+                    // warp before any arithmetic
+                    uint32_t sv[32], dv[32];
+                    tmem_ld32(tl + L::T_S + w * 32, sv);
+                    tmem_ld32(tl + L::T_DP + w * 32, dv);
+                    tmem_wait_ld();
+                    reg_fence32(sv);
+                    reg_fence32(dv);
+                    TRI_TP(1)
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(BAR(L::B_SDPFREE));
                     auto tile = [&](auto masked) {
                         constexpr bool kMasked = decltype(masked)::value;
 #pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            uint32_t sv[16], dv[16];
-                            tmem_ld16(tl + L::T_S + w * 32 + hh * 16, sv);
-                            tmem_ld16(tl + L::T_DP + w * 32 + hh * 16, dv);
-                            tmem_wait_ld();
-                            reg_fence16(sv);
-                            reg_fence16(dv);
-                            if (hh == 1) {
-                                TRI_TP(1)
-                                tc_fence_before();
-                                __syncwarp();
-                                if (lane == 0) mbar_arrive(BAR(L::B_SDPFREE));
+                        for (int cc = 0; cc < 4; ++cc) {  // 8-key chunks of this warpgroup's 32 keys
+                            float mk[8];
+                            if constexpr (kMasked) {
+                                const float4 m0 = lds128f(maskv + cc * 32), m1 = lds128f(maskv + cc * 32 + 16);
+                                mk[0] = m0.x; mk[1] = m0.y; mk[2] = m0.z; mk[3] = m0.w;
+                                mk[4] = m1.x; mk[5] = m1.y; mk[6] = m1.z; mk[7] = m1.w;
                             }
 #pragma unroll
-                            for (int c = 0; c < 2; ++c) {
-                                const int cc = hh * 2 + c;  // 8-key chunk of this warpgroup's 32 keys
-                                float mk[8];
-                                if constexpr (kMasked) {
-                                    const float4 m0 = lds128f(maskv + cc * 32), m1 = lds128f(maskv + cc * 32 + 16);
-                                    mk[0] = m0.x; mk[1] = m0.y; mk[2] = m0.z; mk[3] = m0.w;
-                                    mk[4] = m1.x; mk[5] = m1.y; mk[6] = m1.z; mk[7] = m1.w;
-                                }
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    const int xl = c * 8 + 2 * e;
-                                    const float2 t = ffma2(make_float2(__uint_as_float(sv[xl]), __uint_as_float(sv[xl + 1])),
-                                                           sc2, bf16x2_to_f2(bw[cc * 4 + e]));
-                                    float2 y = ffma2(t, l2e, nl2);
-                                    if constexpr (kMasked) y = fadd2(y, make_float2(mk[2 * e], mk[2 * e + 1]));
-                                    // in key tiles without a mask, one pair in four takes the FMA-pipe exponential
-                                    const float2 pp = (!kMasked && e == 3) ? ex2_fma2(y) : make_float2(ex2(y.x), ex2(y.y));
-                                    const float2 ds = fmul2(pp, fadd2(make_float2(__uint_as_float(dv[xl]),
-                                                                                  __uint_as_float(dv[xl + 1])), nD2));
-                                    pw[cc * 4 + e] = pack_bf16(pp.x, pp.y);
-                                    dw[cc * 4 + e] = pack_bf16(ds.x, ds.y);
-                                }
+                            for (int e = 0; e < 4; ++e) {
+                                const int xl = cc * 8 + 2 * e;
+                                const float2 t = ffma2(make_float2(__uint_as_float(sv[xl]), __uint_as_float(sv[xl + 1])),
+                                                       sc2, bf16x2_to_f2(bw[cc * 4 + e]));
+                                float2 y = ffma2(t, l2e, nl2);
+                                if constexpr (kMasked) y = fadd2(y, make_float2(mk[2 * e], mk[2 * e + 1]));
+                                // in key tiles without a mask, one pair in four takes the FMA-pipe exponential
+                                const float2 pp = (!kMasked && e == 3) ? ex2_fma2(y) : make_float2(ex2(y.x), ex2(y.y));
+                                const float2 ds = fmul2(pp, fadd2(make_float2(__uint_as_float(dv[xl]),
+                                                                              __uint_as_float(dv[xl + 1])), nD2));
+                                pw[cc * 4 + e] = pack_bf16(pp.x, pp.y);
+                                dw[cc * 4 + e] = pack_bf16(ds.x, ds.y);
                             }
                         }
                     };
