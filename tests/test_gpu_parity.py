@@ -195,6 +195,32 @@ def test_uncompensated_variant_runs_and_stays_within_gates():
     check_full(x, got)
 
 
+@pytest.mark.parametrize("wl", [S.Workload("ablation N=256 bias 2N(0,1)", 1, 256, 4, 32, bias_std=2.0, mask="zeros"),
+                                S.Workload("ablation N=200 ragged", 1, 200, 4, 32, mask="ragged", len_lo=150,
+                                           len_hi=200)],
+                         ids=["N256", "N200ragged"])
+def test_residual_compensation_ablation(wl, capsys):
+    """The output-rounding residual (D formed in FP32 from o + resid, versus from the
+    BF16 output o alone; TurboPairFormer pages, "residual compensation").  Measured
+    against the FP64 oracle: dV does not involve D and must be bitwise identical;
+    dQ, dK and dBias must come out closer to the exact gradients with the residual."""
+    x = S.make_inputs(wl, 21)
+    comp = run_gpu(x, "start")
+    unc = run_gpu(x, "start", flags=Bd.TRI_ATTN_BWD_NO_RESIDUAL)
+    assert torch.equal(comp["dv"], unc["dv"])
+    q, k, v, bias, mask, do = oracle_inputs(x, "start")
+    dq, dk, dv, db = O.bwd(q, k, v, bias, mask, do)
+    ref = {"dq": dq, "dk": dk, "dbias": db}
+    e_c = {n: rel(comp[n].numpy(), ref[n]) for n in ref}
+    e_u = {n: rel(unc[n].numpy(), ref[n]) for n in ref}
+    with capsys.disabled():
+        print(f"\n[{wl.name}] rel-RMSE vs FP64, compensated / uncompensated: " +
+              ", ".join(f"{n} {e_c[n]:.3e} / {e_u[n]:.3e} ({100 * (1 - e_c[n] / e_u[n]):+.1f}%)" for n in ref))
+    for n in ref:
+        assert e_c[n] <= GATES[n] and e_u[n] <= GATES[n], n
+        assert e_c[n] < e_u[n], f"{n}: residual did not reduce the error ({e_c[n]:.3e} vs {e_u[n]:.3e})"
+
+
 def test_bounded_wait_expires_and_context_survives():
     Bd.tri_attn_device_error(True)
     Bd.tri_attn_set_wait_limit_ns(2_000_000)  # 2 ms
