@@ -120,13 +120,16 @@ __global__ void __launch_bounds__(256) tri_attn_bwd_prep_kernel(
     for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < n1 + n2 + n3;
          idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         if (idx < n1) {
+            // head fastest: neighbouring threads read the heads of one pair row, which are
+            // contiguous in memory, so a warp streams whole 256-byte rows
             int64_t t = idx;
+            const int h = static_cast<int>(t % H);
+            t /= H;
             const int j = static_cast<int>(t % Np);
             t /= Np;
             const int i = static_cast<int>(t % N);
-            t /= N;
-            const int h = static_cast<int>(t % H);
-            const int b = static_cast<int>(t / H);
+            const int b = static_cast<int>(t / N);
+            const int64_t out = ((static_cast<int64_t>(b) * H + h) * N + i) * Np + j;
             float dsum = 0.f, lv = INFINITY;
             if (j < N) {
                 const uint4* pd = reinterpret_cast<const uint4*>(dout + b * s0 + i * s1 + j * s2 + h * s3);
@@ -147,8 +150,8 @@ __global__ void __launch_bounds__(256) tri_attn_bwd_prep_kernel(
                 }
                 lv = __ldg(lse + ((static_cast<int64_t>(b) * H + h) * N + i) * N + j) * LOG2E;
             }
-            Dv[idx] = dsum;
-            Lv[idx] = lv;
+            Dv[out] = dsum;
+            Lv[out] = lv;
         } else if (idx < n1 + n2) {
             const int64_t e = idx - n1;
             const int k = static_cast<int>(e % Np);
