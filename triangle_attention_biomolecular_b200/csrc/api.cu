@@ -341,7 +341,9 @@ tri_attn_status tri_attn_fwd(const tri_attn_fwd_args* a, tri_attn_stream_t strea
     for (int x = 0; x < 5; ++x) { p.os[x] = a->o.stride[x]; p.rs[x] = a->resid.stride[x]; }
     p.lse = a->lse;
     p.wait_limit_ns = g_wait_limit_ns.load();
-    const unsigned grid = static_cast<unsigned>(B) * p.npairs * H * p.nt;
+    // persistent grid: one CTA per SM (148 on B200), each walking work items
+    const int64_t items = static_cast<int64_t>(B) * p.npairs * H * p.nt;
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(items, 148));
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (d == 32)
         tri::tri_attn_fwd_kernel<32><<<grid, 384, tri::FwdLayout<32>::SMEM, s>>>(mq, mk, mv, mb, p);

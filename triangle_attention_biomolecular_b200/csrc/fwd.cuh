@@ -64,7 +64,7 @@ struct FwdLayout {
     // barrier indices
     static constexpr int B_Q = 0, B_FULL = 1, B_EMPTY = 1 + NS, B_SFULL = 1 + 2 * NS,
                          B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2, B_PVDONE = B_PFULL + 2,
-                         B_EXPD = B_PVDONE + 2, B_DRAIN = B_EXPD + 2, NBAR = B_DRAIN + 1;
+                         B_EXPD = B_PVDONE + 2, B_QFREE = B_EXPD + 2, B_DRAIN = B_QFREE + 1, NBAR = B_DRAIN + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag, mask flags[NS][2]
     static constexpr int SMEM = OFF_MISC + 16 + NS * 2 * 4;
     static_assert(SMEM <= 232448, "shared memory budget");
@@ -110,17 +110,28 @@ __global__ void __launch_bounds__(384, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
     volatile int* mask_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 16);
 
-    // ---- work item: (b, h, pair of rows, query tile), query tile fastest ----
-    int item = blockIdx.x;
-    const int jt = item % p.nt;
-    item /= p.nt;
-    const int ip = item % p.npairs;
-    item /= p.npairs;
-    const int h = item % p.H;
-    const int b = item / p.H;
-    const int i0 = 2 * ip;
-    const int i1 = min(2 * ip + 1, p.N - 1);
-    const bool has1 = (2 * ip + 1) < p.N;
+    // ---- work items (b, h, pair of rows, query tile), query tile fastest.  The grid is
+    // persistent: CTA c takes items c, c + gridDim.x, ..., and every barrier phase runs
+    // on counters that continue across items, so the producer fills the next item's Q
+    // and first stages while the softmax warps finish the current one. ----
+    struct Item {
+        int jt, h, b, i0, i1;
+        bool has1;
+    };
+    auto decode = [&](int item) {
+        Item t;
+        t.jt = item % p.nt;
+        item /= p.nt;
+        const int ip = item % p.npairs;
+        item /= p.npairs;
+        t.h = item % p.H;
+        t.b = item / p.H;
+        t.i0 = 2 * ip;
+        t.i1 = min(2 * ip + 1, p.N - 1);
+        t.has1 = (2 * ip + 1) < p.N;
+        return t;
+    };
+    const int items = p.B * p.npairs * p.H * p.nt;
     const int nkt = p.nt;
 
     if (threadIdx.x == 0) {
@@ -141,6 +152,7 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(BAR(L::B_PVDONE + w), 1);
             mbar_init(BAR(L::B_EXPD + w), 4);
         }
+        mbar_init(BAR(L::B_QFREE), 1);
         mbar_init(BAR(L::B_DRAIN), 1);
         fence_mbar_init();
     }
@@ -161,12 +173,7 @@ __global__ void __launch_bounds__(384, 1)
         int armed[L::NS];
 #pragma unroll
         for (int s = 0; s < L::NS; ++s) armed[s] = 0;
-        auto load_qkv = [&](uint32_t dst, const CUtensorMap* m, uint32_t bar, int i, int j0) {
-            tma_load_5d(dst, m, bar, 0, h, j0, i, b);
-        };
-        auto load_bias = [&](uint32_t dst, uint32_t bar, int k0, int j0) {
-            tma_load_4d(dst, &tm_bias, bar, k0, j0, h, b);
-        };
+        int nq = 0;  // Q loads issued
         const bool leader = elect_one();
         if (!aborted_early) {
             if (leader) {
@@ -174,64 +181,83 @@ __global__ void __launch_bounds__(384, 1)
                 tma_prefetch_map(&tm_k);
                 tma_prefetch_map(&tm_v);
                 tma_prefetch_map(&tm_bias);
-                mbar_arrive_expect_tx(BAR(L::B_Q), 2 * L::QKV_TILE);
-                load_qkv(sb + L::OFF_Q, &tm_q, BAR(L::B_Q), i0, jt * 128);
-                load_qkv(sb + L::OFF_Q + L::QKV_TILE, &tm_q, BAR(L::B_Q), i1, jt * 128);
             }
-            // key-mask rows (user mask, -inf past N) are fetched one stage ahead so
-            // their latency overlaps the wait for a free stage
-            float mnext[2][4];
-            auto fetch_mask = [&](int kt) {
-#pragma unroll
-                for (int w = 0; w < 2; ++w) {
-                    const int i = w ? i1 : i0;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int k = kt * 128 + lane * 4 + e;
-                        float x = -INFINITY;
-                        if (k < p.N) x = p.mask ? __ldg(p.mask + b * p.ms0 + i * p.ms1 + k * p.ms2) : 0.f;
-                        mnext[w][e] = x;
-                    }
-                }
-            };
+            int gs = 0;  // stage fills so far
+            bool ok = true;
             TRI_TRACE_DECL
-            fetch_mask(0);
-            for (int kt = 0; kt < nkt; ++kt) {
-                const int s = kt % L::NS;
-                TRI_TP(1)
-                if (kt >= L::NS && !mbar_wait_warp(BAR(L::B_EMPTY + s), ((kt / L::NS) - 1) & 1, wc, 1)) break;
-                TRI_TP(0)
-                const uint32_t st = sb + L::OFF_STAGES + s * L::STAGE;
+            for (int item = blockIdx.x; ok && item < items; item += gridDim.x) {
+                const Item t = decode(item);
+                auto load_qkv = [&](uint32_t dst, const CUtensorMap* m, uint32_t bar, int i, int j0) {
+                    tma_load_5d(dst, m, bar, 0, t.h, j0, i, t.b);
+                };
+                auto load_bias = [&](uint32_t dst, uint32_t bar, int k0, int j0) {
+                    tma_load_4d(dst, &tm_bias, bar, k0, j0, t.h, t.b);
+                };
+                // key-mask rows (user mask, -inf past N) are fetched one stage ahead so
+                // their latency overlaps the wait for a free stage
+                float mnext[2][4];
+                auto fetch_mask = [&](int kt) {
 #pragma unroll
-                for (int w = 0; w < 2; ++w) {
-                    bool nz = false;
+                    for (int w = 0; w < 2; ++w) {
+                        const int i = w ? t.i1 : t.i0;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) nz |= (mnext[w][e] != 0.f);
-                    float4* dst = reinterpret_cast<float4*>(smem + (st - sb) + L::OFF_MASK + w * 512 + lane * 16);
-                    *dst = make_float4(mnext[w][0], mnext[w][1], mnext[w][2], mnext[w][3]);
-                    const unsigned any = __any_sync(0xFFFFFFFFu, nz);
-                    if (lane == 0) mask_flag[s * 2 + w] = any ? 1 : 0;
-                }
-                __syncwarp();
+                        for (int e = 0; e < 4; ++e) {
+                            const int k = kt * 128 + lane * 4 + e;
+                            float x = -INFINITY;
+                            if (k < p.N) x = p.mask ? __ldg(p.mask + t.b * p.ms0 + i * p.ms1 + k * p.ms2) : 0.f;
+                            mnext[w][e] = x;
+                        }
+                    }
+                };
+                fetch_mask(0);
+                // this item's Q tiles, once the previous item's S products have read the old ones
+                if (nq > 0 && !mbar_wait_warp(BAR(L::B_QFREE), (nq - 1) & 1, wc, 13)) { ok = false; break; }
                 if (leader) {
-                    const uint32_t bar = BAR(L::B_FULL + s);
-                    mbar_arrive_expect_tx(bar, 4 * L::QKV_TILE + L::BIAS_TILE);
-                    load_qkv(st + L::OFF_K0, &tm_k, bar, i0, kt * 128);
-                    load_qkv(st + L::OFF_V0, &tm_v, bar, i0, kt * 128);
-                    load_qkv(st + L::OFF_K1, &tm_k, bar, i1, kt * 128);
-                    load_qkv(st + L::OFF_V1, &tm_v, bar, i1, kt * 128);
-                    load_bias(st + L::OFF_BIAS, bar, kt * 128, jt * 128);
-                    load_bias(st + L::OFF_BIAS + L::BIAS_TILE / 2, bar, kt * 128 + 64, jt * 128);
+                    mbar_arrive_expect_tx(BAR(L::B_Q), 2 * L::QKV_TILE);
+                    load_qkv(sb + L::OFF_Q, &tm_q, BAR(L::B_Q), t.i0, t.jt * 128);
+                    load_qkv(sb + L::OFF_Q + L::QKV_TILE, &tm_q, BAR(L::B_Q), t.i1, t.jt * 128);
                 }
-                armed[s]++;
-                if (kt + 1 < nkt) fetch_mask(kt + 1);
+                ++nq;
+                for (int kt = 0; kt < nkt; ++kt, ++gs) {
+                    const int s = gs % L::NS;
+                    TRI_TP(1)
+                    if (gs >= L::NS && !mbar_wait_warp(BAR(L::B_EMPTY + s), ((gs / L::NS) - 1) & 1, wc, 1)) {
+                        ok = false;
+                        break;
+                    }
+                    TRI_TP(0)
+                    const uint32_t st = sb + L::OFF_STAGES + s * L::STAGE;
+#pragma unroll
+                    for (int w = 0; w < 2; ++w) {
+                        bool nz = false;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) nz |= (mnext[w][e] != 0.f);
+                        float4* dst = reinterpret_cast<float4*>(smem + (st - sb) + L::OFF_MASK + w * 512 + lane * 16);
+                        *dst = make_float4(mnext[w][0], mnext[w][1], mnext[w][2], mnext[w][3]);
+                        const unsigned any = __any_sync(0xFFFFFFFFu, nz);
+                        if (lane == 0) mask_flag[s * 2 + w] = any ? 1 : 0;
+                    }
+                    __syncwarp();
+                    if (leader) {
+                        const uint32_t bar = BAR(L::B_FULL + s);
+                        mbar_arrive_expect_tx(bar, 4 * L::QKV_TILE + L::BIAS_TILE);
+                        load_qkv(st + L::OFF_K0, &tm_k, bar, t.i0, kt * 128);
+                        load_qkv(st + L::OFF_V0, &tm_v, bar, t.i0, kt * 128);
+                        load_qkv(st + L::OFF_K1, &tm_k, bar, t.i1, kt * 128);
+                        load_qkv(st + L::OFF_V1, &tm_v, bar, t.i1, kt * 128);
+                        load_bias(st + L::OFF_BIAS, bar, kt * 128, t.jt * 128);
+                        load_bias(st + L::OFF_BIAS + L::BIAS_TILE / 2, bar, kt * 128 + 64, t.jt * 128);
+                    }
+                    armed[s]++;
+                    if (kt + 1 < nkt) fetch_mask(kt + 1);
+                }
             }
             TRI_TP(1)
             TRI_TRACE_FLUSH_AT(0)
         }
         // never leave with bulk copies still writing into this CTA's shared memory
         if (leader) {
-            if (!aborted_early) drain_wait(BAR(L::B_Q), 0, 100000000ull);
+            if (nq > 0) drain_wait(BAR(L::B_Q), (nq - 1) & 1, 100000000ull);
 #pragma unroll
             for (int s = 0; s < L::NS; ++s)
                 if (armed[s] > 0) drain_wait(BAR(L::B_FULL + s), (armed[s] - 1) & 1, 100000000ull);
@@ -262,59 +288,67 @@ __global__ void __launch_bounds__(384, 1)
                 __syncwarp();
             };
             TRI_TRACE_DECL
-            bool ok = mbar_wait_warp(BAR(L::B_Q), 0, wc, 2);
-            TRI_TP(9)
-            for (int kt = 0; ok && kt < nkt; ++kt) {
-                const int s = kt % L::NS;
-                TRI_TP(4)
-                if (!mbar_wait_warp(BAR(L::B_FULL + s), (kt / L::NS) & 1, wc, 3)) { ok = false; break; }
-                TRI_TP(0)
-                tc_fence_after();
-#pragma unroll
-                for (int w = 0; w < 2; ++w) {
-                    if (kt > 0) {
-                        TRI_TP(4)
-                        if (!mbar_wait_warp(BAR(L::B_SFREE + w), (kt - 1) & 1, wc, 4)) { ok = false; break; }
-                        TRI_TP(1)
-                        tc_fence_after();
-                    }
-                    const uint64_t qd = desc_add(dq0, w * L::QKV_TILE);
-                    const uint64_t kd = desc_add(dst0, s * L::STAGE + (w ? L::OFF_K1 : L::OFF_K0));
-                    if (leader) {
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk)
-                            mma_ss(tmem + w * 256, desc_add(qd, kk * 32), desc_add(kd, kk * 32), IDESC_QK,
-                                   kk > 0 ? 1u : 0u);
-                        mma_commit(BAR(L::B_SFULL + w));
-                    }
-                    __syncwarp();
-                }
-                if (!ok) break;
-                if (kt > 0) {
-                    const int sp = (kt - 1) % L::NS;
+            bool ok = true;
+            int gs = 0, gt = 0, it = 0;  // stages consumed, tiles, items (all continue across items)
+            for (int item = blockIdx.x; ok && item < items; item += gridDim.x, ++it) {
+                if (!mbar_wait_warp(BAR(L::B_Q), it & 1, wc, 2)) { ok = false; break; }
+                TRI_TP(9)
+                for (int kt = 0; kt < nkt; ++kt, ++gs, ++gt) {
+                    const int s = gs % L::NS;
+                    TRI_TP(4)
+                    if (!mbar_wait_warp(BAR(L::B_FULL + s), (gs / L::NS) & 1, wc, 3)) { ok = false; break; }
+                    TRI_TP(0)
+                    tc_fence_after();
 #pragma unroll
                     for (int w = 0; w < 2; ++w) {
-                        TRI_TP(4)
-                        if (!mbar_wait_warp(BAR(L::B_PFULL + w), (kt - 1) & 1, wc, 5)) { ok = false; break; }
-                        TRI_TP(2)
-                        tc_fence_after();
-                        issue_pv(w, sp, kt - 1);
+                        if (gt > 0) {
+                            TRI_TP(4)
+                            if (!mbar_wait_warp(BAR(L::B_SFREE + w), (gt - 1) & 1, wc, 4)) { ok = false; break; }
+                            TRI_TP(1)
+                            tc_fence_after();
+                        }
+                        const uint64_t qd = desc_add(dq0, w * L::QKV_TILE);
+                        const uint64_t kd = desc_add(dst0, s * L::STAGE + (w ? L::OFF_K1 : L::OFF_K0));
+                        if (leader) {
+#pragma unroll
+                            for (int kk = 0; kk < D / 16; ++kk)
+                                mma_ss(tmem + w * 256, desc_add(qd, kk * 32), desc_add(kd, kk * 32), IDESC_QK,
+                                       kk > 0 ? 1u : 0u);
+                            mma_commit(BAR(L::B_SFULL + w));
+                        }
+                        __syncwarp();
                     }
                     if (!ok) break;
-                    if (leader) mma_commit(BAR(L::B_EMPTY + sp));
-                    __syncwarp();
+                    if (kt == nkt - 1) {  // the item's last S products: Q is free once they finish
+                        if (leader) mma_commit(BAR(L::B_QFREE));
+                        __syncwarp();
+                    }
+                    if (kt > 0) {
+                        const int sp = (gs - 1) % L::NS;
+#pragma unroll
+                        for (int w = 0; w < 2; ++w) {
+                            TRI_TP(4)
+                            if (!mbar_wait_warp(BAR(L::B_PFULL + w), (gt - 1) & 1, wc, 5)) { ok = false; break; }
+                            TRI_TP(2)
+                            tc_fence_after();
+                            issue_pv(w, sp, kt - 1);
+                        }
+                        if (!ok) break;
+                        if (leader) mma_commit(BAR(L::B_EMPTY + sp));
+                        __syncwarp();
+                    }
                 }
-            }
-            if (ok) {
-                const int kl = nkt - 1;
-                const int sp = kl % L::NS;
+                if (!ok) break;
+                // the item's last PV
+                const int sp = (gs - 1) % L::NS;
 #pragma unroll
                 for (int w = 0; w < 2; ++w) {
-                    if (!mbar_wait_warp(BAR(L::B_PFULL + w), kl & 1, wc, 5)) { ok = false; break; }
+                    if (!mbar_wait_warp(BAR(L::B_PFULL + w), (gt - 1) & 1, wc, 5)) { ok = false; break; }
                     tc_fence_after();
-                    issue_pv(w, sp, kl);
+                    issue_pv(w, sp, nkt - 1);
                 }
-                if (ok && leader) mma_commit(BAR(L::B_EMPTY + sp));
+                if (!ok) break;
+                if (leader) mma_commit(BAR(L::B_EMPTY + sp));
                 __syncwarp();
             }
             TRI_TP(5)
@@ -336,17 +370,21 @@ __global__ void __launch_bounds__(384, 1)
         const int row = qd * 32 + lane;
         const uint32_t tS = tmem + (static_cast<uint32_t>(qd * 32) << 16) + w * 256;
         const uint32_t tP = tS + 128, tO = tS + 192;
-        const int j = jt * 128 + row;
-        const int i = w ? i1 : i0;
         const float scale = p.scale;
         constexpr float LOG2E = 1.4426950408889634f;
         constexpr float RESCALE_AT = 5.545177444479562f;  // 8 * ln 2
-        float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
+        int gs = 0, gt = 0;  // stages and tiles consumed, continuing across items
         TRI_TRACE_DECL
-        for (int kt = 0; kt < nkt; ++kt) {
-            const int s = kt % L::NS;
-            if (!mbar_wait_warp(BAR(L::B_SFULL + w), kt & 1, wc, 6)) { ok = false; break; }
+        for (int item = blockIdx.x; ok && item < items; item += gridDim.x) {
+        const Item t = decode(item);
+        const int j = t.jt * 128 + row;
+        const int i = w ? t.i1 : t.i0;
+        const int b = t.b, h = t.h;
+        float m_ref = -INFINITY, l = 0.f;
+        for (int kt = 0; kt < nkt; ++kt, ++gs, ++gt) {
+            const int s = gs % L::NS;
+            if (!mbar_wait_warp(BAR(L::B_SFULL + w), gt & 1, wc, 6)) { ok = false; break; }
             if (kt == 0) { TRI_TP(9) } else { TRI_TP(0) }
             tc_fence_after();
             uint32_t r0[32], r1[32], r2[32], r3[32];
@@ -363,7 +401,7 @@ __global__ void __launch_bounds__(384, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(BAR(L::B_SFREE + w));
-            if (!mbar_wait_warp(BAR(L::B_FULL + s), (kt / L::NS) & 1, wc, 7)) { ok = false; break; }
+            if (!mbar_wait_warp(BAR(L::B_FULL + s), (gs / L::NS) & 1, wc, 7)) { ok = false; break; }
             TRI_TP(2)
             const uint32_t st = sb + L::OFF_STAGES + s * L::STAGE;
             float x[128];
@@ -430,8 +468,8 @@ __global__ void __launch_bounds__(384, 1)
             // Ping-pong on the exponential unit: the two warpgroups take turns
             // (WG0 tile kt, WG1 tile kt, WG0 tile kt+1, ...), so one runs its
             // exponentials while the other loads, biases and reduces its next tile.
-            if (w == 1 || kt > 0) {
-                const int turn = w == 1 ? kt : kt - 1;
+            if (w == 1 || gt > 0) {
+                const int turn = w == 1 ? gt : gt - 1;
                 if (!mbar_wait_warp(BAR(L::B_EXPD + (1 - w)), turn & 1, wc, 10)) { ok = false; break; }
             }
             // probabilities into packed BF16 registers first; the previous PV may still be
@@ -464,7 +502,7 @@ __global__ void __launch_bounds__(384, 1)
             TRI_TP(5)
             if (kt > 0) {
                 // PV of the previous tile has finished: the P columns are free and O is stable
-                if (!mbar_wait_warp(BAR(L::B_PVDONE + w), (kt - 1) & 1, wc, 8)) { ok = false; break; }
+                if (!mbar_wait_warp(BAR(L::B_PVDONE + w), (gt - 1) & 1, wc, 8)) { ok = false; break; }
                 tc_fence_after();
             }
             TRI_TP(4)
@@ -495,9 +533,11 @@ __global__ void __launch_bounds__(384, 1)
             if (lane == 0) mbar_arrive(BAR(L::B_PFULL + w));
             TRI_TP(7)
         }
-        if (ok && mbar_wait_warp(BAR(L::B_PVDONE + w), (nkt - 1) & 1, wc, 9)) {
+        if (!ok) break;
+        if (!mbar_wait_warp(BAR(L::B_PVDONE + w), (gt - 1) & 1, wc, 9)) { ok = false; break; }
+        {
             tc_fence_after();
-            const bool store = (j < p.N) && (w == 0 || has1);
+            const bool store = (j < p.N) && (w == 0 || t.has1);
             const float inv_l = __frcp_rn(l);
             __nv_bfloat16* op = p.o + b * p.os[0] + i * p.os[1] + j * p.os[2] + h * p.os[3];
             __nv_bfloat16* rp = p.r + b * p.rs[0] + i * p.rs[1] + j * p.rs[2] + h * p.rs[3];
@@ -529,6 +569,7 @@ __global__ void __launch_bounds__(384, 1)
                     m_ref + lg2(l) * 0.6931471805599453f;
             }
         }
+        }  // items
         TRI_TP(8)
         TRI_TRACE_FLUSH_AT(0)
     }
