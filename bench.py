@@ -296,6 +296,90 @@ def run_ours(args, rank, world, local_rank):
 
 
 # ---------------------------------------------------------------------------
+# second operation: the triangle multiplicative contraction (--op tri_mul)
+# ---------------------------------------------------------------------------
+TRI_MUL_METRIC = "tri-mul contraction fwd+bwd TFLOP/s at N=768, C=128 pair channels, BF16"
+
+
+def run_tri_mul(args, rank, world, local_rank):
+    """One step = forward x = a (x) b over k (outgoing edges) and the backward da, db:
+    three batched N x N x N products per channel, 6*B*C*N^3 flops."""
+    import torch
+    import torch.distributed as dist
+    from triangle_attention_biomolecular_b200 import _binding as Bd
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    Bn, C, N = 1, 128, 768
+    g = torch.Generator().manual_seed(1000 + rank)
+    a, b, dx = (torch.randn((Bn, C, N, N), generator=g).to(torch.bfloat16).to(dev) for _ in range(3))
+    x, da, db = torch.empty_like(a), torch.empty_like(a), torch.empty_like(a)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        Bd.tri_mul_fwd(a, b, x, False, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        Bd.tri_mul_bwd(a, b, dx, da, db, False, stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for s_ in range(args.steps):
+        step(evs[s_])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    st, word = Bd.tri_attn_device_error(True)
+    if st != 0:
+        raise RuntimeError(f"device error word {word:#x}")
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    return {"ms": ms, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "clocks": clocks, "shape": (Bn, C, N)}
+
+
+def tri_mul_cpu_baseline(target_s: float = 10.0):
+    """The FP64 oracle on the host cores over a bounded number of channels."""
+    import numpy as np
+    from oracle import tri_mul_oracle as T
+    N = 768
+    rng = np.random.default_rng(0)
+    a, b, dx = (rng.standard_normal((1, 1, N, N)) for _ in range(3))
+
+    def one():
+        t = time.perf_counter()
+        T.fwd(a, b, "outgoing")
+        T.bwd(a, b, dx, "outgoing")
+        return time.perf_counter() - t
+    one()
+    t1 = one()
+    n = int(max(1, min(128, round(target_s / max(t1, 1e-4)))))
+    t = sum(one() for _ in range(n))
+    return {"value": round(6.0 * N ** 3 * n / t / 1e12, 6), "unit": "TFLOP/s", "cores": os.cpu_count(),
+            "kind": "oracle", "seconds": round(t, 3),
+            "sample": f"{n} of the 128 channels at N=768: FP64 oracle forward + backward (numpy matmul)"}
+
+
+# ---------------------------------------------------------------------------
 # the oracle on host cores (CPU baseline and the reference arm)
 # ---------------------------------------------------------------------------
 def oracle_sample(rows_n: int):
@@ -372,6 +456,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", choices=("crop768", "crop640", "crop384"), default="crop768",
                     help="crop768 is the headline; the smaller crops serve profiler captures")
+    ap.add_argument("--op", choices=("attention", "tri_mul"), default="attention",
+                    help="attention (the headline) or the triangle multiplicative contraction")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle on host cores")
     args = ap.parse_args()
@@ -392,11 +478,42 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        res = run_ours(args, rank, world, local_rank)
+        if args.op == "tri_mul":
+            res = run_tri_mul(args, rank, world, local_rank)
+        else:
+            res = run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
             dist.destroy_process_group()
     if rank != 0:
+        return
+    if args.op == "tri_mul":
+        Bn, C, N = res["shape"]
+        pk, src = peaks()
+        peak = float(pk["bf16_tflops"])
+        step_flops = 6.0 * Bn * C * N ** 3
+        value = world * step_flops * args.steps / (res["ms"] * 1e-3) / 1e12
+        fwd_t = 2.0 * Bn * C * N ** 3 / (res["fwd_ms"] * 1e-3) / 1e12
+        bwd_t = 4.0 * Bn * C * N ** 3 / (res["bwd_ms"] * 1e-3) / 1e12
+        line = {
+            "metric": TRI_MUL_METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(res["ms"] / args.steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "triangle multiplicative contraction, outgoing edges: B=1, C=128, N=768, BF16 "
+                                   "(forward + backward, three batched N^3 products per channel)",
+                       "flops_per_step": step_flops, "l2": "inputs (453 MB) larger than the 126 MB L2; no flush"},
+            "kernels_ms": {"fwd": round(res["fwd_ms"], 4), "bwd": round(res["bwd_ms"], 4)},
+            "roofline": {"kernel": "tri_mul_gemm (fwd)", "bound": "tensor", "achieved": round(fwd_t, 2), "peak": peak,
+                         "unit": "TFLOP/s", "frac": round(fwd_t / peak, 4), "traffic": None,
+                         "peak_source": f"{src} bf16_tflops (burst)"},
+            "bwd_tflops": round(bwd_t, 2),
+            "gpu_launches": 3 * args.steps,
+            "clocks": res["clocks"],
+            "e2e": None,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = tri_mul_cpu_baseline()
+        print(json.dumps(line), flush=True)
         return
     Bn, N, H, d = res["shape"]
     fl = flops(Bn, N, H, d)

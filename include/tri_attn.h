@@ -201,6 +201,50 @@ tri_attn_status tri_attn_bwd_marked(const tri_attn_bwd_args *args, tri_attn_stre
  */
 tri_attn_status tri_attn_bwd_static_scratch(const tri_attn_bwd_args *args, tri_attn_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Triangle multiplicative update: the contraction step.
+ *
+ * The pages name the Triangle Multiplicative Update as the second operation
+ * TurboPairFormer optimises beside triangle attention (page A, opening
+ * paragraph; page B, the paragraph introducing TurboPairFormer) without a
+ * formula; read the AlphaFold way, its only cubic step contracts two projected
+ * pair tensors over the third residue k, for every batch b and channel c:
+ *   outgoing edges (flags 0):            x[b,c,i,j] = sum_k a[b,c,i,k] b[b,c,j,k]
+ *   incoming edges (TRI_MUL_INCOMING):   x[b,c,i,j] = sum_k a[b,c,k,i] b[b,c,k,j]
+ * The projections, gates and LayerNorms around it are per-position work of the
+ * model and are not part of this call.
+ *   a, b, x : BF16 [B,C,N,N], channel-first (the caller permutes the
+ *             channel-last pair representation), strides as tri_attn_tensor4
+ *             with (b, c, row, col) in place of (b, h, j, k): innermost stride
+ *             1, the others non-negative multiples of 8 elements, pointers
+ *             16-byte aligned
+ *   x       : output, BF16 round-to-nearest-even of the FP32 sum
+ * Sizes: 1 <= B, 1 <= C, B*C <= 65535, 1 <= N <= 16384.  Same ownership,
+ * asynchrony, error and determinism rules as the attention calls.
+ */
+#define TRI_MUL_INCOMING 1u
+
+typedef struct {
+    int B, C, N;
+    tri_attn_tensor4 a, b;
+    tri_attn_tensor4 x;
+    unsigned flags; /* 0 (outgoing edges) or TRI_MUL_INCOMING */
+} tri_mul_fwd_args;
+
+/* Backward of the contraction: given dx (the upstream gradient of x), writes
+ *   outgoing:  da[i,k] = sum_j dx[i,j] b[j,k]     db[j,k] = sum_i dx[i,j] a[i,k]
+ *   incoming:  da[k,i] = sum_j dx[i,j] b[k,j]     db[k,j] = sum_i dx[i,j] a[k,i]
+ * (BF16 outputs from FP32 sums).  f.a, f.b and f.flags as in the forward;
+ * f.x is not used. */
+typedef struct {
+    tri_mul_fwd_args f;
+    tri_attn_tensor4 dx;
+    tri_attn_tensor4 da, db;
+} tri_mul_bwd_args;
+
+tri_attn_status tri_mul_fwd(const tri_mul_fwd_args *args, tri_attn_stream_t stream);
+tri_attn_status tri_mul_bwd(const tri_mul_bwd_args *args, tri_attn_stream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char *tri_attn_strerror(tri_attn_status status);
 

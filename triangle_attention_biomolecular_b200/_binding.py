@@ -57,6 +57,15 @@ class FwdArgs(ctypes.Structure):
                 ("o", Tensor5), ("resid", Tensor5), ("lse", ctypes.c_void_p)]
 
 
+class MulFwdArgs(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("C", ctypes.c_int), ("N", ctypes.c_int), ("a", Tensor4), ("b", Tensor4),
+                ("x", Tensor4), ("flags", ctypes.c_uint)]
+
+
+class MulBwdArgs(ctypes.Structure):
+    _fields_ = [("f", MulFwdArgs), ("dx", Tensor4), ("da", Tensor4), ("db", Tensor4)]
+
+
 class BwdArgs(ctypes.Structure):
     _fields_ = [("f", FwdArgs), ("dout", Tensor5), ("dq", Tensor5), ("dk", Tensor5), ("dv", Tensor5),
                 ("dbias", Tensor4), ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
@@ -84,6 +93,10 @@ def load() -> ctypes.CDLL:
             lib.tri_attn_bwd_marked.argtypes = [ctypes.POINTER(BwdArgs), ctypes.c_void_p,
                                                 ctypes.POINTER(ctypes.c_void_p)]
             lib.tri_attn_bwd_marked.restype = ctypes.c_int
+            lib.tri_mul_fwd.argtypes = [ctypes.POINTER(MulFwdArgs), ctypes.c_void_p]
+            lib.tri_mul_fwd.restype = ctypes.c_int
+            lib.tri_mul_bwd.argtypes = [ctypes.POINTER(MulBwdArgs), ctypes.c_void_p]
+            lib.tri_mul_bwd.restype = ctypes.c_int
             lib.tri_attn_bwd_static_scratch.argtypes = [ctypes.POINTER(BwdArgs), ctypes.c_void_p]
             lib.tri_attn_bwd_static_scratch.restype = ctypes.c_int
             lib.tri_attn_bwd_workspace_bytes.argtypes = [ctypes.c_int] * 4
@@ -256,6 +269,41 @@ def tri_attn_bwd_static_scratch(q, k, v, bias, mask, o, resid, lse, dout, dq, dk
     st = load().tri_attn_bwd_static_scratch(ctypes.byref(a), _stream_handle(stream))
     if st != TRI_ATTN_OK:
         raise TriAttnError(st, "tri_attn_bwd_static_scratch")
+
+
+TRI_MUL_INCOMING = 1
+
+
+def _mul_args(a, b, x, incoming: bool) -> MulFwdArgs:
+    B, C, N, N2 = a.shape
+    if N2 != N or tuple(b.shape) != (B, C, N, N):
+        raise TriAttnError(TRI_ATTN_ERR_SHAPE, "a and b must both be [B,C,N,N]")
+    m = MulFwdArgs()
+    m.B, m.C, m.N = B, C, N
+    m.a, m.b = t4(a, "a"), t4(b, "b")
+    if x is not None:
+        m.x = t4(x, "x")
+    m.flags = TRI_MUL_INCOMING if incoming else 0
+    return m
+
+
+def tri_mul_fwd(a, b, x, incoming: bool = False, stream=None) -> None:
+    """x[b,c,i,j] = sum_k a[b,c,i,k] b[b,c,j,k] (outgoing) or sum_k a[b,c,k,i] b[b,c,k,j]
+    (incoming); BF16 [B,C,N,N] CUDA tensors, x written."""
+    m = _mul_args(a, b, x, incoming)
+    st = load().tri_mul_fwd(ctypes.byref(m), _stream_handle(stream))
+    if st != TRI_ATTN_OK:
+        raise TriAttnError(st, "tri_mul_fwd")
+
+
+def tri_mul_bwd(a, b, dx, da, db, incoming: bool = False, stream=None) -> None:
+    """Gradients da, db of the contraction for the upstream gradient dx (all BF16 [B,C,N,N])."""
+    m = MulBwdArgs()
+    m.f = _mul_args(a, b, None, incoming)
+    m.dx, m.da, m.db = t4(dx, "dx"), t4(da, "da"), t4(db, "db")
+    st = load().tri_mul_bwd(ctypes.byref(m), _stream_handle(stream))
+    if st != TRI_ATTN_OK:
+        raise TriAttnError(st, "tri_mul_bwd")
 
 
 def tri_attn_device_error(clear: bool = True):

@@ -21,6 +21,7 @@
 #include "sm100.cuh"
 #include "fwd.cuh"
 #include "bwd.cuh"
+#include "tri_mul.cuh"
 
 namespace {
 
@@ -126,6 +127,12 @@ tri_attn_status ensure_device() {
     ok &= cudaFuncSetAttribute(tri::tri_attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                tri::FwdLayout<64>::SMEM) == cudaSuccess;
     ok &= tri::bwd_set_attributes();
+    ok &= cudaFuncSetAttribute(tri::tri_mul_gemm_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               tri::TriMulLayout::SMEM) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(tri::tri_mul_gemm_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               tri::TriMulLayout::SMEM) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(tri::tri_mul_gemm_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               tri::TriMulLayout::SMEM) == cudaSuccess;
     if (!ok || !encoder()) {
         cudaGetLastError();
         return TRI_ATTN_ERR_CUDA;
@@ -186,6 +193,45 @@ bool map_bias(CUtensorMap* m, const tri_attn_tensor4& t, int B, int N, int H) {
 }
 
 float eff_scale(float s, int d) { return s == 0.f ? 1.0f / std::sqrt(static_cast<float>(d)) : s; }
+
+// ---------------------------------------------------------------------------
+// triangle multiplicative contraction
+// ---------------------------------------------------------------------------
+// 4-D map over a BF16 [B, C, rows, cols] tensor: inner = cols (box 64, 128-byte
+// swizzle), then rows (box box_rows), c and b (box 1).
+bool map_bcrc(CUtensorMap* m, const tri_attn_tensor4& t, int B, int C, int N, uint32_t box_rows) {
+    const uint64_t size[3] = {static_cast<uint64_t>(N), static_cast<uint64_t>(C), static_cast<uint64_t>(B)};
+    const uint64_t st[3] = {static_cast<uint64_t>(t.stride[2]) * 2, static_cast<uint64_t>(t.stride[1]) * 2,
+                            static_cast<uint64_t>(t.stride[0]) * 2};
+    const uint32_t box[3] = {box_rows, 1, 1};
+    return encode_map(m, t.ptr, N, 64, size, st, box, 3, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+tri_attn_status check_mul_sizes(int B, int C, int N) {
+    if (B < 1 || C < 1 || N < 1 || static_cast<int64_t>(B) * C > 65535) return TRI_ATTN_ERR_SHAPE;
+    if (N > 16384) return TRI_ATTN_ERR_UNSUPPORTED;
+    return TRI_ATTN_OK;
+}
+
+// out[z][m][n] = sum_k A(m, k) B(n, k); an operand flagged MN is stored with m (n)
+// contiguous, otherwise with k contiguous
+template <bool A_MN, bool B_MN>
+tri_attn_status tri_mul_gemm(const tri_attn_tensor4& A, const tri_attn_tensor4& Bt, const tri_attn_tensor4& out, int Bn,
+                             int C, int N, cudaStream_t s) {
+    using L = tri::TriMulLayout;
+    CUtensorMap ma, mb;
+    if (!map_bcrc(&ma, A, Bn, C, N, A_MN ? 64 : L::BM) || !map_bcrc(&mb, Bt, Bn, C, N, B_MN ? 64 : L::BN))
+        return TRI_ATTN_ERR_STRIDE;
+    tri::TriMulGemmParams p{};
+    p.N = N;
+    p.C = C;
+    p.out = static_cast<__nv_bfloat16*>(out.ptr);
+    for (int x = 0; x < 4; ++x) p.os[x] = out.stride[x];
+    p.wait_limit_ns = g_wait_limit_ns.load();
+    const dim3 grid((N + L::BM - 1) / L::BM, (N + L::BN - 1) / L::BN, static_cast<unsigned>(Bn * C));
+    tri::tri_mul_gemm_kernel<A_MN, B_MN><<<grid, L::THREADS, L::SMEM, s>>>(ma, mb, p);
+    return cudaGetLastError() == cudaSuccess ? TRI_ATTN_OK : TRI_ATTN_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -376,6 +422,40 @@ tri_attn_status tri_attn_bwd_marked(const tri_attn_bwd_args* a, tri_attn_stream_
     if ((st = ensure_device())) return st;
     return tri::bwd_launch(a, ws, eff_scale(a->f.scale, d), g_wait_limit_ns.load(),
                            reinterpret_cast<cudaStream_t>(stream), markers);
+}
+
+tri_attn_status tri_mul_fwd(const tri_mul_fwd_args* a, tri_attn_stream_t stream) {
+    if (!a) return TRI_ATTN_ERR_NULL;
+    tri_attn_status st = check_mul_sizes(a->B, a->C, a->N);
+    if (st) return st;
+    if ((st = check_t4(a->a)) || (st = check_t4(a->b)) || (st = check_t4(a->x))) return st;
+    if (a->flags & ~TRI_MUL_INCOMING) return TRI_ATTN_ERR_UNSUPPORTED;
+    if ((st = ensure_device())) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (a->flags & TRI_MUL_INCOMING)  // x[i,j] = sum_k a[k,i] b[k,j]: both operands i/j-contiguous
+        return tri_mul_gemm<true, true>(a->a, a->b, a->x, a->B, a->C, a->N, s);
+    return tri_mul_gemm<false, false>(a->a, a->b, a->x, a->B, a->C, a->N, s);  // sum_k a[i,k] b[j,k]
+}
+
+tri_attn_status tri_mul_bwd(const tri_mul_bwd_args* a, tri_attn_stream_t stream) {
+    if (!a) return TRI_ATTN_ERR_NULL;
+    const tri_mul_fwd_args& f = a->f;
+    tri_attn_status st = check_mul_sizes(f.B, f.C, f.N);
+    if (st) return st;
+    if ((st = check_t4(f.a)) || (st = check_t4(f.b)) || (st = check_t4(a->dx)) || (st = check_t4(a->da)) ||
+        (st = check_t4(a->db)))
+        return st;
+    if (f.flags & ~TRI_MUL_INCOMING) return TRI_ATTN_ERR_UNSUPPORTED;
+    if ((st = ensure_device())) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (f.flags & TRI_MUL_INCOMING) {
+        // da[k,i] = sum_j b[k,j] dx[i,j];  db[k,j] = sum_i a[k,i] dx[i,j]
+        if ((st = tri_mul_gemm<false, false>(f.b, a->dx, a->da, f.B, f.C, f.N, s))) return st;
+        return tri_mul_gemm<false, true>(f.a, a->dx, a->db, f.B, f.C, f.N, s);
+    }
+    // da[i,k] = sum_j dx[i,j] b[j,k];  db[j,k] = sum_i dx[i,j] a[i,k]
+    if ((st = tri_mul_gemm<false, true>(a->dx, f.b, a->da, f.B, f.C, f.N, s))) return st;
+    return tri_mul_gemm<true, true>(a->dx, f.a, a->db, f.B, f.C, f.N, s);
 }
 
 tri_attn_status tri_attn_device_error(int clear, uint32_t* word) {

@@ -71,14 +71,6 @@ struct FwdLayout {
     static_assert(QKV_TILE % 1024 == 0 && STAGE % 1024 == 0, "1 KB tile alignment");
 };
 
-// Bounded wait used only while draining on the way out: ignores the abort flag.
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > limit_ns) break;
-    }
-}
-
 __device__ __forceinline__ void reg_fence16(uint32_t (&r)[16]) {
     asm volatile(""
                  : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),

@@ -50,7 +50,7 @@ __device__ unsigned long long* g_trace;
 // site codes: high byte = kernel, low bits = wait site
 enum : uint32_t {
     ERR_TIMEOUT_BIT = 0x80000000u,
-    KERNEL_FWD = 1u << 16, KERNEL_BWD_MAIN = 2u << 16, KERNEL_BWD_DBIAS = 3u << 16,
+    KERNEL_FWD = 1u << 16, KERNEL_BWD_MAIN = 2u << 16, KERNEL_BWD_DBIAS = 3u << 16, KERNEL_TRIMUL = 4u << 16,
     KERNEL_SELFTEST = 15u << 16,
 };
 
@@ -126,6 +126,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
             *w.abort_flag = 1;
             return false;
         }
+    }
+}
+
+// Bounded wait used only while draining on the way out: ignores the abort flag.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > limit_ns) break;
     }
 }
 
