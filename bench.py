@@ -111,11 +111,11 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_crop768.md")
 
 
 def kernel_source_digest() -> str:
-    """sha256 over the kernel sources and the ABI header, in name order."""
-    import glob
+    """sha256 over the sources the attention kernels are compiled from (their device
+    code and shared helpers), in name order."""
     import hashlib
-    files = sorted(glob.glob(os.path.join(ROOT, "triangle_attention_biomolecular_b200", "csrc", "*")))
-    files.append(os.path.join(ROOT, "include", "tri_attn.h"))
+    csrc = os.path.join(ROOT, "triangle_attention_biomolecular_b200", "csrc")
+    files = [os.path.join(csrc, n) for n in ("bwd.cuh", "fwd.cuh", "sm100.cuh")]
     h = hashlib.sha256()
     for fn in files:
         h.update(os.path.basename(fn).encode())
