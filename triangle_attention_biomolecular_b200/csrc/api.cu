@@ -225,10 +225,13 @@ tri_attn_status tri_mul_gemm(const tri_attn_tensor4& A, const tri_attn_tensor4& 
     tri::TriMulGemmParams p{};
     p.N = N;
     p.C = C;
+    p.Z = Bn * C;
     p.out = static_cast<__nv_bfloat16*>(out.ptr);
     for (int x = 0; x < 4; ++x) p.os[x] = out.stride[x];
     p.wait_limit_ns = g_wait_limit_ns.load();
-    const dim3 grid((N + L::BM - 1) / L::BM, (N + L::BN - 1) / L::BN, static_cast<unsigned>(Bn * C));
+    // persistent grid: one CTA per SM (148 on B200) walking the output tiles
+    const int64_t tiles = static_cast<int64_t>((N + L::BM - 1) / L::BM) * ((N + L::BN - 1) / L::BN) * Bn * C;
+    const dim3 grid(static_cast<unsigned>(std::min<int64_t>(tiles, 148)));
     tri::tri_mul_gemm_kernel<A_MN, B_MN><<<grid, L::THREADS, L::SMEM, s>>>(ma, mb, p);
     return cudaGetLastError() == cudaSuccess ? TRI_ATTN_OK : TRI_ATTN_ERR_CUDA;
 }
