@@ -296,6 +296,73 @@ def run_ours(args, rank, world, local_rank):
 
 
 # ---------------------------------------------------------------------------
+# all configurations (--sweep): one JSON line per workload
+# ---------------------------------------------------------------------------
+def run_sweep(args):
+    """Forward-only and forward+backward times of every workload family: the three
+    crops and the batched ragged sweep (B=2, N in 128..1024, d in 32/64, lengths
+    L_b ~ U{N/2..N}).  TFLOP/s by the formula and effective (4*H*d*sum_b N^2*L_b per
+    forward pass, 14*... per step), % of the BF16 peak, and for N <= 512 the
+    algorithmic bytes per second against the HBM peak."""
+    import torch
+    from triangle_attention_biomolecular_b200 import _binding as Bd
+    from triangle_attention_biomolecular_b200 import synthetic as S
+    dev = torch.device("cuda", 0)
+    pk, src = peaks()
+    peak, hbm = float(pk["bf16_tflops"]), float(pk["hbm_gbs"])
+    wls = [S.CROP384, S.CROP640, S.CROP768] + [S.sweep(N, d) for d in S.SWEEP_DS for N in S.SWEEP_NS]
+    for wl in wls:
+        x = S.make_inputs(wl, S.seed_for(9, wl.N + wl.d))
+        q, k, v, do, bias = (x[n].to(dev) for n in ("q", "k", "v", "dout", "bias"))
+        mask = x["mask"].to(dev) if x["mask"] is not None else None
+        Bn, N, H, d = wl.B, wl.N, wl.H, wl.d
+        o, r = torch.empty_like(q), torch.empty_like(q)
+        lse = torch.empty((Bn, H, N, N), dtype=torch.float32, device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+        Np = (N + 7) // 8 * 8
+        db = torch.empty((Bn, H, N, Np), dtype=torch.bfloat16, device=dev)[..., :N]
+        ws = torch.empty(Bd.tri_attn_bwd_workspace_bytes(Bn, N, H, d), dtype=torch.uint8, device=dev)
+        fwd = lambda: Bd.tri_attn_fwd(q, k, v, bias, mask, o, r, lse)
+        bwd = lambda: Bd.tri_attn_bwd(q, k, v, bias, mask, o, r, lse, do, dq, dk, dv, db, ws)
+
+        def timed(fn, n):
+            for _ in range(3):
+                fn()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(n):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / n
+        n_iter = max(5, min(200, int(2e12 / (14.0 * Bn * H * N ** 3 * d))))
+        t_f = timed(fwd, n_iter)
+        t_fb = timed(lambda: (fwd(), bwd()), n_iter)
+        st, word = Bd.tri_attn_device_error(True)
+        if st != 0:
+            raise RuntimeError(f"device error word {word:#x} in {wl.name}")
+        L = [int(v_) for v_ in x["lengths"]]
+        cube = H * N ** 3 * d * Bn
+        eff = H * d * sum(N * N * l_ for l_ in L)
+        pair = Bn * N * N * H * d * 2
+        fwd_bytes = 5 * pair + Bn * H * N * N * (2 + 4) + Bn * N * N * 4
+        line = {"metric": "tri-attn TFLOP/s per workload", "workload": wl.name, "B": Bn, "N": N, "H": H, "d": d,
+                "mask": wl.mask, "orientation": wl.orientation, "iters": n_iter,
+                "fwd_ms": round(t_f, 4), "fwd_tflops": round(4.0 * cube / (t_f * 1e-3) / 1e12, 2),
+                "fwd_tflops_effective": round(4.0 * eff / (t_f * 1e-3) / 1e12, 2),
+                "fwd_bwd_ms": round(t_fb, 4), "fwd_bwd_tflops": round(14.0 * cube / (t_fb * 1e-3) / 1e12, 2),
+                "fwd_bwd_tflops_effective": round(14.0 * eff / (t_fb * 1e-3) / 1e12, 2),
+                "pct_of_bf16_peak": round(100.0 * 14.0 * cube / (t_fb * 1e-3) / 1e12 / peak, 2),
+                "peak_source": f"{src} bf16_tflops {peak}"}
+        if N <= 512:
+            gbs = fwd_bytes / (t_f * 1e-3) / 1e9
+            line["fwd_algorithmic_gbs"] = round(gbs, 1)
+            line["fwd_pct_of_hbm"] = round(100.0 * gbs / hbm, 2)
+        print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
 # second operation: the triangle multiplicative contraction (--op tri_mul)
 # ---------------------------------------------------------------------------
 TRI_MUL_METRIC = "tri-mul contraction fwd+bwd TFLOP/s at N=768, C=128 pair channels, BF16"
@@ -458,6 +525,8 @@ def main():
                     help="crop768 is the headline; the smaller crops serve profiler captures")
     ap.add_argument("--op", choices=("attention", "tri_mul"), default="attention",
                     help="attention (the headline) or the triangle multiplicative contraction")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every workload (crops and the ragged N/d sweep), one JSON line each")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle on host cores")
     args = ap.parse_args()
@@ -467,6 +536,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.sweep:
+        run_sweep(args)
         return
 
     import datetime
