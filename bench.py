@@ -424,6 +424,56 @@ def run_tri_mul(args, rank, world, local_rank):
     return {"ms": ms, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "clocks": clocks, "shape": (Bn, C, N)}
 
 
+GATE_METRIC = "gated output projection GB/s at N=768 (589,824 pair positions, 128 channels), BF16"
+
+
+def run_gate(args):
+    """One step = y = (sigmoid(z Wg) * o) Wo over every pair position of the crop768
+    pair tensor; HBM-bound: z, o read and y written, 3 x R x 128 x 2 bytes."""
+    import torch
+    from triangle_attention_biomolecular_b200 import _binding as Bd
+    dev = torch.device("cuda", 0)
+    R = 768 * 768
+    g = torch.Generator().manual_seed(5)
+    z, o = (torch.randn((R, 128), generator=g).to(torch.bfloat16).to(dev) for _ in range(2))
+    wg, wo = ((torch.randn((128, 128), generator=g) / 128 ** 0.5).to(torch.bfloat16).to(dev) for _ in range(2))
+    y = torch.empty_like(z)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        Bd.tri_gate_fwd(z, o, wg, wo, y, stream)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(0)
+    sampler.start()
+    time.sleep(0.3)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(args.steps):
+        Bd.tri_gate_fwd(z, o, wg, wo, y, stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    st, word = Bd.tri_attn_device_error(True)
+    if st != 0:
+        raise RuntimeError(f"device error word {word:#x}")
+    ms = t0.elapsed_time(t1) / args.steps
+    pk, src = peaks()
+    hbm = float(pk["hbm_gbs"])
+    nbytes = 3 * R * 128 * 2 + 2 * 128 * 128 * 2
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    line = {"metric": GATE_METRIC, "value": round(gbs, 1), "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "gated output projection y = (sigmoid(z Wg) * o) Wo, R = 768^2 pair positions, "
+                                   "cz = H*d = 128", "bytes_per_step": nbytes,
+                       "l2": "inputs (302 MB) larger than the 126 MB L2; no flush"},
+            "tflops": round(2 * 2 * R * 128 * 128 / (ms * 1e-3) / 1e12, 2),
+            "roofline": {"kernel": "tri_gate_fwd", "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm,
+                         "unit": "GB/s", "frac": round(gbs / hbm, 4), "traffic": None, "peak_source": f"{src} hbm_gbs"},
+            "gpu_launches": args.steps, "clocks": clocks, "e2e": None}
+    print(json.dumps(line), flush=True)
+
+
 def tri_mul_cpu_baseline(target_s: float = 10.0):
     """The FP64 oracle on the host cores over a bounded number of channels."""
     import numpy as np
@@ -523,8 +573,9 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", choices=("crop768", "crop640", "crop384"), default="crop768",
                     help="crop768 is the headline; the smaller crops serve profiler captures")
-    ap.add_argument("--op", choices=("attention", "tri_mul"), default="attention",
-                    help="attention (the headline) or the triangle multiplicative contraction")
+    ap.add_argument("--op", choices=("attention", "tri_mul", "gate"), default="attention",
+                    help="attention (the headline), the triangle multiplicative contraction, or the gated "
+                         "output projection")
     ap.add_argument("--sweep", action="store_true",
                     help="time every workload (crops and the ragged N/d sweep), one JSON line each")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
@@ -539,6 +590,9 @@ def main():
         return
     if args.sweep:
         run_sweep(args)
+        return
+    if args.op == "gate":
+        run_gate(args)
         return
 
     import datetime

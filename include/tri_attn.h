@@ -245,6 +245,31 @@ typedef struct {
 tri_attn_status tri_mul_fwd(const tri_mul_fwd_args *args, tri_attn_stream_t stream);
 tri_attn_status tri_mul_bwd(const tri_mul_bwd_args *args, tri_attn_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Gated output projection around the attention (no counterpart on the pages,
+ * which describe the attention itself; the AlphaFold-style steps on either
+ * side of it, fused):  for every pair position r,
+ *     g = sigmoid(z[r,:] Wg),   y[r,:] = (g * o[r,:]) Wo
+ *   z  : BF16 [R, 128], the attention block's pair input (cz = 128)
+ *   o  : BF16 [R, 128], the attention output with heads concatenated (H*d = 128)
+ *   wg : BF16 [128, 128] row-major, wg[cz][co];  wo: BF16 [128, 128], wo[co][cz]
+ *   y  : BF16 [R, 128] output (RNE of the FP32 result)
+ * Row strides in elements (multiples of 8); pointers 16-byte aligned; R >= 1.
+ * No biases.  Same ownership, asynchrony and error rules as the other calls.
+ */
+typedef struct {
+    int R;
+    const void *z;
+    int64_t z_stride;
+    const void *o;
+    int64_t o_stride;
+    const void *wg, *wo;
+    void *y;
+    int64_t y_stride;
+} tri_gate_fwd_args;
+
+tri_attn_status tri_gate_fwd(const tri_gate_fwd_args *args, tri_attn_stream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char *tri_attn_strerror(tri_attn_status status);
 

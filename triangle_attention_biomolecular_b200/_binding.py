@@ -62,6 +62,12 @@ class MulFwdArgs(ctypes.Structure):
                 ("x", Tensor4), ("flags", ctypes.c_uint)]
 
 
+class GateFwdArgs(ctypes.Structure):
+    _fields_ = [("R", ctypes.c_int), ("z", ctypes.c_void_p), ("z_stride", ctypes.c_int64), ("o", ctypes.c_void_p),
+                ("o_stride", ctypes.c_int64), ("wg", ctypes.c_void_p), ("wo", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("y_stride", ctypes.c_int64)]
+
+
 class MulBwdArgs(ctypes.Structure):
     _fields_ = [("f", MulFwdArgs), ("dx", Tensor4), ("da", Tensor4), ("db", Tensor4)]
 
@@ -93,6 +99,8 @@ def load() -> ctypes.CDLL:
             lib.tri_attn_bwd_marked.argtypes = [ctypes.POINTER(BwdArgs), ctypes.c_void_p,
                                                 ctypes.POINTER(ctypes.c_void_p)]
             lib.tri_attn_bwd_marked.restype = ctypes.c_int
+            lib.tri_gate_fwd.argtypes = [ctypes.POINTER(GateFwdArgs), ctypes.c_void_p]
+            lib.tri_gate_fwd.restype = ctypes.c_int
             lib.tri_mul_fwd.argtypes = [ctypes.POINTER(MulFwdArgs), ctypes.c_void_p]
             lib.tri_mul_fwd.restype = ctypes.c_int
             lib.tri_mul_bwd.argtypes = [ctypes.POINTER(MulBwdArgs), ctypes.c_void_p]
@@ -304,6 +312,28 @@ def tri_mul_bwd(a, b, dx, da, db, incoming: bool = False, stream=None) -> None:
     st = load().tri_mul_bwd(ctypes.byref(m), _stream_handle(stream))
     if st != TRI_ATTN_OK:
         raise TriAttnError(st, "tri_mul_bwd")
+
+
+def tri_gate_fwd(z, o, wg, wo, y, stream=None) -> None:
+    """y = (sigmoid(z wg) * o) wo row by row; z, o, y BF16 [R, 128] (rows may be padded),
+    wg, wo BF16 [128, 128] contiguous."""
+    import torch
+    for t, n in ((z, "z"), (o, "o"), (y, "y"), (wg, "wg"), (wo, "wo")):
+        if t.dtype != torch.bfloat16 or t.dim() != 2 or t.shape[1] != 128 or t.stride(1) != 1:
+            raise TriAttnError(TRI_ATTN_ERR_DTYPE, f"{n} must be a BF16 [*, 128] tensor with unit column stride")
+    if wg.shape[0] != 128 or wo.shape[0] != 128 or not wg.is_contiguous() or not wo.is_contiguous():
+        raise TriAttnError(TRI_ATTN_ERR_SHAPE, "wg and wo must be contiguous [128, 128]")
+    if o.shape[0] != z.shape[0] or y.shape[0] != z.shape[0]:
+        raise TriAttnError(TRI_ATTN_ERR_SHAPE, "z, o and y must have the same number of rows")
+    a = GateFwdArgs()
+    a.R = z.shape[0]
+    a.z, a.z_stride = z.data_ptr(), z.stride(0)
+    a.o, a.o_stride = o.data_ptr(), o.stride(0)
+    a.wg, a.wo = wg.data_ptr(), wo.data_ptr()
+    a.y, a.y_stride = y.data_ptr(), y.stride(0)
+    st = load().tri_gate_fwd(ctypes.byref(a), _stream_handle(stream))
+    if st != TRI_ATTN_OK:
+        raise TriAttnError(st, "tri_gate_fwd")
 
 
 def tri_attn_device_error(clear: bool = True):

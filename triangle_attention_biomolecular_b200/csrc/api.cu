@@ -22,6 +22,7 @@
 #include "fwd.cuh"
 #include "bwd.cuh"
 #include "tri_mul.cuh"
+#include "tri_gate.cuh"
 
 namespace {
 
@@ -133,6 +134,8 @@ tri_attn_status ensure_device() {
                                tri::TriMulLayout::SMEM) == cudaSuccess;
     ok &= cudaFuncSetAttribute(tri::tri_mul_gemm_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                tri::TriMulLayout::SMEM) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(tri::tri_gate_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               tri::TriGateLayout::SMEM) == cudaSuccess;
     if (!ok || !encoder()) {
         cudaGetLastError();
         return TRI_ATTN_ERR_CUDA;
@@ -205,6 +208,15 @@ bool map_bcrc(CUtensorMap* m, const tri_attn_tensor4& t, int B, int C, int N, ui
                             static_cast<uint64_t>(t.stride[0]) * 2};
     const uint32_t box[3] = {box_rows, 1, 1};
     return encode_map(m, t.ptr, N, 64, size, st, box, 3, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// 2-D map over a BF16 [rows, 128] matrix with the given row stride: box 64 x box_rows,
+// 128-byte swizzle
+bool map_rows128(CUtensorMap* m, const void* ptr, int64_t rows, int64_t row_stride, uint32_t box_rows) {
+    const uint64_t size[1] = {static_cast<uint64_t>(rows)};
+    const uint64_t st[1] = {static_cast<uint64_t>(row_stride) * 2};
+    const uint32_t box[1] = {box_rows};
+    return encode_map(m, const_cast<void*>(ptr), 128, 64, size, st, box, 1, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 tri_attn_status check_mul_sizes(int B, int C, int N) {
@@ -459,6 +471,33 @@ tri_attn_status tri_mul_bwd(const tri_mul_bwd_args* a, tri_attn_stream_t stream)
     // da[i,k] = sum_j dx[i,j] b[j,k];  db[j,k] = sum_i dx[i,j] a[i,k]
     if ((st = tri_mul_gemm<false, true>(a->dx, f.b, a->da, f.B, f.C, f.N, s))) return st;
     return tri_mul_gemm<true, true>(a->dx, f.a, a->db, f.B, f.C, f.N, s);
+}
+
+tri_attn_status tri_gate_fwd(const tri_gate_fwd_args* a, tri_attn_stream_t stream) {
+    if (!a) return TRI_ATTN_ERR_NULL;
+    if (!a->z || !a->o || !a->wg || !a->wo || !a->y) return TRI_ATTN_ERR_NULL;
+    if (a->R < 1) return TRI_ATTN_ERR_SHAPE;
+    for (int64_t st : {a->z_stride, a->o_stride, a->y_stride})
+        if (st < 128 || st % 8) return TRI_ATTN_ERR_STRIDE;
+    for (const void* ptr : {a->z, a->o, a->wg, a->wo, static_cast<const void*>(a->y)})
+        if (!aligned16(ptr)) return TRI_ATTN_ERR_ALIGN;
+    tri_attn_status st = ensure_device();
+    if (st) return st;
+    using L = tri::TriGateLayout;
+    CUtensorMap mz, mo, mwg, mwo;
+    if (!map_rows128(&mz, a->z, a->R, a->z_stride, L::BM) || !map_rows128(&mo, a->o, a->R, a->o_stride, L::BM) ||
+        !map_rows128(&mwg, a->wg, 128, 128, 128) || !map_rows128(&mwo, a->wo, 128, 128, 128))
+        return TRI_ATTN_ERR_STRIDE;
+    tri::TriGateParams p{};
+    p.R = a->R;
+    p.y = static_cast<__nv_bfloat16*>(a->y);
+    p.ys = a->y_stride;
+    p.wait_limit_ns = g_wait_limit_ns.load();
+    const int64_t tiles = (static_cast<int64_t>(a->R) + L::BM - 1) / L::BM;
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, 148));  // persistent, one CTA per SM
+    tri::tri_gate_fwd_kernel<<<grid, L::THREADS, L::SMEM, reinterpret_cast<cudaStream_t>(stream)>>>(mz, mo, mwg, mwo,
+                                                                                                   p);
+    return cudaGetLastError() == cudaSuccess ? TRI_ATTN_OK : TRI_ATTN_ERR_CUDA;
 }
 
 tri_attn_status tri_attn_device_error(int clear, uint32_t* word) {
