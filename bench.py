@@ -424,53 +424,69 @@ def run_tri_mul(args, rank, world, local_rank):
     return {"ms": ms, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "clocks": clocks, "shape": (Bn, C, N)}
 
 
-GATE_METRIC = "gated output projection GB/s at N=768 (589,824 pair positions, 128 channels), BF16"
+GATE_METRIC = ("gated output projection fwd+bwd GB/s at N=768 (589,824 pair positions, 128 channels), BF16")
 
 
 def run_gate(args):
-    """One step = y = (sigmoid(z Wg) * o) Wo over every pair position of the crop768
-    pair tensor; HBM-bound: z, o read and y written, 3 x R x 128 x 2 bytes."""
+    """One step = forward y = (sigmoid(z Wg) * o) Wo and backward (dz, do, dWg, dWo for an
+    upstream dy) over every pair position of the crop768 pair tensor.  HBM-bound: the
+    forward reads z, o and writes y, the backward reads z, o, dy and writes dz, do:
+    8 x R x 128 x 2 bytes (plus the weights)."""
     import torch
     from triangle_attention_biomolecular_b200 import _binding as Bd
     dev = torch.device("cuda", 0)
     R = 768 * 768
     g = torch.Generator().manual_seed(5)
-    z, o = (torch.randn((R, 128), generator=g).to(torch.bfloat16).to(dev) for _ in range(2))
+    z, o, dy = (torch.randn((R, 128), generator=g).to(torch.bfloat16).to(dev) for _ in range(3))
     wg, wo = ((torch.randn((128, 128), generator=g) / 128 ** 0.5).to(torch.bfloat16).to(dev) for _ in range(2))
-    y = torch.empty_like(z)
+    y, dz, d_o = (torch.empty_like(z) for _ in range(3))
+    dwg, dwo = (torch.empty((128, 128), device=dev) for _ in range(2))
+    ws = torch.empty(Bd.tri_gate_bwd_workspace_bytes(R), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
+    fwd = lambda: Bd.tri_gate_fwd(z, o, wg, wo, y, stream)
+    bwd = lambda: Bd.tri_gate_bwd(z, o, wg, wo, dy, dz, d_o, dwg, dwo, ws, stream)
     for _ in range(args.warmup):
-        Bd.tri_gate_fwd(z, o, wg, wo, y, stream)
+        fwd()
+        bwd()
     torch.cuda.synchronize()
     sampler = ClockSampler(0)
     sampler.start()
     time.sleep(0.3)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps + 1)]
     torch.cuda.synchronize()
-    t0.record(stream)
-    for _ in range(args.steps):
-        Bd.tri_gate_fwd(z, o, wg, wo, y, stream)
-    t1.record(stream)
+    ev[0].record(stream)
+    for i in range(args.steps):
+        fwd()
+        ev[2 * i + 1].record(stream)
+        bwd()
+        ev[2 * i + 2].record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
     st, word = Bd.tri_attn_device_error(True)
     if st != 0:
         raise RuntimeError(f"device error word {word:#x}")
-    ms = t0.elapsed_time(t1) / args.steps
+    f_ms = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(args.steps)) / args.steps
+    b_ms = sum(ev[2 * i + 1].elapsed_time(ev[2 * i + 2]) for i in range(args.steps)) / args.steps
+    ms = f_ms + b_ms
     pk, src = peaks()
     hbm = float(pk["hbm_gbs"])
-    nbytes = 3 * R * 128 * 2 + 2 * 128 * 128 * 2
-    gbs = nbytes / (ms * 1e-3) / 1e9
+    row = R * 128 * 2
+    f_bytes, b_bytes = 3 * row + 2 * 128 * 128 * 2, 5 * row + 2 * 128 * 128 * 2
+    gbs = (f_bytes + b_bytes) / (ms * 1e-3) / 1e9
+    b_gbs = b_bytes / (b_ms * 1e-3) / 1e9
     line = {"metric": GATE_METRIC, "value": round(gbs, 1), "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "gated output projection y = (sigmoid(z Wg) * o) Wo, R = 768^2 pair positions, "
-                                   "cz = H*d = 128", "bytes_per_step": nbytes,
-                       "l2": "inputs (302 MB) larger than the 126 MB L2; no flush"},
-            "tflops": round(2 * 2 * R * 128 * 128 / (ms * 1e-3) / 1e12, 2),
-            "roofline": {"kernel": "tri_gate_fwd", "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm,
-                         "unit": "GB/s", "frac": round(gbs / hbm, 4), "traffic": None, "peak_source": f"{src} hbm_gbs"},
-            "gpu_launches": args.steps, "clocks": clocks, "e2e": None}
+            "config": {"workload": "gated output projection y = (sigmoid(z Wg) * o) Wo and its backward, "
+                                   "R = 768^2 pair positions, cz = H*d = 128",
+                       "bytes_per_step": f_bytes + b_bytes, "fwd_ms": round(f_ms, 4), "bwd_ms": round(b_ms, 4),
+                       "fwd_gbs": round(f_bytes / (f_ms * 1e-3) / 1e9, 1), "bwd_gbs": round(b_gbs, 1),
+                       "l2": "inputs (151 MB per tensor) larger than the 126 MB L2; no flush"},
+            "tflops": round(7 * 2 * R * 128 * 128 / (ms * 1e-3) / 1e12, 2),  # 2 + 5 contractions
+            "roofline": {"kernel": "tri_gate_bwd", "bound": "hbm", "achieved": round(b_gbs, 1), "peak": hbm,
+                         "unit": "GB/s", "frac": round(b_gbs / hbm, 4), "traffic": None,
+                         "peak_source": f"{src} hbm_gbs"},
+            "gpu_launches": 3 * args.steps, "clocks": clocks, "e2e": None}
     print(json.dumps(line), flush=True)
 
 

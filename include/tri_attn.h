@@ -270,6 +270,40 @@ typedef struct {
 
 tri_attn_status tri_gate_fwd(const tri_gate_fwd_args *args, tri_attn_stream_t stream);
 
+/* Backward of tri_gate_fwd for the upstream gradient dy (a = g * o):
+ *     dA = dy Wo^T,  do = dA * g,  dl = dA * o * g * (1 - g),
+ *     dz = dl Wg^T,  dWo = sum_r a^T dy,  dWg = sum_r z^T dl
+ *   f      : the forward's arguments (f.y is not used)
+ *   dy     : BF16 [R, 128] upstream gradient
+ *   dz, d_o: BF16 [R, 128] outputs (overwritten)
+ *   dwg    : FP32 [128, 128] row-major, dwg[cz][co] (overwritten)
+ *   dwo    : FP32 [128, 128] row-major, dwo[co][cz] (overwritten)
+ *   workspace, workspace_bytes : caller-owned device scratch of at least
+ *            tri_gate_bwd_workspace_bytes(R) bytes, 16-byte aligned (partial
+ *            weight-gradient sums of each CTA).
+ * The weight gradients are summed in a fixed order, so repeated calls with the
+ * same inputs give bitwise-identical results.  Strides, alignment and errors
+ * as for tri_gate_fwd; TRI_ATTN_ERR_WORKSPACE if the workspace is NULL or too
+ * small. */
+typedef struct {
+    tri_gate_fwd_args f;
+    const void *dy;
+    int64_t dy_stride;
+    void *dz;
+    int64_t dz_stride;
+    void *d_o;
+    int64_t do_stride;
+    float *dwg, *dwo;
+    void *workspace;
+    size_t workspace_bytes;
+} tri_gate_bwd_args;
+
+/* Bytes of workspace tri_gate_bwd needs for R pair positions (pure function;
+ * 0 for R < 1). */
+size_t tri_gate_bwd_workspace_bytes(int R);
+
+tri_attn_status tri_gate_bwd(const tri_gate_bwd_args *args, tri_attn_stream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char *tri_attn_strerror(tri_attn_status status);
 

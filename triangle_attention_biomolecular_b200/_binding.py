@@ -68,6 +68,13 @@ class GateFwdArgs(ctypes.Structure):
                 ("y_stride", ctypes.c_int64)]
 
 
+class GateBwdArgs(ctypes.Structure):
+    _fields_ = [("f", GateFwdArgs), ("dy", ctypes.c_void_p), ("dy_stride", ctypes.c_int64), ("dz", ctypes.c_void_p),
+                ("dz_stride", ctypes.c_int64), ("d_o", ctypes.c_void_p), ("do_stride", ctypes.c_int64),
+                ("dwg", ctypes.c_void_p), ("dwo", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+
 class MulBwdArgs(ctypes.Structure):
     _fields_ = [("f", MulFwdArgs), ("dx", Tensor4), ("da", Tensor4), ("db", Tensor4)]
 
@@ -101,6 +108,10 @@ def load() -> ctypes.CDLL:
             lib.tri_attn_bwd_marked.restype = ctypes.c_int
             lib.tri_gate_fwd.argtypes = [ctypes.POINTER(GateFwdArgs), ctypes.c_void_p]
             lib.tri_gate_fwd.restype = ctypes.c_int
+            lib.tri_gate_bwd.argtypes = [ctypes.POINTER(GateBwdArgs), ctypes.c_void_p]
+            lib.tri_gate_bwd.restype = ctypes.c_int
+            lib.tri_gate_bwd_workspace_bytes.argtypes = [ctypes.c_int]
+            lib.tri_gate_bwd_workspace_bytes.restype = ctypes.c_size_t
             lib.tri_mul_fwd.argtypes = [ctypes.POINTER(MulFwdArgs), ctypes.c_void_p]
             lib.tri_mul_fwd.restype = ctypes.c_int
             lib.tri_mul_bwd.argtypes = [ctypes.POINTER(MulBwdArgs), ctypes.c_void_p]
@@ -334,6 +345,47 @@ def tri_gate_fwd(z, o, wg, wo, y, stream=None) -> None:
     st = load().tri_gate_fwd(ctypes.byref(a), _stream_handle(stream))
     if st != TRI_ATTN_OK:
         raise TriAttnError(st, "tri_gate_fwd")
+
+
+def _check_rows128(ts, names):
+    import torch
+    for t, n in zip(ts, names):
+        if t.dtype != torch.bfloat16 or t.dim() != 2 or t.shape[1] != 128 or t.stride(1) != 1:
+            raise TriAttnError(TRI_ATTN_ERR_DTYPE, f"{n} must be a BF16 [*, 128] tensor with unit column stride")
+
+
+def tri_gate_bwd_workspace_bytes(R: int) -> int:
+    return int(load().tri_gate_bwd_workspace_bytes(R))
+
+
+def tri_gate_bwd(z, o, wg, wo, dy, dz, d_o, dwg, dwo, workspace, stream=None) -> None:
+    """Gradients of y = (sigmoid(z wg) * o) wo for the upstream dy: dz, d_o BF16 [R, 128]
+    (rows may be padded), dwg, dwo FP32 [128, 128] contiguous, workspace a uint8 CUDA
+    tensor of at least tri_gate_bwd_workspace_bytes(R) bytes."""
+    import torch
+    _check_rows128((z, o, dy, dz, d_o, wg, wo), ("z", "o", "dy", "dz", "d_o", "wg", "wo"))
+    if wg.shape[0] != 128 or wo.shape[0] != 128 or not wg.is_contiguous() or not wo.is_contiguous():
+        raise TriAttnError(TRI_ATTN_ERR_SHAPE, "wg and wo must be contiguous [128, 128]")
+    for t, n in ((dwg, "dwg"), (dwo, "dwo")):
+        if t.dtype != torch.float32 or tuple(t.shape) != (128, 128) or not t.is_contiguous():
+            raise TriAttnError(TRI_ATTN_ERR_DTYPE, f"{n} must be a contiguous FP32 [128, 128] tensor")
+    R = z.shape[0]
+    if any(t.shape[0] != R for t in (o, dy, dz, d_o)):
+        raise TriAttnError(TRI_ATTN_ERR_SHAPE, "z, o, dy, dz and d_o must have the same number of rows")
+    a = GateBwdArgs()
+    a.f.R = R
+    a.f.z, a.f.z_stride = z.data_ptr(), z.stride(0)
+    a.f.o, a.f.o_stride = o.data_ptr(), o.stride(0)
+    a.f.wg, a.f.wo = wg.data_ptr(), wo.data_ptr()
+    a.f.y, a.f.y_stride = None, 128
+    a.dy, a.dy_stride = dy.data_ptr(), dy.stride(0)
+    a.dz, a.dz_stride = dz.data_ptr(), dz.stride(0)
+    a.d_o, a.do_stride = d_o.data_ptr(), d_o.stride(0)
+    a.dwg, a.dwo = dwg.data_ptr(), dwo.data_ptr()
+    a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    st = load().tri_gate_bwd(ctypes.byref(a), _stream_handle(stream))
+    if st != TRI_ATTN_OK:
+        raise TriAttnError(st, "tri_gate_bwd")
 
 
 def tri_attn_device_error(clear: bool = True):

@@ -136,6 +136,8 @@ tri_attn_status ensure_device() {
                                tri::TriMulLayout::SMEM) == cudaSuccess;
     ok &= cudaFuncSetAttribute(tri::tri_gate_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                tri::TriGateLayout::SMEM) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(tri::tri_gate_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               tri::TriGateBwdLayout::SMEM) == cudaSuccess;
     if (!ok || !encoder()) {
         cudaGetLastError();
         return TRI_ATTN_ERR_CUDA;
@@ -497,6 +499,57 @@ tri_attn_status tri_gate_fwd(const tri_gate_fwd_args* a, tri_attn_stream_t strea
     const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, 148));  // persistent, one CTA per SM
     tri::tri_gate_fwd_kernel<<<grid, L::THREADS, L::SMEM, reinterpret_cast<cudaStream_t>(stream)>>>(mz, mo, mwg, mwo,
                                                                                                    p);
+    return cudaGetLastError() == cudaSuccess ? TRI_ATTN_OK : TRI_ATTN_ERR_CUDA;
+}
+
+namespace {
+constexpr int kGateMaxCtas = 148;  // persistent grid: one CTA per SM
+int64_t gate_ctas(int R) {
+    return std::min<int64_t>((static_cast<int64_t>(R) + tri::TriGateBwdLayout::BM - 1) / tri::TriGateBwdLayout::BM,
+                             kGateMaxCtas);
+}
+}  // namespace
+
+size_t tri_gate_bwd_workspace_bytes(int R) {
+    if (R < 1) return 0;
+    return static_cast<size_t>(gate_ctas(R)) * tri::TriGateBwdLayout::PARTIAL_FLOATS * sizeof(float);
+}
+
+tri_attn_status tri_gate_bwd(const tri_gate_bwd_args* a, tri_attn_stream_t stream) {
+    if (!a) return TRI_ATTN_ERR_NULL;
+    const tri_gate_fwd_args& f = a->f;
+    if (!f.z || !f.o || !f.wg || !f.wo || !a->dy || !a->dz || !a->d_o || !a->dwg || !a->dwo) return TRI_ATTN_ERR_NULL;
+    if (f.R < 1) return TRI_ATTN_ERR_SHAPE;
+    for (int64_t st : {f.z_stride, f.o_stride, a->dy_stride, a->dz_stride, a->do_stride})
+        if (st < 128 || st % 8) return TRI_ATTN_ERR_STRIDE;
+    for (const void* ptr : {f.z, f.o, f.wg, f.wo, a->dy, static_cast<const void*>(a->dz),
+                            static_cast<const void*>(a->d_o), static_cast<const void*>(a->dwg),
+                            static_cast<const void*>(a->dwo)})
+        if (!aligned16(ptr)) return TRI_ATTN_ERR_ALIGN;
+    if (!a->workspace || !aligned16(a->workspace) || a->workspace_bytes < tri_gate_bwd_workspace_bytes(f.R))
+        return TRI_ATTN_ERR_WORKSPACE;
+    tri_attn_status st = ensure_device();
+    if (st) return st;
+    using L = tri::TriGateBwdLayout;
+    CUtensorMap mz, mdy, mwg, mwo;
+    if (!map_rows128(&mz, f.z, f.R, f.z_stride, L::BM) || !map_rows128(&mdy, a->dy, f.R, a->dy_stride, L::BM) ||
+        !map_rows128(&mwg, f.wg, 128, 128, 128) || !map_rows128(&mwo, f.wo, 128, 128, 128))
+        return TRI_ATTN_ERR_STRIDE;
+    tri::TriGateBwdParams p{};
+    p.R = f.R;
+    p.o = static_cast<const __nv_bfloat16*>(f.o);
+    p.os = f.o_stride;
+    p.dz = static_cast<__nv_bfloat16*>(a->dz);
+    p.dzs = a->dz_stride;
+    p.d_o = static_cast<__nv_bfloat16*>(a->d_o);
+    p.dos = a->do_stride;
+    p.partial = static_cast<float*>(a->workspace);
+    p.wait_limit_ns = g_wait_limit_ns.load();
+    const int grid = static_cast<int>(gate_ctas(f.R));
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    tri::tri_gate_bwd_kernel<<<grid, L::THREADS, L::SMEM, s>>>(mz, mdy, mwg, mwo, p);
+    constexpr int n4 = L::PARTIAL_FLOATS / 4;
+    tri::tri_gate_wsum_kernel<<<(n4 + 255) / 256, 256, 0, s>>>(p.partial, grid, a->dwg, a->dwo);
     return cudaGetLastError() == cudaSuccess ? TRI_ATTN_OK : TRI_ATTN_ERR_CUDA;
 }
 
