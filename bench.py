@@ -435,7 +435,7 @@ def run_gate(args):
     import torch
     from triangle_attention_biomolecular_b200 import _binding as Bd
     dev = torch.device("cuda", 0)
-    R = 768 * 768
+    R = args.gate_rows
     g = torch.Generator().manual_seed(5)
     z, o, dy = (torch.randn((R, 128), generator=g).to(torch.bfloat16).to(dev) for _ in range(3))
     wg, wo = ((torch.randn((128, 128), generator=g) / 128 ** 0.5).to(torch.bfloat16).to(dev) for _ in range(2))
@@ -478,7 +478,7 @@ def run_gate(args):
             "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": "gated output projection y = (sigmoid(z Wg) * o) Wo and its backward, "
-                                   "R = 768^2 pair positions, cz = H*d = 128",
+                                   f"R = {R} pair positions, cz = H*d = 128",
                        "bytes_per_step": f_bytes + b_bytes, "fwd_ms": round(f_ms, 4), "bwd_ms": round(b_ms, 4),
                        "fwd_gbs": round(f_bytes / (f_ms * 1e-3) / 1e9, 1), "bwd_gbs": round(b_gbs, 1),
                        "l2": "inputs (151 MB per tensor) larger than the 126 MB L2; no flush"},
@@ -589,6 +589,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", choices=("crop768", "crop640", "crop384"), default="crop768",
                     help="crop768 is the headline; the smaller crops serve profiler captures")
+    ap.add_argument("--gate-rows", type=int, default=768 * 768,
+                    help="pair positions R of the --op gate workload (default 768^2; smaller only for profiling)")
     ap.add_argument("--op", choices=("attention", "tri_mul", "gate"), default="attention",
                     help="attention (the headline), the triangle multiplicative contraction, or the gated "
                          "output projection")

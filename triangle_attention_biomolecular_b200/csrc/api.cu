@@ -486,19 +486,18 @@ tri_attn_status tri_gate_fwd(const tri_gate_fwd_args* a, tri_attn_stream_t strea
     tri_attn_status st = ensure_device();
     if (st) return st;
     using L = tri::TriGateLayout;
-    CUtensorMap mz, mo, mwg, mwo;
+    CUtensorMap mz, mo, mwg, mwo, my;
     if (!map_rows128(&mz, a->z, a->R, a->z_stride, L::BM) || !map_rows128(&mo, a->o, a->R, a->o_stride, L::BM) ||
-        !map_rows128(&mwg, a->wg, 128, 128, 128) || !map_rows128(&mwo, a->wo, 128, 128, 128))
+        !map_rows128(&mwg, a->wg, 128, 128, 128) || !map_rows128(&mwo, a->wo, 128, 128, 128) ||
+        !map_rows128(&my, a->y, a->R, a->y_stride, 32))
         return TRI_ATTN_ERR_STRIDE;
     tri::TriGateParams p{};
     p.R = a->R;
-    p.y = static_cast<__nv_bfloat16*>(a->y);
-    p.ys = a->y_stride;
     p.wait_limit_ns = g_wait_limit_ns.load();
     const int64_t tiles = (static_cast<int64_t>(a->R) + L::BM - 1) / L::BM;
     const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, 148));  // persistent, one CTA per SM
     tri::tri_gate_fwd_kernel<<<grid, L::THREADS, L::SMEM, reinterpret_cast<cudaStream_t>(stream)>>>(mz, mo, mwg, mwo,
-                                                                                                   p);
+                                                                                                   my, p);
     return cudaGetLastError() == cudaSuccess ? TRI_ATTN_OK : TRI_ATTN_ERR_CUDA;
 }
 
@@ -531,25 +530,23 @@ tri_attn_status tri_gate_bwd(const tri_gate_bwd_args* a, tri_attn_stream_t strea
     tri_attn_status st = ensure_device();
     if (st) return st;
     using L = tri::TriGateBwdLayout;
-    CUtensorMap mz, mdy, mwg, mwo;
+    CUtensorMap mz, mdy, mwg, mwo, mdz, mdo;
     if (!map_rows128(&mz, f.z, f.R, f.z_stride, L::BM) || !map_rows128(&mdy, a->dy, f.R, a->dy_stride, L::BM) ||
-        !map_rows128(&mwg, f.wg, 128, 128, 128) || !map_rows128(&mwo, f.wo, 128, 128, 128))
+        !map_rows128(&mwg, f.wg, 128, 128, 128) || !map_rows128(&mwo, f.wo, 128, 128, 128) ||
+        !map_rows128(&mdz, a->dz, f.R, a->dz_stride, 32) || !map_rows128(&mdo, a->d_o, f.R, a->do_stride, 32))
         return TRI_ATTN_ERR_STRIDE;
     tri::TriGateBwdParams p{};
     p.R = f.R;
     p.o = static_cast<const __nv_bfloat16*>(f.o);
     p.os = f.o_stride;
-    p.dz = static_cast<__nv_bfloat16*>(a->dz);
-    p.dzs = a->dz_stride;
-    p.d_o = static_cast<__nv_bfloat16*>(a->d_o);
-    p.dos = a->do_stride;
     p.partial = static_cast<float*>(a->workspace);
     p.wait_limit_ns = g_wait_limit_ns.load();
     const int grid = static_cast<int>(gate_ctas(f.R));
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    tri::tri_gate_bwd_kernel<<<grid, L::THREADS, L::SMEM, s>>>(mz, mdy, mwg, mwo, p);
-    constexpr int n4 = L::PARTIAL_FLOATS / 4;
-    tri::tri_gate_wsum_kernel<<<(n4 + 255) / 256, 256, 0, s>>>(p.partial, grid, a->dwg, a->dwo);
+    tri::tri_gate_bwd_kernel<<<grid, L::THREADS, L::SMEM, s>>>(mz, mdy, mwg, mwo, mdz, mdo, p);
+    constexpr int n4 = L::PARTIAL_FLOATS / 4, per_block = tri::kWsumThreads / 8;
+    tri::tri_gate_wsum_kernel<<<(n4 + per_block - 1) / per_block, tri::kWsumThreads, 0, s>>>(p.partial, grid, a->dwg,
+                                                                                             a->dwo);
     return cudaGetLastError() == cudaSuccess ? TRI_ATTN_OK : TRI_ATTN_ERR_CUDA;
 }
 

@@ -10,17 +10,18 @@
 // weight matrices resident and streams 128-position tiles through two
 // tcgen05 contractions with the gate in between.
 //
-// B200 mapping (one persistent CTA per SM, 192 threads):
-//  * warp 4 TMA producer: Wg, Wo once (MN-major B operands, 32 KB each), then
-//    per tile z (K-major A operand) and o (read by the epilogue) through a
-//    two-stage ring, 64 KB per stage;
-//  * warp 5 MMA issuer: G = z Wg into one of two 128-column TMEM accumulators,
+// B200 mapping (one persistent CTA per SM, 320 threads):
+//  * warp 8 TMA producer: Wg, Wo once (MN-major B operands, 32 KB each), then
+//    per tile z (K-major A operand) into one of two slots and o into one of
+//    three slots;
+//  * warp 9 MMA issuer: G = z Wg into one of two 128-column TMEM accumulators,
 //    later Y = a Wo into one of two more;
-//  * warps 0-3 (one row per thread): sigmoid of G (exp2 and reciprocal on the
-//    MUFU unit), a = g * o, BF16 a written to shared memory in the 128-byte-
-//    swizzled K-major layout the second MMA reads; then Y -> BF16 -> global,
-//    one tile behind, so the tensor cores, the MUFU unit and the stores of
-//    neighbouring tiles overlap.
+//  * warps 0-7 (warp w: rows 32 (w % 4) .. +31, one per thread, channel half
+//    w / 4): sigmoid of G (exp2 on the FMA pipe, reciprocal on the MUFU unit),
+//    a = g * o written in place over o -- whose 128-byte-swizzled K-major tile
+//    is exactly the A operand the second MMA reads -- then, one tile behind,
+//    Y -> BF16 into the same slot and out with a TMA store, so the tensor
+//    cores, the MUFU unit and the stores of neighbouring tiles overlap.
 #pragma once
 
 #include "sm100.cuh"
@@ -39,28 +40,27 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, 
 }
 
 struct TriGateParams {
-    int R;                  // pair positions
-    __nv_bfloat16* y;       // [R, 128]
-    int64_t ys;             // row stride (elements)
+    int R;  // pair positions
     uint64_t wait_limit_ns;
 };
 
 struct TriGateLayout {
     static constexpr int C = 128, BM = 128;
-    static constexpr int W_TILE = C * C * 2;          // 32 KB
-    static constexpr int X_TILE = BM * C * 2;         // 32 KB (two 64-column halves of 16 KB)
-    static constexpr int NS = 2;
+    static constexpr int W_TILE = C * C * 2;   // 32 KB
+    static constexpr int X_TILE = BM * C * 2;  // 32 KB (two 64-column halves of 16 KB)
+    static constexpr int HALF = X_TILE / 2;
+    static constexpr int NZ = 2, NO = 3;       // z slots, o slots
     static constexpr int OFF_WG = 0, OFF_WO = W_TILE;
-    static constexpr int OFF_STAGE = 2 * W_TILE;      // [NS][z, o]
-    static constexpr int STAGE = 2 * X_TILE;
-    static constexpr int OFF_A = OFF_STAGE + NS * STAGE;  // gated a, K-major, two halves
-    static constexpr int OFF_BAR = OFF_A + X_TILE;
-    static constexpr int B_W = 0, B_FULL = 1, B_XEMPTY = 1 + NS, B_GFULL = 1 + 2 * NS, B_GFREE = B_GFULL + 2,
-                         B_AFULL = B_GFREE + 2, B_AFREE = B_AFULL + 1, B_YFULL = B_AFREE + 1, B_YFREE = B_YFULL + 2,
-                         B_DRAIN = B_YFREE + 2, NBAR = B_DRAIN + 1;
+    static constexpr int OFF_Z = 2 * W_TILE;                // [NZ] z
+    static constexpr int OFF_O = OFF_Z + NZ * X_TILE;       // [NO] o, then a, then y
+    static constexpr int OFF_BAR = OFF_O + NO * X_TILE;
+    static constexpr int B_W = 0, B_ZFULL = 1, B_ZEMPTY = B_ZFULL + NZ, B_OFULL = B_ZEMPTY + NZ,
+                         B_OEMPTY = B_OFULL + NO, B_GFULL = B_OEMPTY + NO, B_GFREE = B_GFULL + 2,
+                         B_AFULL = B_GFREE + 2, B_YFULL = B_AFULL + 1, B_YFREE = B_YFULL + 2, B_DRAIN = B_YFREE + 2,
+                         NBAR = B_DRAIN + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack for 1 KB alignment
-    static constexpr int THREADS = 192;
+    static constexpr int EPI_WARPS = 8, W_PRODUCER = 8, W_MMA = 9, THREADS = 320;
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -70,10 +70,35 @@ __device__ __forceinline__ float rcp_approx(float x) {
     return y;
 }
 
-__global__ void __launch_bounds__(192, 1)
+// g = sigmoid(x) = 1 / (1 + e), e = 2^(-x log2 e), and h = 1 - g = e g (formed as a
+// product, so it keeps its relative accuracy when the gate saturates at 1), for a pair
+// of logits.  e comes from the FMA-pipe exp2 (relative error 1.4e-4), leaving the MUFU
+// unit only the reciprocal; its argument is clamped to [-125, 126], where the result
+// stays a normal number (g then rounds to 1 or to about 1e-38).
+__device__ __forceinline__ void sigmoid2(float x0, float x1, float2& g, float2& h) {
+    constexpr float NLOG2E = -1.4426950408889634f;
+    const float2 e = ex2_fma2(make_float2(fminf(x0 * NLOG2E, 126.f), fminf(x1 * NLOG2E, 126.f)));
+    g = make_float2(rcp_approx(1.f + e.x), rcp_approx(1.f + e.y));
+    h = make_float2(e.x * g.x, e.y * g.y);
+}
+
+// 2-D tiled TMA store from shared memory, tracked by the issuing thread's bulk group.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, uint32_t src, int c0, int c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// every bulk store this thread committed has finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// ... and has completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+__global__ void __launch_bounds__(320, 1)
     tri_gate_fwd_kernel(const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_o,
                         const __grid_constant__ CUtensorMap tm_wg, const __grid_constant__ CUtensorMap tm_wo,
-                        const TriGateParams p) {
+                        const __grid_constant__ CUtensorMap tm_y, const TriGateParams p) {
     using L = TriGateLayout;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
@@ -88,18 +113,21 @@ __global__ void __launch_bounds__(192, 1)
     if (threadIdx.x == 0) {
         *abort_flag = device_error_pending() ? 1 : 0;
         mbar_init(BAR(L::B_W), 1);
-        for (int s = 0; s < L::NS; ++s) {
-            mbar_init(BAR(L::B_FULL + s), 1);
-            mbar_init(BAR(L::B_XEMPTY + s), 1 + 4);  // MMA done with z + epilogue done with o
+        for (int i = 0; i < L::NZ; ++i) {
+            mbar_init(BAR(L::B_ZFULL + i), 1);
+            mbar_init(BAR(L::B_ZEMPTY + i), 1);
+        }
+        for (int i = 0; i < L::NO; ++i) {
+            mbar_init(BAR(L::B_OFULL + i), 1);
+            mbar_init(BAR(L::B_OEMPTY + i), L::EPI_WARPS);  // every warp's y box read out
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(BAR(L::B_GFULL + x), 1);
-            mbar_init(BAR(L::B_GFREE + x), 4);
+            mbar_init(BAR(L::B_GFREE + x), L::EPI_WARPS);
             mbar_init(BAR(L::B_YFULL + x), 1);
-            mbar_init(BAR(L::B_YFREE + x), 4);
+            mbar_init(BAR(L::B_YFREE + x), L::EPI_WARPS);
         }
-        mbar_init(BAR(L::B_AFULL), 4);
-        mbar_init(BAR(L::B_AFREE), 1);
+        mbar_init(BAR(L::B_AFULL), L::EPI_WARPS);
         mbar_init(BAR(L::B_DRAIN), 1);
         fence_mbar_init();
     }
@@ -114,10 +142,10 @@ __global__ void __launch_bounds__(192, 1)
     const WaitCtx wc{p.wait_limit_ns, KERNEL_TRIGATE, abort_flag};
     const bool aborted_early = *abort_flag != 0;
 
-    if (warp == 4) {
+    if (warp == L::W_PRODUCER) {
         // =========================== TMA producer ===========================
         const bool leader = elect_one();
-        int armed[L::NS] = {};
+        int zarmed[L::NZ] = {}, oarmed[L::NO] = {};
         bool w_armed = false;
         if (!aborted_early) {
             if (leader) {
@@ -133,67 +161,84 @@ __global__ void __launch_bounds__(192, 1)
             w_armed = true;
             int gt = 0;
             for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++gt) {
-                const int s = gt % L::NS;
-                if (gt >= L::NS && !mbar_wait_warp(BAR(L::B_XEMPTY + s), ((gt / L::NS) - 1) & 1, wc, 1)) break;
+                const int zs = gt % L::NZ, os = gt % L::NO;
+                if (gt >= L::NZ && !mbar_wait_warp(BAR(L::B_ZEMPTY + zs), ((gt / L::NZ) - 1) & 1, wc, 1)) break;
                 if (leader) {
-                    const uint32_t bar = BAR(L::B_FULL + s);
-                    const uint32_t st = sb + L::OFF_STAGE + s * L::STAGE;
-                    mbar_arrive_expect_tx(bar, L::STAGE);
-                    tma_load_2d(st, &tm_z, bar, 0, t * L::BM);
-                    tma_load_2d(st + L::X_TILE / 2, &tm_z, bar, 64, t * L::BM);
-                    tma_load_2d(st + L::X_TILE, &tm_o, bar, 0, t * L::BM);
-                    tma_load_2d(st + L::X_TILE + L::X_TILE / 2, &tm_o, bar, 64, t * L::BM);
+                    const uint32_t bar = BAR(L::B_ZFULL + zs), dst = sb + L::OFF_Z + zs * L::X_TILE;
+                    mbar_arrive_expect_tx(bar, L::X_TILE);
+                    tma_load_2d(dst, &tm_z, bar, 0, t * L::BM);
+                    tma_load_2d(dst + L::HALF, &tm_z, bar, 64, t * L::BM);
                 }
-                armed[s]++;
+                zarmed[zs]++;
+                if (gt >= L::NO && !mbar_wait_warp(BAR(L::B_OEMPTY + os), ((gt / L::NO) - 1) & 1, wc, 11)) break;
+                if (leader) {
+                    const uint32_t bar = BAR(L::B_OFULL + os), dst = sb + L::OFF_O + os * L::X_TILE;
+                    mbar_arrive_expect_tx(bar, L::X_TILE);
+                    tma_load_2d(dst, &tm_o, bar, 0, t * L::BM);
+                    tma_load_2d(dst + L::HALF, &tm_o, bar, 64, t * L::BM);
+                }
+                oarmed[os]++;
             }
         }
         if (leader) {
             if (w_armed) drain_wait(BAR(L::B_W), 0, 100000000ull);
 #pragma unroll
-            for (int s = 0; s < L::NS; ++s)
-                if (armed[s] > 0) drain_wait(BAR(L::B_FULL + s), (armed[s] - 1) & 1, 100000000ull);
+            for (int i = 0; i < L::NZ; ++i)
+                if (zarmed[i] > 0) drain_wait(BAR(L::B_ZFULL + i), (zarmed[i] - 1) & 1, 100000000ull);
+#pragma unroll
+            for (int i = 0; i < L::NO; ++i)
+                if (oarmed[i] > 0) drain_wait(BAR(L::B_OFULL + i), (oarmed[i] - 1) & 1, 100000000ull);
         }
-    } else if (warp == 5) {
+    } else if (warp == L::W_MMA) {
         // =========================== MMA issuer =============================
         const bool leader = elect_one();
         if (!aborted_early) {
             constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, false, true);
             // A (z, a): K-major, two 64-column halves 16 KB apart; B (Wg, Wo): MN-major,
             // 64-column chunks 16 KB apart (LBO), 8-k-row groups 1 KB apart (SBO)
-            const uint64_t dz0 = smem_desc(sb + L::OFF_STAGE, 16, 1024, SWZ_128B);
-            const uint64_t da0 = smem_desc(sb + L::OFF_A, 16, 1024, SWZ_128B);
-            const uint64_t dwg = smem_desc(sb + L::OFF_WG, L::W_TILE / 2, 1024, SWZ_128B);
-            const uint64_t dwo = smem_desc(sb + L::OFF_WO, L::W_TILE / 2, 1024, SWZ_128B);
+            const uint64_t dz0 = smem_desc(sb + L::OFF_Z, 16, 1024, SWZ_128B);
+            const uint64_t da0 = smem_desc(sb + L::OFF_O, 16, 1024, SWZ_128B);
+            const uint64_t dwg = smem_desc(sb + L::OFF_WG, L::HALF, 1024, SWZ_128B);
+            const uint64_t dwo = smem_desc(sb + L::OFF_WO, L::HALF, 1024, SWZ_128B);
             bool ok = mbar_wait_warp(BAR(L::B_W), 0, wc, 2);
+            TRI_TRACE_DECL
             int lt = 0;
             for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++lt) {
-                const int x = lt & 1, s = lt % L::NS;
-                if (!mbar_wait_warp(BAR(L::B_FULL + s), (lt / L::NS) & 1, wc, 3)) { ok = false; break; }
+                const int x = lt & 1, zs = lt % L::NZ, os = lt % L::NO;
+                TRI_TP(5)
+                if (!mbar_wait_warp(BAR(L::B_ZFULL + zs), (lt / L::NZ) & 1, wc, 3)) { ok = false; break; }
+                TRI_TP(0)
                 if (lt >= 2 && !mbar_wait_warp(BAR(L::B_GFREE + x), ((lt >> 1) - 1) & 1, wc, 4)) { ok = false; break; }
+                TRI_TP(1)
                 tc_fence_after();
                 if (leader) {
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_ss(tmem + x * 128, desc_add(dz0, s * L::STAGE + (kk >> 2) * (L::X_TILE / 2) + (kk & 3) * 32),
+                        mma_ss(tmem + x * 128, desc_add(dz0, zs * L::X_TILE + (kk >> 2) * L::HALF + (kk & 3) * 32),
                                desc_add(dwg, kk * 2048), IDESC, kk > 0 ? 1u : 0u);
                     mma_commit(BAR(L::B_GFULL + x));
-                    mma_commit(BAR(L::B_XEMPTY + s));
+                    mma_commit(BAR(L::B_ZEMPTY + zs));
                 }
                 __syncwarp();
-                // the gated a of this tile is in shared memory; Y[x] was read two tiles ago
+                // the gated a of this tile is in its o slot; Y[x] was read two tiles ago
+                TRI_TP(5)
                 if (!mbar_wait_warp(BAR(L::B_AFULL), lt & 1, wc, 5)) { ok = false; break; }
+                TRI_TP(2)
                 if (lt >= 2 && !mbar_wait_warp(BAR(L::B_YFREE + x), ((lt >> 1) - 1) & 1, wc, 6)) { ok = false; break; }
+                TRI_TP(3)
                 tc_fence_after();
                 if (leader) {
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_ss(tmem + 256 + x * 128, desc_add(da0, (kk >> 2) * (L::X_TILE / 2) + (kk & 3) * 32),
+                        mma_ss(tmem + 256 + x * 128,
+                               desc_add(da0, os * L::X_TILE + (kk >> 2) * L::HALF + (kk & 3) * 32),
                                desc_add(dwo, kk * 2048), IDESC, kk > 0 ? 1u : 0u);
                     mma_commit(BAR(L::B_YFULL + x));
-                    mma_commit(BAR(L::B_AFREE));
                 }
                 __syncwarp();
             }
+            TRI_TP(5)
+            TRI_TRACE_FLUSH_AT(0)
             if (leader) {
                 mma_commit(BAR(L::B_DRAIN));
                 drain_wait(BAR(L::B_DRAIN), 0, 100000000ull);
@@ -201,100 +246,108 @@ __global__ void __launch_bounds__(192, 1)
             __syncwarp();
         }
     } else {
-        // =========================== gate + epilogue (warps 0-3) =============
+        // =========================== gate + epilogue (warps 0-7) =============
         if (!aborted_early) {
-            constexpr float LOG2E = 1.4426950408889634f;
-            const int row = warp * 32 + lane;
-            const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+            const int q = warp & 3, h = warp >> 2;
+            const int row = q * 32 + lane;
+            const uint32_t tl = tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 64;
+            const uint32_t box = h * L::HALF + q * 32 * 128;  // this warp's 32 x 64 box within a slot
             bool ok = true;
-            // Y of tile lt (local index) -> BF16 -> global
+            TRI_TRACE_DECL
+            // Y of tile lt (local index) -> BF16 into its o slot -> TMA store
             auto store_y = [&](int lt, int t) -> bool {
                 const int x = lt & 1;
+                TRI_TP(6)
                 if (!mbar_wait_warp(BAR(L::B_YFULL + x), (lt >> 1) & 1, wc, 9)) return false;
+                TRI_TP(4)
                 tc_fence_after();
-                const int r = t * L::BM + row;
-                __nv_bfloat16* dst = p.y + static_cast<int64_t>(r) * p.ys;
-#pragma unroll 1
-                for (int c0 = 0; c0 < L::C; c0 += 32) {
+                const uint32_t slot = sb + L::OFF_O + (lt % L::NO) * L::X_TILE + h * L::HALF;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
                     uint32_t v[32];
-                    tmem_ld32(tl + 256 + x * 128 + c0, v);
+                    tmem_ld32(tl + 256 + x * 128 + 32 * j, v);
                     tmem_wait_ld();
-                    if (c0 == L::C - 32) {
+                    if (j == 1) {
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(BAR(L::B_YFREE + x));
                     }
-                    if (r < p.R) {
 #pragma unroll
-                        for (int e = 0; e < 32; e += 8) {
-                            uint4 q;
-                            q.x = pack_bf16(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-                            q.y = pack_bf16(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-                            q.z = pack_bf16(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]));
-                            q.w = pack_bf16(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7]));
-                            *reinterpret_cast<uint4*>(dst + c0 + e) = q;
-                        }
+                    for (int e = 0; e < 32; e += 8) {
+                        uint4 w;
+                        w.x = pack_bf16(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                        w.y = pack_bf16(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+                        w.z = pack_bf16(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]));
+                        w.w = pack_bf16(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7]));
+                        const int c = 4 * j + (e >> 3);
+                        sts128(slot + row * 128 + ((c ^ (row & 7)) << 4), w);
                     }
                 }
+                fence_proxy_async_smem();
+                __syncwarp();
+                const int box_row = t * L::BM + q * 32;
+                if (lane == 0 && box_row < p.R) {
+                    tma_store_2d(&tm_y, sb + L::OFF_O + (lt % L::NO) * L::X_TILE + box, h * 64, box_row);
+                    bulk_commit();
+                }
+                TRI_TP(5)
                 return true;
             };
             int lt = 0, prev_t = -1;
             for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++lt) {
-                const int x = lt & 1, s = lt % L::NS;
+                const int x = lt & 1, os = lt % L::NO;
+                TRI_TP(6)
                 if (!mbar_wait_warp(BAR(L::B_GFULL + x), (lt >> 1) & 1, wc, 7)) { ok = false; break; }
+                if (lt >= 2) {  // the y box of tile lt - 2 has left its slot
+                    if (lane == 0) {
+                        bulk_wait_read_all();
+                        mbar_arrive(BAR(L::B_OEMPTY + (lt - 2) % L::NO));
+                    }
+                    __syncwarp();
+                }
+                TRI_TP(0)
+                if (!mbar_wait_warp(BAR(L::B_OFULL + os), (lt / L::NO) & 1, wc, 8)) { ok = false; break; }
                 tc_fence_after();
-                // o of this tile arrived with z (the MMA has already waited for the stage)
-                if (!mbar_wait_warp(BAR(L::B_FULL + s), (lt / L::NS) & 1, wc, 8)) { ok = false; break; }
-                const uint32_t orow = sb + L::OFF_STAGE + s * L::STAGE + L::X_TILE + row * 128;
-                const uint32_t arow = sb + L::OFF_A + row * 128;
+                const uint32_t orow = sb + L::OFF_O + os * L::X_TILE + h * L::HALF + row * 128;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {  // 64-column halves
-                    uint32_t ga[32], gb[32];
-                    tmem_ld32(tl + x * 128 + h * 64, ga);
-                    tmem_ld32(tl + x * 128 + h * 64 + 32, gb);
+                for (int j = 0; j < 2; ++j) {  // 32-column chunks
+                    uint32_t gv[32];
+                    tmem_ld32(tl + x * 128 + 32 * j, gv);
                     tmem_wait_ld();
-                    if (h == 1) {
+                    if (j == 1) {
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(BAR(L::B_GFREE + x));
                     }
-                    uint32_t aw[32];
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {  // 16-byte chunks of 8 channels
-                        const uint4 ob = lds128(orow + h * (L::X_TILE / 2) + ((c ^ (row & 7)) << 4));
+                    for (int c = 0; c < 4; ++c) {  // 16-byte chunks of 8 channels
+                        const int cc = 4 * j + c;
+                        const uint32_t addr = orow + ((cc ^ (row & 7)) << 4);
+                        const uint4 ob = lds128(addr);
                         const uint32_t ow[4] = {ob.x, ob.y, ob.z, ob.w};
+                        uint32_t aw[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const int k = c * 8 + 2 * e;
-                            // sigmoid(G) = 1 / (1 + 2^(-G log2 e))
-                            const float l0 = __uint_as_float(k < 32 ? ga[k] : gb[k - 32]);
-                            const float l1 = __uint_as_float(k + 1 < 32 ? ga[k + 1] : gb[k + 1 - 32]);
-                            const float g0 = rcp_approx(1.f + ex2(-l0 * LOG2E));
-                            const float g1 = rcp_approx(1.f + ex2(-l1 * LOG2E));
-                            aw[c * 4 + e] = pack_bf16(g0 * bf16lo(ow[e]), g1 * bf16hi(ow[e]));
+                            float2 g, hh;
+                            sigmoid2(__uint_as_float(gv[8 * c + 2 * e]), __uint_as_float(gv[8 * c + 2 * e + 1]), g, hh);
+                            aw[e] = pack_bf16(g.x * bf16lo(ow[e]), g.y * bf16hi(ow[e]));
                         }
+                        sts128(addr, make_uint4(aw[0], aw[1], aw[2], aw[3]));  // a over o, in place
                     }
-                    if (h == 0 && lt > 0 && !mbar_wait_warp(BAR(L::B_AFREE), (lt - 1) & 1, wc, 10)) {
-                        ok = false;
-                        break;
-                    }
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        sts128(arow + h * (L::X_TILE / 2) + ((c ^ (row & 7)) << 4),
-                               make_uint4(aw[4 * c], aw[4 * c + 1], aw[4 * c + 2], aw[4 * c + 3]));
                 }
-                if (!ok) break;
+                TRI_TP(1)
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(BAR(L::B_AFULL));
-                    mbar_arrive(BAR(L::B_XEMPTY + s));
-                }
+                if (lane == 0) mbar_arrive(BAR(L::B_AFULL));
+                TRI_TP(3)
                 // the previous tile's output, while the tensor cores work on this one
                 if (prev_t >= 0 && !(ok = store_y(lt - 1, prev_t))) break;
                 prev_t = t;
             }
             if (ok && prev_t >= 0) store_y(lt - 1, prev_t);
+            if (lane == 0) bulk_wait_all();  // every y box has reached global memory
+            TRI_TP(6)
+            TRI_TRACE_FLUSH_AT(0)
         }
     }
     tc_fence_before();
@@ -325,6 +378,10 @@ __global__ void __launch_bounds__(192, 1)
 // CTA's tiles.  Even tiles put G and dz in P and dA in Q, odd tiles the other
 // way round, so that the next tile's G is computed while this tile's dz is
 // drained, and its dA while its G is being gated.
+// do and dz leave through shared memory and TMA stores (one 32-row x 64-column
+// box per epilogue warp): do in the dy slot of the tile's stage once MMA5 has
+// consumed dy, dz in the z slot once MMA4 has consumed z; the epilogue then
+// hands the stage back to the producer.
 // Each CTA writes its FP32 dWg, dWo partial sums to a workspace; a second
 // kernel adds the partials in CTA order (deterministic for a given R).
 //
@@ -333,19 +390,15 @@ __global__ void __launch_bounds__(192, 1)
 // Per tile, each epilogue thread: A1 reads G, writes a = g * o (BF16) into
 // the shared tile X and keeps g and s = o g (1 - g), both rounded to BF16, in
 // registers (s is formed in FP32 from the FP32 g, so 1 - g keeps its relative
-// accuracy for saturated gates); A2 reads dA, stores do = dA g, forms
-// dl = dA s, and once MMA5 has finished with a overwrites X with dl; B reads
-// dz and stores it.  o comes straight from global memory into
-// registers, prefetched one tile ahead.
+// accuracy for saturated gates); A2 reads dA and forms do = dA g and
+// dl = dA s, and once MMA5 has finished with a and dy writes dl over a in X and
+// do into the dy slot; B reads dz into the z slot.  o comes straight from
+// global memory into registers, prefetched one tile ahead.
 // ===========================================================================
 struct TriGateBwdParams {
     int R;
     const __nv_bfloat16* o;
     int64_t os;
-    __nv_bfloat16* dz;
-    int64_t dzs;
-    __nv_bfloat16* d_o;
-    int64_t dos;
     float* partial;  // [gridDim.x][2][128][128]: dWg, dWo partial sums of each CTA
     uint64_t wait_limit_ns;
 };
@@ -383,6 +436,7 @@ __device__ __forceinline__ uint4 ldg128_nc(const void* p) {
 __global__ void __launch_bounds__(320, 1)
     tri_gate_bwd_kernel(const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_dy,
                         const __grid_constant__ CUtensorMap tm_wg, const __grid_constant__ CUtensorMap tm_wo,
+                        const __grid_constant__ CUtensorMap tm_dz, const __grid_constant__ CUtensorMap tm_do,
                         const TriGateBwdParams p) {
     using L = TriGateBwdLayout;
     extern __shared__ uint8_t smem_raw[];
@@ -400,7 +454,7 @@ __global__ void __launch_bounds__(320, 1)
         mbar_init(BAR(L::B_W), 1);
         for (int s = 0; s < L::NS; ++s) {
             mbar_init(BAR(L::B_FULL + s), 1);
-            mbar_init(BAR(L::B_XEMPTY + s), 1);
+            mbar_init(BAR(L::B_XEMPTY + s), L::EPI_WARPS);  // both output boxes of every warp read out
         }
         for (int b : {L::B_GFULL, L::B_DAFULL, L::B_AFREE, L::B_DZFULL, L::B_ACC}) mbar_init(BAR(b), 1);
         for (int b : {L::B_A1DONE, L::B_A2DONE, L::B_DLFULL, L::B_BDONE}) mbar_init(BAR(b), L::EPI_WARPS);
@@ -474,14 +528,18 @@ __global__ void __launch_bounds__(320, 1)
             };
             const uint32_t wg = sb + L::OFF_WG, wo = sb + L::OFF_WO, xb = sb + L::OFF_X;
             bool ok = mbar_wait_warp(BAR(L::B_W), 0, wc, 2);
+            TRI_TRACE_DECL
             int lt = 0;
             for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++lt) {
                 const int s = lt % L::NS, par = lt & 1;
                 const uint32_t slot_g = tmem + (par ? 128u : 0u), slot_d = tmem + (par ? 0u : 128u);
                 const uint32_t zt = sb + L::OFF_STAGE + s * L::STAGE, dyt = zt + L::X_TILE;
                 // MMA1: G into the slot last holding the previous tile's dA
+                TRI_TP(5)
                 if (!mbar_wait_warp(BAR(L::B_FULL + s), (lt / L::NS) & 1, wc, 3)) { ok = false; break; }
+                TRI_TP(0)
                 if (lt > 0 && !mbar_wait_warp(BAR(L::B_A2DONE), (lt - 1) & 1, wc, 4)) { ok = false; break; }
+                TRI_TP(1)
                 tc_fence_after();
                 if (leader) {
 #pragma unroll
@@ -490,7 +548,9 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 __syncwarp();
                 // MMA2: dA into the slot last holding the previous tile's dz
+                TRI_TP(5)
                 if (lt > 0 && !mbar_wait_warp(BAR(L::B_BDONE), (lt - 1) & 1, wc, 5)) { ok = false; break; }
+                TRI_TP(2)
                 tc_fence_after();
                 if (leader) {
 #pragma unroll
@@ -499,7 +559,9 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 __syncwarp();
                 // MMA5: dWo += a^T dy
+                TRI_TP(5)
                 if (!mbar_wait_warp(BAR(L::B_A1DONE), lt & 1, wc, 6)) { ok = false; break; }
+                TRI_TP(3)
                 tc_fence_after();
                 if (leader) {
 #pragma unroll
@@ -509,7 +571,9 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 __syncwarp();
                 // MMA3: dz into G's slot (read by A1 before dl was written);  MMA4: dWg += z^T dl
+                TRI_TP(5)
                 if (!mbar_wait_warp(BAR(L::B_DLFULL), lt & 1, wc, 7)) { ok = false; break; }
+                TRI_TP(4)
                 tc_fence_after();
                 if (leader) {
 #pragma unroll
@@ -518,40 +582,89 @@ __global__ void __launch_bounds__(320, 1)
                     for (int kk = 0; kk < 8; ++kk)
                         mma_ss(tmem + 256, mnmaj(zt, kk), mnmaj(xb, kk), ID_MM, (lt > 0 || kk > 0) ? 1u : 0u);
                     mma_commit(BAR(L::B_DZFULL));
-                    mma_commit(BAR(L::B_XEMPTY + s));
                 }
                 __syncwarp();
             }
+            TRI_TP(5)
+            TRI_TRACE_FLUSH_AT(0)
             if (leader) mma_commit(BAR(L::B_ACC));  // every contraction above has completed
             __syncwarp();
         }
     } else {
         // =========================== epilogue (warps 0-7) =====================
         if (!aborted_early) {
-            constexpr float LOG2E = 1.4426950408889634f;
             const int q = warp & 3, h = warp >> 2;
             const int row = q * 32 + lane;
             const uint32_t tl = tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 64;
             const uint32_t xrow = sb + L::OFF_X + h * L::HALF + row * 128;
             const int ch0 = h * 64;  // first channel of this thread
-            uint4 ov[8];             // o[r, ch0 .. ch0 + 63] of the current tile
+            // o[r, ch0 .. ch0 + 63] of the current tile as eight 16-byte chunks.  Loaded
+            // coalesced -- lane 8a + b, load i fetches chunk b of warp row 8a + i, so one load
+            // covers four whole 128-byte lines -- then transposed within each group of
+            // eight lanes (three butterfly exchange steps) so that lane L holds row L.
+            uint32_t ov[8][4];
             auto load_o = [&](int t) {
-                const int r = t * L::BM + row;
-                const __nv_bfloat16* src = p.o + static_cast<int64_t>(r) * p.os + ch0;
+                const int a8 = lane >> 3, b8 = lane & 7;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) ov[c] = r < p.R ? ldg128_nc(src + 8 * c) : make_uint4(0, 0, 0, 0);
+                for (int i = 0; i < 8; ++i) {
+                    const int r = t * L::BM + q * 32 + 8 * a8 + i;
+                    const uint4 v = r < p.R ? ldg128_nc(p.o + static_cast<int64_t>(r) * p.os + ch0 + 8 * b8)
+                                            : make_uint4(0, 0, 0, 0);
+                    ov[i][0] = v.x;
+                    ov[i][1] = v.y;
+                    ov[i][2] = v.z;
+                    ov[i][3] = v.w;
+                }
+            };
+            auto transpose_o = [&]() {
+#pragma unroll
+                for (int k = 0; k < 3; ++k) {
+                    const int m = 1 << k;
+                    const bool up = (lane & m) != 0;
+#pragma unroll
+                    for (int i0 = 0; i0 < 8; ++i0) {
+                        if (i0 & m) continue;
+                        const int i1 = i0 | m;
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            const uint32_t recv = __shfl_xor_sync(0xffffffffu, up ? ov[i0][w] : ov[i1][w], m);
+                            if (up)
+                                ov[i0][w] = recv;
+                            else
+                                ov[i1][w] = recv;
+                        }
+                    }
+                }
             };
             bool ok = true;
             int lt = 0;
             if (blockIdx.x < tiles) load_o(blockIdx.x);
+            TRI_TRACE_DECL
             for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++lt) {
                 const int par = lt & 1;
                 const uint32_t slot_g = tl + (par ? 128u : 0u), slot_d = tl + (par ? 0u : 128u);
-                const int r = t * L::BM + row;
-                const bool live = r < p.R;
+                TRI_TP(7)
+#ifdef TRI_TRACE
+                {  // time the wait for this tile's o on its own
+                    uint32_t x_ = 0;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) x_ ^= ov[c][0] ^ ov[c][3];
+                    if (x_ == 0x9e3779b9u) asm volatile("" ::: "memory");
+                }
+                TRI_TP(9)
+#endif
                 // ---- A1: g = sigmoid(G), a = g * o -> X; keep g and s = o g (1 - g) ----
                 if (!mbar_wait_warp(BAR(L::B_GFULL), lt & 1, wc, 8)) { ok = false; break; }
+                if (lt > 0) {  // the previous tile's do and dz boxes have left its stage
+                    if (lane == 0) {
+                        bulk_wait_read_all();
+                        mbar_arrive(BAR(L::B_XEMPTY + (lt - 1) % L::NS));
+                    }
+                    __syncwarp();
+                }
+                TRI_TP(0)
                 tc_fence_after();
+                transpose_o();
                 uint32_t gw[32], sw[32];  // BF16 pairs of g and s for the 64 channels
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {  // 16-column chunks
@@ -560,18 +673,17 @@ __global__ void __launch_bounds__(320, 1)
                     tmem_wait_ld();
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {  // 8 channels
-                        const uint4 o4 = ov[2 * j + c];
-                        const uint32_t ow[4] = {o4.x, o4.y, o4.z, o4.w};
+                        const uint32_t* ow = ov[2 * j + c];
                         uint32_t aw[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int k = 8 * c + 2 * e;
-                            const float g0 = rcp_approx(1.f + ex2(-__uint_as_float(v[k]) * LOG2E));
-                            const float g1 = rcp_approx(1.f + ex2(-__uint_as_float(v[k + 1]) * LOG2E));
+                            float2 g, h;  // g and 1 - g
+                            sigmoid2(__uint_as_float(v[k]), __uint_as_float(v[k + 1]), g, h);
                             const float o0 = bf16lo(ow[e]), o1 = bf16hi(ow[e]);
-                            aw[e] = pack_bf16(g0 * o0, g1 * o1);
-                            gw[8 * j + 4 * c + e] = pack_bf16(g0, g1);
-                            sw[8 * j + 4 * c + e] = pack_bf16(o0 * (g0 * (1.f - g0)), o1 * (g1 * (1.f - g1)));
+                            aw[e] = pack_bf16(g.x * o0, g.y * o1);
+                            gw[8 * j + 4 * c + e] = pack_bf16(g.x, g.y);
+                            sw[8 * j + 4 * c + e] = pack_bf16(o0 * (g.x * h.x), o1 * (g.y * h.y));
                         }
                         const int cc = 2 * j + c;  // 16-byte chunk within the 128-byte row
                         sts128(xrow + ((cc ^ (row & 7)) << 4), make_uint4(aw[0], aw[1], aw[2], aw[3]));
@@ -581,11 +693,12 @@ __global__ void __launch_bounds__(320, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(BAR(L::B_A1DONE));
-                // ---- A2: dA -> do = dA g (global), dl = dA s (registers) ----
+                TRI_TP(1)
+                // ---- A2: dA -> do = dA g, dl = dA s (registers) ----
                 if (!mbar_wait_warp(BAR(L::B_DAFULL), lt & 1, wc, 9)) { ok = false; break; }
+                TRI_TP(2)
                 tc_fence_after();
-                uint32_t dlw[32];
-                __nv_bfloat16* dodst = p.d_o + static_cast<int64_t>(r) * p.dos + ch0;
+                uint32_t dlw[32], dow[32];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     uint32_t v[16];
@@ -593,35 +706,48 @@ __global__ void __launch_bounds__(320, 1)
                     tmem_wait_ld();
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
-                        uint32_t dw[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int k = 8 * c + 2 * e, w = 8 * j + 4 * c + e;
                             const float da0 = __uint_as_float(v[k]), da1 = __uint_as_float(v[k + 1]);
-                            dw[e] = pack_bf16(da0 * bf16lo(gw[w]), da1 * bf16hi(gw[w]));
+                            dow[w] = pack_bf16(da0 * bf16lo(gw[w]), da1 * bf16hi(gw[w]));
                             dlw[w] = pack_bf16(da0 * bf16lo(sw[w]), da1 * bf16hi(sw[w]));
                         }
-                        if (live)
-                            *reinterpret_cast<uint4*>(dodst + 16 * j + 8 * c) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(BAR(L::B_A2DONE));
-                // ---- dl -> X once MMA5 has read a ----
+                TRI_TP(3)
+                // ---- dl -> X, do -> dy slot, once MMA5 has read a and dy ----
                 if (!mbar_wait_warp(BAR(L::B_AFREE), lt & 1, wc, 10)) { ok = false; break; }
+                TRI_TP(4)
+                const uint32_t zslot = sb + L::OFF_STAGE + (lt % L::NS) * L::STAGE, dyslot = zslot + L::X_TILE;
+                const uint32_t box = h * L::HALF + q * 32 * 128;  // this warp's 32 x 64 box in a slot
+                const int box_row = t * L::BM + q * 32;
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
+                for (int c = 0; c < 8; ++c) {
+                    const uint32_t off = row * 128 + ((c ^ (row & 7)) << 4);
                     sts128(xrow + ((c ^ (row & 7)) << 4), make_uint4(dlw[4 * c], dlw[4 * c + 1], dlw[4 * c + 2], dlw[4 * c + 3]));
+                    sts128(dyslot + h * L::HALF + off,
+                           make_uint4(dow[4 * c], dow[4 * c + 1], dow[4 * c + 2], dow[4 * c + 3]));
+                }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(BAR(L::B_DLFULL));
+                if (lane == 0) {
+                    mbar_arrive(BAR(L::B_DLFULL));
+                    if (box_row < p.R) {
+                        tma_store_2d(&tm_do, dyslot + box, ch0, box_row);
+                        bulk_commit();
+                    }
+                }
                 // fetch the next tile's o while this tile's dz is formed and drained
                 if (t + static_cast<int>(gridDim.x) < tiles) load_o(t + gridDim.x);
-                // ---- B: dz -> global ----
+                TRI_TP(5)
+                // ---- B: dz -> z slot -> global ----
                 if (!mbar_wait_warp(BAR(L::B_DZFULL), lt & 1, wc, 11)) { ok = false; break; }
+                TRI_TP(6)
                 tc_fence_after();
-                __nv_bfloat16* dzdst = p.dz + static_cast<int64_t>(r) * p.dzs + ch0;
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     uint32_t v[32];
@@ -632,19 +758,26 @@ __global__ void __launch_bounds__(320, 1)
                         __syncwarp();
                         if (lane == 0) mbar_arrive(BAR(L::B_BDONE));
                     }
-                    if (live) {
 #pragma unroll
-                        for (int e = 0; e < 32; e += 8) {
-                            uint4 w;
-                            w.x = pack_bf16(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-                            w.y = pack_bf16(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-                            w.z = pack_bf16(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]));
-                            w.w = pack_bf16(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7]));
-                            *reinterpret_cast<uint4*>(dzdst + 32 * j + e) = w;
-                        }
+                    for (int e = 0; e < 32; e += 8) {
+                        uint4 w;
+                        w.x = pack_bf16(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                        w.y = pack_bf16(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+                        w.z = pack_bf16(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]));
+                        w.w = pack_bf16(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7]));
+                        const int c = 4 * j + (e >> 3);
+                        sts128(zslot + h * L::HALF + row * 128 + ((c ^ (row & 7)) << 4), w);
                     }
                 }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && box_row < p.R) {
+                    tma_store_2d(&tm_dz, zslot + box, ch0, box_row);
+                    bulk_commit();
+                }
             }
+            if (lane == 0) bulk_wait_all();  // every output box has reached global memory
+            TRI_TP(7)
             // ---- weight-gradient partial sums -> workspace ----
             if (ok && mbar_wait_warp(BAR(L::B_ACC), 0, wc, 12)) {
                 tc_fence_after();
@@ -663,6 +796,8 @@ __global__ void __launch_bounds__(320, 1)
                     }
                 }
             }
+            TRI_TP(8)
+            TRI_TRACE_FLUSH_AT(0)
         }
     }
     tc_fence_before();
@@ -673,50 +808,54 @@ __global__ void __launch_bounds__(320, 1)
     }
 }
 
-// dW[w][i][j] = sum over CTAs b = 0, 1, ... of partial[b][w][i][j], in that order
-// (four interleaved running sums, combined at the end, so the result is the same
-// on every run for the same number of partials).
-__global__ void __launch_bounds__(256) tri_gate_wsum_kernel(const float* __restrict__ partial, int nparts,
-                                                             float* __restrict__ dwg, float* __restrict__ dwo) {
+// dW[w][i][j] = sum over CTAs b of partial[b][w][i][j].  Eight threads share each
+// float4 of the result: thread k adds partials k, k + 8, k + 16, ... in that order,
+// then the eight partial sums are combined by a butterfly (pairwise sums are
+// commutative, so every lane ends with the same bits).  The association is fixed
+// by the number of partials alone, so repeated runs give identical results.
+constexpr int kWsumThreads = 256;
+__global__ void __launch_bounds__(kWsumThreads) tri_gate_wsum_kernel(const float* __restrict__ partial, int nparts,
+                                                                      float* __restrict__ dwg, float* __restrict__ dwo) {
     if (device_error_pending()) return;
     constexpr int N4 = TriGateBwdLayout::PARTIAL_FLOATS / 4;
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;  // float4 index in [0, N4)
-    if (i >= N4) return;
+    const int i = blockIdx.x * (kWsumThreads / 8) + (threadIdx.x >> 3);  // float4 index in [0, N4)
+    const int k = threadIdx.x & 7;
+    if (i >= N4) return;  // whole groups of eight leave together
     const float4* src = reinterpret_cast<const float4*>(partial) + i;
-    float4 acc[4];
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    int b = k;
+    for (; b + 24 < nparts; b += 32) {
+        float4 x[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-    int b = 0;
-    for (; b + 4 <= nparts; b += 4) {
+        for (int u = 0; u < 4; ++u) x[u] = src[static_cast<int64_t>(b + 8 * u) * N4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const float4 x = src[static_cast<int64_t>(b + u) * N4];
-            acc[u].x += x.x;
-            acc[u].y += x.y;
-            acc[u].z += x.z;
-            acc[u].w += x.w;
+            acc.x += x[u].x;
+            acc.y += x[u].y;
+            acc.z += x[u].z;
+            acc.w += x[u].w;
         }
+    }
+    for (; b < nparts; b += 8) {
+        const float4 x = src[static_cast<int64_t>(b) * N4];
+        acc.x += x.x;
+        acc.y += x.y;
+        acc.z += x.z;
+        acc.w += x.w;
     }
 #pragma unroll
-    for (int u = 0; u < 3; ++u) {
-        if (b + u < nparts) {
-            const float4 x = src[static_cast<int64_t>(b + u) * N4];
-            acc[u].x += x.x;
-            acc[u].y += x.y;
-            acc[u].z += x.z;
-            acc[u].w += x.w;
-        }
+    for (int m = 1; m < 8; m <<= 1) {
+        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, m);
+        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, m);
+        acc.z += __shfl_xor_sync(0xffffffffu, acc.z, m);
+        acc.w += __shfl_xor_sync(0xffffffffu, acc.w, m);
     }
-    float4 r;
-    r.x = (acc[0].x + acc[1].x) + (acc[2].x + acc[3].x);
-    r.y = (acc[0].y + acc[1].y) + (acc[2].y + acc[3].y);
-    r.z = (acc[0].z + acc[1].z) + (acc[2].z + acc[3].z);
-    r.w = (acc[0].w + acc[1].w) + (acc[2].w + acc[3].w);
+    if (k != 0) return;
     constexpr int HALF4 = N4 / 2;
     if (i < HALF4)
-        reinterpret_cast<float4*>(dwg)[i] = r;
+        reinterpret_cast<float4*>(dwg)[i] = acc;
     else
-        reinterpret_cast<float4*>(dwo)[i - HALF4] = r;
+        reinterpret_cast<float4*>(dwo)[i - HALF4] = acc;
 }
 
 }  // namespace tri
