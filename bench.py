@@ -38,6 +38,24 @@ WORKLOAD = "crop768 triangle attention fwd+bwd (starting node): B=1, N=768, H=4,
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time of the timed region: every rank passes its own and all
+    get the maximum (a collective; every rank must call it)."""
+    if world == 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    tt = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def whole_job_rate(world: int, work_per_step: float, steps: int, ms: float, scale: float = 1e12) -> float:
+    """Whole-job throughput: every rank did `steps` steps of `work_per_step` each (weak
+    scaling: replicas of the same workload) within the slowest rank's `ms`."""
+    return world * work_per_step * steps / (ms * 1e-3) / scale
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -199,11 +217,7 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     st, word = Bd.tri_attn_device_error(True)
     if st != 0:
         raise RuntimeError(f"device error word {word:#x} during timing")
@@ -278,16 +292,12 @@ def run_ours(args, rank, world, local_rank):
             e2e_step(n)
         a1.record(s_out)
         torch.cuda.synchronize()
-        ems = a0.elapsed_time(a1)
-        if world > 1:
-            tt = torch.tensor([ems], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ems = float(tt.item())
+        ems = max_over_ranks(a0.elapsed_time(a1), world, dev)
         st, word = Bd.tri_attn_device_error(True)
         if st != 0:
             raise RuntimeError(f"device error word {word:#x} during the end-to-end leg")
         fl = flops(Bn, N, H, d)["step"]
-        e2e = {"value": round(world * fl * n_e2e / (ems * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+        e2e = {"value": round(whole_job_rate(world, fl, n_e2e, ems), 3), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
                "ms_per_step": round(ems / n_e2e, 4),
                "pipelining": "two buffer sets; H2D, compute and D2H on three streams"}
@@ -411,11 +421,7 @@ def run_tri_mul(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     st, word = Bd.tri_attn_device_error(True)
     if st != 0:
         raise RuntimeError(f"device error word {word:#x}")
@@ -636,7 +642,7 @@ def main():
         pk, src = peaks()
         peak = float(pk["bf16_tflops"])
         step_flops = 6.0 * Bn * C * N ** 3
-        value = world * step_flops * args.steps / (res["ms"] * 1e-3) / 1e12
+        value = whole_job_rate(world, step_flops, args.steps, res["ms"])
         fwd_t = 2.0 * Bn * C * N ** 3 / (res["fwd_ms"] * 1e-3) / 1e12
         bwd_t = 4.0 * Bn * C * N ** 3 / (res["bwd_ms"] * 1e-3) / 1e12
         line = {
@@ -665,7 +671,7 @@ def main():
     peak = float(pk["bf16_tflops"])
     ms = res["ms"]
     per_step_ms = ms / args.steps
-    value = world * fl["step"] * args.steps / (ms * 1e-3) / 1e12
+    value = whole_job_rate(world, fl["step"], args.steps, ms)
     km = res["kern_ms"]
     algo = {"fwd": fl["fwd"], "bwd_main": fl["bwd_main"], "bwd_dbias": fl["bwd_dbias"]}
     dom = max(algo, key=lambda n: km[n])
@@ -700,7 +706,7 @@ def main():
                      "peak_source": f"{src} bf16_tflops (burst)"},
         "step_ms": {k: round(v, 4) for k, v in res["step_stats"].items()},
         "roofs_ms": {k: round(v, 4) for k, v in roofs_ms.items()},
-        "effective_tflops": round(world * eff_flops * args.steps / (ms * 1e-3) / 1e12, 3),
+        "effective_tflops": round(whole_job_rate(world, eff_flops, args.steps, ms), 3),
         "gpu_launches": 4 * args.steps,
         "clocks": res["clocks"],
         "e2e": res["e2e"],

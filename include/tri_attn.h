@@ -168,6 +168,46 @@ tri_attn_status tri_attn_bwd(const tri_attn_bwd_args *args, tri_attn_stream_t st
 tri_attn_status tri_attn_bwd_marked(const tri_attn_bwd_args *args, tri_attn_stream_t stream,
                                     void *const *markers);
 
+/* ---------------------------------------------------------------------------
+ * Row shards (a 1-D split of the rows i across devices, as in Design-CP's
+ * row-wise partitioning of the pair representation).  The problems of
+ * different rows i are independent except for dBias, the sum over i of the
+ * score gradient: each shard returns its share of that sum in FP32, and
+ * tri_attn_dbias_sum adds the shares of all shards in a fixed order.
+ *
+ * A shard call covers rows i0 .. i0+rows-1 of the full problem:
+ *   args->N            : the full N (the j and k extent; bias is [B,H,N,N])
+ *   q,k,v,o,resid,dout,dq,dk,dv : point at row i0 (strides unchanged)
+ *   mask.ptr           : points at row i0 (if not NULL)
+ *   lse                : this shard's own contiguous FP32 [B,H,rows,N] array
+ *   1 <= rows <= N, else TRI_ATTN_ERR_SHAPE.
+ * With rows = N and no offset, tri_attn_fwd_rows equals tri_attn_fwd bit for
+ * bit, and so do the o, resid, lse, dq, dk, dv of a shard and of the whole.
+ * --------------------------------------------------------------------------- */
+tri_attn_status tri_attn_fwd_rows(const tri_attn_fwd_args *args, int rows, tri_attn_stream_t stream);
+
+/* Workspace bytes of tri_attn_bwd_rows (pure function; 0 for invalid sizes). */
+size_t tri_attn_bwd_rows_workspace_bytes(int B, int rows, int N, int H, int d);
+
+/* Number P of FP32 dBias partial sums tri_attn_bwd_rows writes for these sizes
+ * (pure function, the same for every shard of equal rows; 0 if invalid). */
+int tri_attn_bwd_rows_dbias_parts(int B, int rows, int N, int H, int d);
+
+/* Backward of one shard: dq, dk, dv of its rows as tri_attn_bwd does, and its
+ * share of dBias as P contiguous FP32 [B,H,N,N] arrays in dbias_parts
+ * (caller-owned, 16-byte aligned, P * B*H*N*N floats, overwritten); their sum
+ * is the shard's sum over its rows of the score gradient.  args->dbias is not
+ * used.  Workspace: tri_attn_bwd_rows_workspace_bytes. */
+tri_attn_status tri_attn_bwd_rows(const tri_attn_bwd_args *args, int rows, float *dbias_parts,
+                                  tri_attn_stream_t stream);
+
+/* dbias = BF16 RNE of the sum of nparts contiguous FP32 [B,H,N,N] arrays,
+ * added in ascending index order (the shards' partials gathered in rank
+ * order: every device that calls this on the same gathered array gets the
+ * same bits).  parts 16-byte aligned; dbias strides as in tri_attn_bwd. */
+tri_attn_status tri_attn_dbias_sum(const float *parts, int nparts, int B, int H, int N, tri_attn_tensor4 dbias,
+                                   tri_attn_stream_t stream);
+
 /* Size of the static scratch area of tri_attn_bwd_static_scratch, per device:
  * 64 MiB, enough for every size whose tri_attn_bwd_workspace_bytes is at most
  * that (for example B=1, N=768, H=4 at d=32 or d=64). */

@@ -1,0 +1,56 @@
+"""The multi-rank plumbing of bench.py on CPU (gloo ranks, no GPU): the timed region
+is the slowest rank's, every rank receives it, the whole-job value counts every rank's
+steps, and the reference arm runs on rank 0 only."""
+import argparse
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+import bench
+
+
+def free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, tmpdir):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        mine = 2.5 + 1.5 * rank  # this rank's time of the timed region
+        got = bench.max_over_ranks(mine, world, torch.device("cpu"))
+        np.save(os.path.join(tmpdir, f"ms{rank}.npy"), np.array([mine, got]))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_every_rank_gets_the_slowest_time(world, tmp_path):
+    import torch.multiprocessing as mp
+    mp.spawn(_worker, args=(world, free_port(), str(tmp_path)), nprocs=world, join=True)
+    res = [np.load(tmp_path / f"ms{r}.npy") for r in range(world)]
+    slowest = max(r[0] for r in res)
+    assert all(r[1] == slowest for r in res)
+
+
+def test_single_rank_needs_no_process_group():
+    assert bench.max_over_ranks(1.25, 1, torch.device("cpu")) == 1.25
+
+
+def test_whole_job_rate_counts_every_rank():
+    # 3 ranks x 10 steps x 2e12 flops in 40 ms -> 1500 TFLOP/s for the job, 500 per rank
+    assert bench.whole_job_rate(3, 2e12, 10, 40.0) == pytest.approx(1500.0)
+    assert bench.whole_job_rate(1, 2e12, 10, 40.0) == pytest.approx(500.0)
+
+
+def test_reference_arm_runs_on_rank_zero_only(capsys):
+    args = argparse.Namespace(steps=1, warmup=0, gpus=2, workload="crop768", op="attention")
+    bench.run_reference(args, rank=1, world=2)
+    assert capsys.readouterr().out == ""

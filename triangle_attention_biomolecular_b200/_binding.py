@@ -120,6 +120,18 @@ def load() -> ctypes.CDLL:
             lib.tri_attn_bwd_static_scratch.restype = ctypes.c_int
             lib.tri_attn_bwd_workspace_bytes.argtypes = [ctypes.c_int] * 4
             lib.tri_attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+            lib.tri_attn_fwd_rows.argtypes = [ctypes.POINTER(FwdArgs), ctypes.c_int, ctypes.c_void_p]
+            lib.tri_attn_fwd_rows.restype = ctypes.c_int
+            lib.tri_attn_bwd_rows.argtypes = [ctypes.POINTER(BwdArgs), ctypes.c_int, ctypes.c_void_p,
+                                              ctypes.c_void_p]
+            lib.tri_attn_bwd_rows.restype = ctypes.c_int
+            lib.tri_attn_bwd_rows_workspace_bytes.argtypes = [ctypes.c_int] * 5
+            lib.tri_attn_bwd_rows_workspace_bytes.restype = ctypes.c_size_t
+            lib.tri_attn_bwd_rows_dbias_parts.argtypes = [ctypes.c_int] * 5
+            lib.tri_attn_bwd_rows_dbias_parts.restype = ctypes.c_int
+            lib.tri_attn_dbias_sum.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, Tensor4, ctypes.c_void_p]
+            lib.tri_attn_dbias_sum.restype = ctypes.c_int
             lib.tri_attn_strerror.argtypes = [ctypes.c_int]
             lib.tri_attn_strerror.restype = ctypes.c_char_p
             lib.tri_attn_device_error.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_uint32)]
@@ -190,20 +202,22 @@ def _stream_handle(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def fwd_args(q, k, v, bias, mask, o, resid, lse, scale: float = 0.0) -> FwdArgs:
+def fwd_args(q, k, v, bias, mask, o, resid, lse, scale: float = 0.0, rows_ok: bool = False) -> FwdArgs:
+    """Pair tensors [B,R,N,H,d]: R = N for the whole problem; with rows_ok, R <= N rows
+    of a row shard (views starting at its first row), lse [B,H,R,N], mask [B,R,N]."""
     import torch
-    B, N, N2, H, d = q.shape
-    if N2 != N:
+    B, R, N, H, d = q.shape
+    if R != N and not (rows_ok and 1 <= R <= N):
         raise TriAttnError(TRI_ATTN_ERR_SHAPE, "q must be [B,N,N,H,d]")
     for name, t in (("k", k), ("v", v), ("o", o), ("resid", resid)):
-        if tuple(t.shape) != (B, N, N, H, d):
-            raise TriAttnError(TRI_ATTN_ERR_SHAPE, f"{name} shape {tuple(t.shape)} != {(B, N, N, H, d)}")
+        if tuple(t.shape) != (B, R, N, H, d):
+            raise TriAttnError(TRI_ATTN_ERR_SHAPE, f"{name} shape {tuple(t.shape)} != {(B, R, N, H, d)}")
     if tuple(bias.shape) != (B, H, N, N):
         raise TriAttnError(TRI_ATTN_ERR_SHAPE, "bias must be [B,H,N,N]")
-    if mask is not None and tuple(mask.shape) != (B, N, N):
+    if mask is not None and tuple(mask.shape) != (B, R, N):
         raise TriAttnError(TRI_ATTN_ERR_SHAPE, "mask must be [B,N,N] (b,i,k)")
     _check_tensor(lse, "lse", torch.float32, 4)
-    if tuple(lse.shape) != (B, H, N, N) or not lse.is_contiguous():
+    if tuple(lse.shape) != (B, H, R, N) or not lse.is_contiguous():
         raise TriAttnError(TRI_ATTN_ERR_SHAPE, "lse must be a contiguous [B,H,N,N] float32 tensor")
     a = FwdArgs()
     a.B, a.N, a.H, a.d = B, N, H, d
@@ -241,13 +255,18 @@ def tri_attn_fwd(q, k, v, bias, mask, o, resid, lse, scale: float = 0.0, stream=
 
 
 def bwd_args(q, k, v, bias, mask, o, resid, lse, dout, dq, dk, dv, dbias, workspace,
-             scale: float = 0.0, flags: int = 0) -> BwdArgs:
+             scale: float = 0.0, flags: int = 0, rows_ok: bool = False) -> BwdArgs:
     import torch
     a = BwdArgs()
-    a.f = fwd_args(q, k, v, bias, mask, o, resid, lse, scale)
+    a.f = fwd_args(q, k, v, bias, mask, o, resid, lse, scale, rows_ok)
+    shape = tuple(q.shape)
+    for name, t in (("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv)):
+        if tuple(t.shape) != shape:
+            raise TriAttnError(TRI_ATTN_ERR_SHAPE, f"{name} shape {tuple(t.shape)} != {shape}")
     a.dout = t5(dout, "dout")
     a.dq, a.dk, a.dv = t5(dq, "dq"), t5(dk, "dk"), t5(dv, "dv")
-    a.dbias = t4(dbias, "dbias")
+    if dbias is not None:
+        a.dbias = t4(dbias, "dbias")
     if workspace is None:
         a.workspace, a.workspace_bytes = None, 0
     else:
@@ -288,6 +307,57 @@ def tri_attn_bwd_static_scratch(q, k, v, bias, mask, o, resid, lse, dout, dq, dk
     st = load().tri_attn_bwd_static_scratch(ctypes.byref(a), _stream_handle(stream))
     if st != TRI_ATTN_OK:
         raise TriAttnError(st, "tri_attn_bwd_static_scratch")
+
+
+def tri_attn_bwd_rows_workspace_bytes(B: int, rows: int, N: int, H: int, d: int) -> int:
+    return int(load().tri_attn_bwd_rows_workspace_bytes(B, rows, N, H, d))
+
+
+def tri_attn_bwd_rows_dbias_parts(B: int, rows: int, N: int, H: int, d: int) -> int:
+    return int(load().tri_attn_bwd_rows_dbias_parts(B, rows, N, H, d))
+
+
+def tri_attn_fwd_rows(q, k, v, bias, mask, o, resid, lse, scale: float = 0.0, stream=None) -> None:
+    """Forward of a row shard: pair tensors are [B,R,N,H,d] views starting at the shard's
+    first row (mask [B,R,N] likewise), bias the full [B,H,N,N], lse its own [B,H,R,N]."""
+    a = fwd_args(q, k, v, bias, mask, o, resid, lse, scale, rows_ok=True)
+    st = load().tri_attn_fwd_rows(ctypes.byref(a), q.shape[1], _stream_handle(stream))
+    if st != TRI_ATTN_OK:
+        raise TriAttnError(st, "tri_attn_fwd_rows")
+
+
+def tri_attn_bwd_rows(q, k, v, bias, mask, o, resid, lse, dout, dq, dk, dv, dbias_parts, workspace,
+                      scale: float = 0.0, flags: int = 0, stream=None) -> None:
+    """Backward of a row shard: dq, dk, dv of its rows and its share of dBias as
+    FP32 partial sums, dbias_parts a contiguous float32 [P,B,H,N,N] tensor with
+    P = tri_attn_bwd_rows_dbias_parts(...)."""
+    import torch
+    a = bwd_args(q, k, v, bias, mask, o, resid, lse, dout, dq, dk, dv, None, workspace, scale, flags,
+                 rows_ok=True)
+    B, R, N, H, d = q.shape
+    P = tri_attn_bwd_rows_dbias_parts(B, R, N, H, d)
+    if (dbias_parts.dtype != torch.float32 or not dbias_parts.is_contiguous()
+            or tuple(dbias_parts.shape) != (P, B, H, N, N)):
+        raise TriAttnError(TRI_ATTN_ERR_SHAPE, f"dbias_parts must be a contiguous float32 {(P, B, H, N, N)} tensor")
+    st = load().tri_attn_bwd_rows(ctypes.byref(a), R, ctypes.c_void_p(dbias_parts.data_ptr()),
+                                  _stream_handle(stream))
+    if st != TRI_ATTN_OK:
+        raise TriAttnError(st, "tri_attn_bwd_rows")
+
+
+def tri_attn_dbias_sum(parts, dbias, stream=None) -> None:
+    """dbias (BF16 [B,H,N,N]) = sum over the first axis of parts (contiguous float32
+    [P,B,H,N,N]), added in ascending index order."""
+    import torch
+    if parts.dtype != torch.float32 or not parts.is_contiguous() or parts.dim() != 5:
+        raise TriAttnError(TRI_ATTN_ERR_SHAPE, "parts must be a contiguous float32 [P,B,H,N,N] tensor")
+    P, B, H, N, N2 = parts.shape
+    if N2 != N or tuple(dbias.shape) != (B, H, N, N):
+        raise TriAttnError(TRI_ATTN_ERR_SHAPE, "dbias must be [B,H,N,N] matching parts")
+    st = load().tri_attn_dbias_sum(ctypes.c_void_p(parts.data_ptr()), P, B, H, N, t4(dbias, "dbias"),
+                                   _stream_handle(stream))
+    if st != TRI_ATTN_OK:
+        raise TriAttnError(st, "tri_attn_dbias_sum")
 
 
 TRI_MUL_INCOMING = 1

@@ -179,8 +179,9 @@ bool encode_map(CUtensorMap* m, void* ptr, uint64_t inner, uint32_t inner_box, c
 }
 
 // Pair tensor [B,N,N,H,d] map: coordinates (c, h, j, i, b), box d x 1 x 128 x 1 x 1.
-bool map_pair(CUtensorMap* m, const tri_attn_tensor5& t, int B, int N, int H, int d) {
-    const uint64_t size[4] = {static_cast<uint64_t>(H), static_cast<uint64_t>(N), static_cast<uint64_t>(N),
+// R: the rows i the map covers (N, or a row shard); the j extent is always N
+bool map_pair(CUtensorMap* m, const tri_attn_tensor5& t, int B, int R, int N, int H, int d) {
+    const uint64_t size[4] = {static_cast<uint64_t>(H), static_cast<uint64_t>(N), static_cast<uint64_t>(R),
                               static_cast<uint64_t>(B)};
     const uint64_t st[4] = {static_cast<uint64_t>(t.stride[3]) * 2, static_cast<uint64_t>(t.stride[2]) * 2,
                             static_cast<uint64_t>(t.stride[1]) * 2, static_cast<uint64_t>(t.stride[0]) * 2};
@@ -270,20 +271,21 @@ bool bwd_set_attributes() {
     return ok;
 }
 
-tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, float scale, uint64_t wait_ns,
-                           cudaStream_t stream, void* const* markers) {
+tri_attn_status bwd_launch(const tri_attn_bwd_args* a, int R, float* parts, const BwdWorkspace& ws, float scale,
+                           uint64_t wait_ns, cudaStream_t stream, void* const* markers) {
     auto mark = [&](int m) {
         if (markers && markers[m]) cudaEventRecord(static_cast<cudaEvent_t>(markers[m]), stream);
     };
     const tri_attn_fwd_args& f = a->f;
     const int B = f.B, N = f.N, H = f.H, d = f.d;
     CUtensorMap mq, mk, mv, mdo;
-    if (!map_pair(&mq, f.q, B, N, H, d) || !map_pair(&mk, f.k, B, N, H, d) || !map_pair(&mv, f.v, B, N, H, d) ||
-        !map_pair(&mdo, a->dout, B, N, H, d))
+    if (!map_pair(&mq, f.q, B, R, N, H, d) || !map_pair(&mk, f.k, B, R, N, H, d) ||
+        !map_pair(&mv, f.v, B, R, N, H, d) || !map_pair(&mdo, a->dout, B, R, N, H, d))
         return TRI_ATTN_ERR_STRIDE;
     uint8_t* wsb = static_cast<uint8_t*>(a->workspace);
     BwdParams p{};
     p.B = B; p.N = N; p.H = H;
+    p.R = R;
     p.nt = (N + 127) / 128;
     p.Np = ws.Np;
     p.dq_tmem = (256 + 2 * d + p.nt * d <= 512) ? 1 : 0;
@@ -296,7 +298,8 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, f
     p.bias = static_cast<const __nv_bfloat16*>(f.bias.ptr);
     p.bs0 = f.bias.stride[0]; p.bs1 = f.bias.stride[1]; p.bs2 = f.bias.stride[2];
     p.dq_slots = reinterpret_cast<float*>(wsb + ws.off_dq);
-    p.part = reinterpret_cast<float*>(wsb + ws.off_part);
+    p.part = parts ? parts : reinterpret_cast<float*>(wsb + ws.off_part);
+    p.part_out = parts ? 1 : 0;
     p.chunks = ws.chunks;
     p.dq = static_cast<__nv_bfloat16*>(a->dq.ptr);
     p.dk = static_cast<__nv_bfloat16*>(a->dk.ptr);
@@ -307,8 +310,8 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, f
     p.wait_limit_ns = wait_ns;
 
     const int64_t rows = static_cast<int64_t>(B) * H * N * N;
-    const int64_t prep_items = static_cast<int64_t>(B) * H * N * ws.Np + static_cast<int64_t>(B) * N * ws.Np +
-                               static_cast<int64_t>(B) * N * 32;
+    const int64_t prep_items = static_cast<int64_t>(B) * H * R * ws.Np + static_cast<int64_t>(B) * R * ws.Np +
+                               static_cast<int64_t>(B) * R * 32;
     const unsigned prep_grid = static_cast<unsigned>(std::min<int64_t>((prep_items + 255) / 256, 148 * 16));
     const auto& sm = f.mask.stride;
     const int use_resid = (a->flags & TRI_ATTN_BWD_NO_RESIDUAL) ? 0 : 1;
@@ -321,7 +324,7 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, f
             static_cast<const __nv_bfloat16*>(a->dout.ptr), sd[0], sd[1], sd[2], sd[3],
             static_cast<const __nv_bfloat16*>(f.o.ptr), so[0], so[1], so[2], so[3],
             static_cast<const __nv_bfloat16*>(f.resid.ptr), sr[0], sr[1], sr[2], sr[3], use_resid, f.lse, f.mask.ptr,
-            sm[0], sm[1], sm[2], Dv, Lv, Mv, Fv, B, N, H, ws.Np, p.nt);
+            sm[0], sm[1], sm[2], Dv, Lv, Mv, Fv, B, N, R, H, ws.Np, p.nt);
         mark(1);
         tri_attn_bwd_main_kernel<32><<<ws.grid_main, MainLayout<32>::THREADS, MainLayout<32>::SMEM, stream>>>(mq, mk, mv, mdo, p);
         mark(2);
@@ -332,14 +335,14 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, f
             static_cast<const __nv_bfloat16*>(a->dout.ptr), sd[0], sd[1], sd[2], sd[3],
             static_cast<const __nv_bfloat16*>(f.o.ptr), so[0], so[1], so[2], so[3],
             static_cast<const __nv_bfloat16*>(f.resid.ptr), sr[0], sr[1], sr[2], sr[3], use_resid, f.lse, f.mask.ptr,
-            sm[0], sm[1], sm[2], Dv, Lv, Mv, Fv, B, N, H, ws.Np, p.nt);
+            sm[0], sm[1], sm[2], Dv, Lv, Mv, Fv, B, N, R, H, ws.Np, p.nt);
         mark(1);
         tri_attn_bwd_main_kernel<64><<<ws.grid_main, MainLayout<64>::THREADS, MainLayout<64>::SMEM, stream>>>(mq, mk, mv, mdo, p);
         mark(2);
         tri_attn_bwd_dbias_kernel<64><<<db_grid, DbLayout<64>::THREADS, DbLayout<64>::SMEM, stream>>>(
             mq, mk, mv, mdo, bias, f.bias.stride[0], f.bias.stride[1], f.bias.stride[2], p);
     }
-    if (ws.chunks > 1) {
+    if (ws.chunks > 1 && !parts) {
         const unsigned rg = static_cast<unsigned>(std::min<int64_t>((rows + 255) / 256, 148 * 16));
         tri_attn_bwd_dbias_reduce_kernel<<<rg, 256, 0, stream>>>(p.part, ws.chunks, B, H, N, p.dbias,
                                                                   a->dbias.stride[0], a->dbias.stride[1],
@@ -383,19 +386,26 @@ const char* tri_attn_strerror(tri_attn_status s) {
 
 void tri_attn_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns ? ns : 1); }
 
-tri_attn_status tri_attn_fwd(const tri_attn_fwd_args* a, tri_attn_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// the forward over rows 0 .. R-1 of the given tensors (R = N: the whole problem)
+tri_attn_status fwd_impl(const tri_attn_fwd_args* a, int R, tri_attn_stream_t stream) {
     tri_attn_status st = check_fwd_args(a);
     if (st) return st;
+    if (R < 1 || R > a->N) return TRI_ATTN_ERR_SHAPE;
     if ((st = ensure_device())) return st;
     const int B = a->B, N = a->N, H = a->H, d = a->d;
     CUtensorMap mq, mk, mv, mb;
-    if (!map_pair(&mq, a->q, B, N, H, d) || !map_pair(&mk, a->k, B, N, H, d) || !map_pair(&mv, a->v, B, N, H, d) ||
-        !map_bias(&mb, a->bias, B, N, H))
+    if (!map_pair(&mq, a->q, B, R, N, H, d) || !map_pair(&mk, a->k, B, R, N, H, d) ||
+        !map_pair(&mv, a->v, B, R, N, H, d) || !map_bias(&mb, a->bias, B, N, H))
         return TRI_ATTN_ERR_STRIDE;
     tri::FwdParams p{};
     p.B = B; p.N = N; p.H = H;
+    p.R = R;
     p.nt = (N + 127) / 128;
-    p.npairs = (N + 1) / 2;
+    p.npairs = (R + 1) / 2;
     p.scale = eff_scale(a->scale, d);
     p.mask = a->mask.ptr;
     p.ms0 = a->mask.stride[0]; p.ms1 = a->mask.stride[1]; p.ms2 = a->mask.stride[2];
@@ -415,30 +425,87 @@ tri_attn_status tri_attn_fwd(const tri_attn_fwd_args* a, tri_attn_stream_t strea
     return cudaGetLastError() == cudaSuccess ? TRI_ATTN_OK : TRI_ATTN_ERR_CUDA;
 }
 
-size_t tri_attn_bwd_workspace_bytes(int B, int N, int H, int d) {
-    if (check_sizes(B, N, H, d)) return 0;
-    return tri::bwd_workspace_layout(B, N, H, d).total;
-}
-
-tri_attn_status tri_attn_bwd(const tri_attn_bwd_args* a, tri_attn_stream_t stream) {
-    return tri_attn_bwd_marked(a, stream, nullptr);
-}
-
-tri_attn_status tri_attn_bwd_marked(const tri_attn_bwd_args* a, tri_attn_stream_t stream, void* const* markers) {
+// the backward over rows 0 .. R-1; parts == nullptr: dBias (BF16) for those rows
+// as the whole sum over i; otherwise dBias leaves as FP32 partial sums in parts
+tri_attn_status bwd_impl(const tri_attn_bwd_args* a, int R, float* parts, tri_attn_stream_t stream,
+                         void* const* markers) {
     if (!a) return TRI_ATTN_ERR_NULL;
     tri_attn_status st = check_fwd_args(&a->f);
     if (st) return st;
+    if (R < 1 || R > a->f.N) return TRI_ATTN_ERR_SHAPE;
     const tri_attn_tensor5* t5[] = {&a->dout, &a->dq, &a->dk, &a->dv};
     for (const auto* t : t5)
         if ((st = check_t5(*t))) return st;
-    if ((st = check_t4(a->dbias))) return st;
+    if (parts) {
+        if (!aligned16(parts)) return TRI_ATTN_ERR_ALIGN;
+    } else if ((st = check_t4(a->dbias))) {
+        return st;
+    }
     const int B = a->f.B, N = a->f.N, H = a->f.H, d = a->f.d;
-    const tri::BwdWorkspace ws = tri::bwd_workspace_layout(B, N, H, d);
-    if (!a->workspace || a->workspace_bytes < ws.total) return TRI_ATTN_ERR_WORKSPACE;
+    const tri::BwdWorkspace ws = tri::bwd_workspace_layout(B, R, N, H, d);
+    const size_t need = parts ? ws.off_part : ws.total;  // shard calls keep no partials of their own
+    if (!a->workspace || a->workspace_bytes < need) return TRI_ATTN_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(a->workspace) & 255u) return TRI_ATTN_ERR_ALIGN;
     if ((st = ensure_device())) return st;
-    return tri::bwd_launch(a, ws, eff_scale(a->f.scale, d), g_wait_limit_ns.load(),
+    return tri::bwd_launch(a, R, parts, ws, eff_scale(a->f.scale, d), g_wait_limit_ns.load(),
                            reinterpret_cast<cudaStream_t>(stream), markers);
+}
+
+}  // namespace
+
+extern "C" {
+
+tri_attn_status tri_attn_fwd(const tri_attn_fwd_args* a, tri_attn_stream_t stream) {
+    return fwd_impl(a, a ? a->N : 0, stream);
+}
+
+tri_attn_status tri_attn_fwd_rows(const tri_attn_fwd_args* a, int rows, tri_attn_stream_t stream) {
+    return fwd_impl(a, rows, stream);
+}
+
+size_t tri_attn_bwd_workspace_bytes(int B, int N, int H, int d) {
+    if (check_sizes(B, N, H, d)) return 0;
+    return tri::bwd_workspace_layout(B, N, N, H, d).total;
+}
+
+size_t tri_attn_bwd_rows_workspace_bytes(int B, int rows, int N, int H, int d) {
+    if (check_sizes(B, N, H, d) || rows < 1 || rows > N) return 0;
+    return tri::bwd_workspace_layout(B, rows, N, H, d).off_part;
+}
+
+int tri_attn_bwd_rows_dbias_parts(int B, int rows, int N, int H, int d) {
+    if (check_sizes(B, N, H, d) || rows < 1 || rows > N) return 0;
+    return tri::bwd_workspace_layout(B, rows, N, H, d).chunks;
+}
+
+tri_attn_status tri_attn_bwd(const tri_attn_bwd_args* a, tri_attn_stream_t stream) {
+    return bwd_impl(a, a ? a->f.N : 0, nullptr, stream, nullptr);
+}
+
+tri_attn_status tri_attn_bwd_marked(const tri_attn_bwd_args* a, tri_attn_stream_t stream, void* const* markers) {
+    return bwd_impl(a, a ? a->f.N : 0, nullptr, stream, markers);
+}
+
+tri_attn_status tri_attn_bwd_rows(const tri_attn_bwd_args* a, int rows, float* dbias_parts,
+                                  tri_attn_stream_t stream) {
+    if (!dbias_parts) return TRI_ATTN_ERR_NULL;
+    return bwd_impl(a, rows, dbias_parts, stream, nullptr);
+}
+
+tri_attn_status tri_attn_dbias_sum(const float* parts, int nparts, int B, int H, int N, tri_attn_tensor4 dbias,
+                                   tri_attn_stream_t stream) {
+    if (!parts) return TRI_ATTN_ERR_NULL;
+    if (!aligned16(parts)) return TRI_ATTN_ERR_ALIGN;
+    if (nparts < 1 || B < 1 || H < 1 || N < 1 || N > kMaxN) return TRI_ATTN_ERR_SHAPE;
+    tri_attn_status st = check_t4(dbias);
+    if (st) return st;
+    if ((st = ensure_device())) return st;
+    const int64_t total = static_cast<int64_t>(B) * H * N * N;
+    const unsigned rg = static_cast<unsigned>(std::min<int64_t>((total + 255) / 256, 148 * 16));
+    tri::tri_attn_bwd_dbias_reduce_kernel<<<rg, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        parts, nparts, B, H, N, static_cast<__nv_bfloat16*>(dbias.ptr), dbias.stride[0], dbias.stride[1],
+        dbias.stride[2]);
+    return cudaGetLastError() == cudaSuccess ? TRI_ATTN_OK : TRI_ATTN_ERR_CUDA;
 }
 
 tri_attn_status tri_mul_fwd(const tri_mul_fwd_args* a, tri_attn_stream_t stream) {

@@ -50,7 +50,8 @@ struct BwdWorkspace {
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-inline BwdWorkspace bwd_workspace_layout(int B, int N, int H, int d) {
+// R: rows i the launch covers (N for the whole problem, fewer for a row shard)
+inline BwdWorkspace bwd_workspace_layout(int B, int R, int N, int H, int d) {
     BwdWorkspace w{};
     const size_t nt = (N + 127) / 128;
     const size_t tiles = static_cast<size_t>(B) * H * nt * nt;
@@ -58,20 +59,20 @@ inline BwdWorkspace bwd_workspace_layout(int B, int N, int H, int d) {
     if (tiles < static_cast<size_t>(kChunkTarget)) {
         chunks = static_cast<int>(kChunkTarget / tiles);
         chunks = chunks < 1 ? 1 : chunks;
-        const int max_chunks = (N + 7) / 8;  // at least 8 rows per chunk
+        const int max_chunks = (R + 7) / 8;  // at least 8 rows per chunk
         chunks = chunks > max_chunks ? max_chunks : chunks;
     }
     w.chunks = chunks;
     w.Np = static_cast<int>(nt * 128);
-    const size_t problems = static_cast<size_t>(B) * N * H;
+    const size_t problems = static_cast<size_t>(B) * R * H;
     w.grid_main = static_cast<int>(problems < static_cast<size_t>(kDqSlots) ? problems : kDqSlots);
-    const size_t bhnp = static_cast<size_t>(B) * H * N * w.Np;
-    const size_t bnp = static_cast<size_t>(B) * N * w.Np;
+    const size_t bhnp = static_cast<size_t>(B) * H * R * w.Np;
+    const size_t bnp = static_cast<size_t>(B) * R * w.Np;
     w.off_D = 0;
     w.off_L = align256(bhnp * 4);
     w.off_M = w.off_L + align256(bhnp * 4);
     w.off_F = w.off_M + align256(bnp * 4);
-    w.off_dq = w.off_F + align256(static_cast<size_t>(B) * N * 32 * 4);
+    w.off_dq = w.off_F + align256(static_cast<size_t>(B) * R * 32 * 4);
     w.off_part = w.off_dq + align256(static_cast<size_t>(kDqSlots) * N * d * 4);
     const size_t bhnn = static_cast<size_t>(B) * H * N * N;
     w.total = w.off_part + (chunks > 1 ? align256(static_cast<size_t>(chunks) * bhnn * 4) : 0);
@@ -80,17 +81,19 @@ inline BwdWorkspace bwd_workspace_layout(int B, int N, int H, int d) {
 
 struct BwdParams {
     int B, N, H, nt, Np;
+    int R;            // rows i this launch covers (N, or a shard of the rows)
     float scale;
-    const float* Lv;  // [B,H,N,Np] lse * log2(e); +inf past N
-    const float* Dv;  // [B,H,N,Np] D; 0 past N
-    const float* Mv;  // [B,N,Np]   mask * log2(e); -inf past N
-    const int* Fv;    // [B,N,32]   1 where a key tile needs the mask add
+    const float* Lv;  // [B,H,R,Np] lse * log2(e); +inf past N
+    const float* Dv;  // [B,H,R,Np] D; 0 past N
+    const float* Mv;  // [B,R,Np]   mask * log2(e); -inf past N
+    const int* Fv;    // [B,R,32]   1 where a key tile needs the mask add
     const __nv_bfloat16* bias;  // [B,H,N,N] (read directly by the softmax warps of the main kernel)
     int64_t bs0, bs1, bs2;
     float* dq_slots;  // [kDqSlots][N][d] (used when dq_tmem == 0)
     int dq_tmem;      // 1: dQ for every query tile stays in TMEM across key tiles
-    float* part;      // [chunks][B,H,N,N] (chunks > 1)
+    float* part;      // [chunks][B,H,N,N] (chunks > 1, or always when part_out)
     int chunks;
+    int part_out;     // 1: dBias leaves as FP32 partial sums in part, never as BF16
     __nv_bfloat16 *dq, *dk, *dv, *dbias;
     int64_t dqs[5], dks[5], dvs[5], dbs[4];
     uint64_t wait_limit_ns;
@@ -112,11 +115,11 @@ __global__ void __launch_bounds__(256) tri_attn_bwd_prep_kernel(
     const __nv_bfloat16* __restrict__ r, int64_t r0, int64_t r1, int64_t r2, int64_t r3, int use_resid,
     const float* __restrict__ lse, const float* __restrict__ mask, int64_t m0, int64_t m1, int64_t m2,
     float* __restrict__ Dv, float* __restrict__ Lv, float* __restrict__ Mv, int* __restrict__ Fv, int B, int N,
-    int H, int Np, int nt) {
+    int R, int H, int Np, int nt) {
     constexpr float LOG2E = 1.4426950408889634f;
-    const int64_t n1 = static_cast<int64_t>(B) * H * N * Np;
-    const int64_t n2 = static_cast<int64_t>(B) * N * Np;
-    const int64_t n3 = static_cast<int64_t>(B) * N * 32;
+    const int64_t n1 = static_cast<int64_t>(B) * H * R * Np;
+    const int64_t n2 = static_cast<int64_t>(B) * R * Np;
+    const int64_t n3 = static_cast<int64_t>(B) * R * 32;
     for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < n1 + n2 + n3;
          idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         if (idx < n1) {
@@ -127,9 +130,9 @@ __global__ void __launch_bounds__(256) tri_attn_bwd_prep_kernel(
             t /= H;
             const int j = static_cast<int>(t % Np);
             t /= Np;
-            const int i = static_cast<int>(t % N);
-            const int b = static_cast<int>(t / N);
-            const int64_t out = ((static_cast<int64_t>(b) * H + h) * N + i) * Np + j;
+            const int i = static_cast<int>(t % R);
+            const int b = static_cast<int>(t / R);
+            const int64_t out = ((static_cast<int64_t>(b) * H + h) * R + i) * Np + j;
             float dsum = 0.f, lv = INFINITY;
             if (j < N) {
                 const uint4* pd = reinterpret_cast<const uint4*>(dout + b * s0 + i * s1 + j * s2 + h * s3);
@@ -148,7 +151,7 @@ __global__ void __launch_bounds__(256) tri_attn_bwd_prep_kernel(
                         dsum = fmaf(bf16hi(aw[e]), bf16hi(ow[e]) + bf16hi(rw[e]), dsum);
                     }
                 }
-                lv = __ldg(lse + ((static_cast<int64_t>(b) * H + h) * N + i) * N + j) * LOG2E;
+                lv = __ldg(lse + ((static_cast<int64_t>(b) * H + h) * R + i) * N + j) * LOG2E;
             }
             Dv[out] = dsum;
             Lv[out] = lv;
@@ -156,8 +159,8 @@ __global__ void __launch_bounds__(256) tri_attn_bwd_prep_kernel(
             const int64_t e = idx - n1;
             const int k = static_cast<int>(e % Np);
             const int64_t t = e / Np;
-            const int i = static_cast<int>(t % N);
-            const int b = static_cast<int>(t / N);
+            const int i = static_cast<int>(t % R);
+            const int b = static_cast<int>(t / R);
             float mv = -INFINITY;
             if (k < N) mv = mask ? __ldg(mask + b * m0 + i * m1 + k * m2) * LOG2E : 0.f;
             Mv[e] = mv;
@@ -165,8 +168,8 @@ __global__ void __launch_bounds__(256) tri_attn_bwd_prep_kernel(
             const int64_t e = idx - n1 - n2;
             const int kt = static_cast<int>(e % 32);
             const int64_t t = e / 32;
-            const int i = static_cast<int>(t % N);
-            const int b = static_cast<int>(t / N);
+            const int i = static_cast<int>(t % R);
+            const int b = static_cast<int>(t / R);
             int f = 0;
             if (kt < nt) {
                 if ((kt + 1) * 128 > N) f = 1;  // padded keys need the -inf
@@ -230,11 +233,11 @@ __global__ void __launch_bounds__(640, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
     const int nt = p.nt;
-    const int problems = p.B * p.N * p.H;
+    const int problems = p.B * p.R * p.H;
     // problem index -> (b, h, i) with i fastest so concurrent CTAs share a head's bias
     auto decode = [&](int pr, int& b, int& h, int& i) {
-        i = pr % p.N;
-        const int t = pr / p.N;
+        i = pr % p.R;
+        const int t = pr / p.R;
         h = t % p.H;
         b = t / p.H;
     };
@@ -302,9 +305,9 @@ __global__ void __launch_bounds__(640, 1)
                 auto load_pair = [&](uint32_t dst, const CUtensorMap* m, uint32_t bar, int row0) {
                     tma_load_5d(dst, m, bar, 0, h, row0, i, b);
                 };
-                const float* mrow = p.Mv + (static_cast<int64_t>(b) * p.N + i) * p.Np;
-                const int* frow = p.Fv + (static_cast<int64_t>(b) * p.N + i) * 32;
-                const int64_t vrow = ((static_cast<int64_t>(b) * p.H + h) * p.N + i) * p.Np;
+                const float* mrow = p.Mv + (static_cast<int64_t>(b) * p.R + i) * p.Np;
+                const int* frow = p.Fv + (static_cast<int64_t>(b) * p.R + i) * 32;
+                const int64_t vrow = ((static_cast<int64_t>(b) * p.H + h) * p.R + i) * p.Np;
                 for (int kt = 0; ok && kt < nt; ++kt) {
                     const int ks = gk % L::KVS;
                     if (gk >= L::KVS && !mbar_wait_warp(BAR(L::B_KVEMPTY + ks), ((gk / L::KVS) - 1) & 1, wc, 1)) {
@@ -786,9 +789,9 @@ __global__ void __launch_bounds__(640, 1)
     item /= nt;
     const int h = item % p.H;
     const int b = item / p.H;
-    const int rows_per = (p.N + p.chunks - 1) / p.chunks;
+    const int rows_per = (p.R + p.chunks - 1) / p.chunks;
     const int i_begin = chunk * rows_per;
-    const int i_end = min(p.N, i_begin + rows_per);
+    const int i_end = min(p.R, i_begin + rows_per);
     const int nrows = max(0, i_end - i_begin);
 
     if (threadIdx.x == 0) {
@@ -841,8 +844,8 @@ __global__ void __launch_bounds__(640, 1)
                     const uint32_t bar = BAR(L::B_FULL + s);
                     const uint32_t base = sb + s * L::STAGE;
                     const uint32_t vec = sb + L::OFF_VEC + s * L::VEC;
-                    const int64_t vrow = ((static_cast<int64_t>(b) * p.H + h) * p.N + i) * p.Np + jt * 128;
-                    const int64_t mrow = (static_cast<int64_t>(b) * p.N + i) * p.Np + kt * 128;
+                    const int64_t vrow = ((static_cast<int64_t>(b) * p.H + h) * p.R + i) * p.Np + jt * 128;
+                    const int64_t mrow = (static_cast<int64_t>(b) * p.R + i) * p.Np + kt * 128;
                     mbar_arrive_expect_tx(bar, L::STAGE + L::VEC);
                     auto ld = [&](uint32_t dst, const CUtensorMap* m, int row0) {
                         tma_load_5d(dst, m, bar, 0, h, row0, i, b);
@@ -854,7 +857,7 @@ __global__ void __launch_bounds__(640, 1)
                     bulk_load(vec, p.Lv + vrow, 512, bar);
                     bulk_load(vec + 512, p.Dv + vrow, 512, bar);
                     bulk_load(vec + 1024, p.Mv + mrow, 512, bar);
-                    bulk_load(vec + 1536, p.Fv + (static_cast<int64_t>(b) * p.N + i) * 32, 128, bar);
+                    bulk_load(vec + 1536, p.Fv + (static_cast<int64_t>(b) * p.R + i) * 32, 128, bar);
                 }
                 armed[s]++;
             }
@@ -1001,7 +1004,7 @@ __global__ void __launch_bounds__(640, 1)
         TRI_TP(3)
         if (ok && j < p.N) {
             const int k0 = kt * 128 + w * 32;
-            if (p.chunks == 1) {
+            if (p.chunks == 1 && !p.part_out) {
                 __nv_bfloat16* dst = p.dbias + b * p.dbs[0] + h * p.dbs[1] + static_cast<int64_t>(j) * p.dbs[2] + k0;
 #pragma unroll
                 for (int e = 0; e < 32; e += 8) {
@@ -1039,11 +1042,13 @@ __global__ void __launch_bounds__(640, 1)
     }
 }
 
-// ascending-chunk sum of the dBias partials -> BF16
+// ascending-index sum of dBias partials (the chunks of one launch, or the chunks of
+// every row shard in rank order) -> BF16
 __global__ void __launch_bounds__(256) tri_attn_bwd_dbias_reduce_kernel(const float* __restrict__ part, int chunks,
                                                                         int B, int H, int N,
                                                                         __nv_bfloat16* __restrict__ dbias,
                                                                         int64_t s0, int64_t s1, int64_t s2) {
+    if (device_error_pending()) return;
     const int64_t total = static_cast<int64_t>(B) * H * N * N;
     for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
          idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -1064,7 +1069,8 @@ __global__ void __launch_bounds__(256) tri_attn_bwd_dbias_reduce_kernel(const fl
 // host side
 // ===========================================================================
 bool bwd_set_attributes();
-tri_attn_status bwd_launch(const tri_attn_bwd_args* a, const BwdWorkspace& ws, float scale, uint64_t wait_ns,
-                           cudaStream_t stream, void* const* markers);
+// R: rows i covered; parts: NULL, or where dBias goes as FP32 partial sums
+tri_attn_status bwd_launch(const tri_attn_bwd_args* a, int R, float* parts, const BwdWorkspace& ws, float scale,
+                           uint64_t wait_ns, cudaStream_t stream, void* const* markers);
 
 }  // namespace tri

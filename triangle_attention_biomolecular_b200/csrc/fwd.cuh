@@ -37,6 +37,7 @@ namespace tri {
 
 struct FwdParams {
     int B, N, H, nt, npairs;
+    int R;  // rows i this launch covers (N, or a shard of the rows)
     float scale;
     const float* mask;
     int64_t ms0, ms1, ms2;
@@ -119,8 +120,8 @@ __global__ void __launch_bounds__(384, 1)
         t.h = item % p.H;
         t.b = item / p.H;
         t.i0 = 2 * ip;
-        t.i1 = min(2 * ip + 1, p.N - 1);
-        t.has1 = (2 * ip + 1) < p.N;
+        t.i1 = min(2 * ip + 1, p.R - 1);
+        t.has1 = (2 * ip + 1) < p.R;
         return t;
     };
     const int items = p.B * p.npairs * p.H * p.nt;
@@ -557,7 +558,7 @@ __global__ void __launch_bounds__(384, 1)
                 }
             }
             if (store) {
-                p.lse[((static_cast<int64_t>(b) * p.H + h) * p.N + i) * p.N + j] =
+                p.lse[((static_cast<int64_t>(b) * p.H + h) * p.R + i) * p.N + j] =
                     m_ref + lg2(l) * 0.6931471805599453f;
             }
         }
