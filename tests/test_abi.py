@@ -24,12 +24,14 @@ def lib():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(tri_attn_[a-z0-9_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(tri_(?:attn|mul|gate)_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_functions()
-    assert "tri_attn_fwd" in names and "tri_attn_bwd" in names
+    for n in ("tri_attn_fwd", "tri_attn_bwd", "tri_attn_fwd_rows", "tri_attn_dbias_sum", "tri_mul_fwd",
+              "tri_gate_bwd"):
+        assert n in names
     for n in names:
         assert hasattr(lib, n), f"missing export {n}"
 
@@ -41,7 +43,7 @@ def test_library_does_not_link_the_driver():
 
 def test_strerror_covers_every_status(lib):
     seen = set()
-    for code in range(11):
+    for code in range(12):
         s = B.tri_attn_strerror(code)
         assert s and s not in seen
         seen.add(s)
@@ -152,6 +154,39 @@ def test_valid_arguments_without_a_device_report_cuda_error(lib):
     assert lib.tri_attn_bwd(ctypes.byref(a), None) in (B.TRI_ATTN_ERR_CUDA, B.TRI_ATTN_ERR_ARCH)
 
 
+def test_row_shard_validation_codes(lib):
+    a = _fake_args()
+    assert lib.tri_attn_fwd_rows(ctypes.byref(a), 0, None) == B.TRI_ATTN_ERR_SHAPE
+    assert lib.tri_attn_fwd_rows(ctypes.byref(a), 65, None) == B.TRI_ATTN_ERR_SHAPE  # more rows than N
+    assert lib.tri_attn_fwd_rows(None, 8, None) == B.TRI_ATTN_ERR_NULL
+    # sizes: a block needs no more workspace than the whole problem, and P partials >= 1
+    whole = lib.tri_attn_bwd_workspace_bytes(1, 64, 2, 32)
+    for rows in (1, 7, 32, 64):
+        assert 0 < lib.tri_attn_bwd_rows_workspace_bytes(1, rows, 64, 2, 32) <= whole
+        assert lib.tri_attn_bwd_rows_dbias_parts(1, rows, 64, 2, 32) >= 1
+    assert lib.tri_attn_bwd_rows_workspace_bytes(1, 0, 64, 2, 32) == 0
+    assert lib.tri_attn_bwd_rows_dbias_parts(1, 65, 64, 2, 32) == 0
+    assert lib.tri_attn_bwd_rows_dbias_parts(1, 64, 64, 2, 48) == 0
+    parts = 0x5000000
+    b = _bwd_args(lib)
+    b.dbias.ptr = None  # not used by a shard call
+    b.workspace_bytes = lib.tri_attn_bwd_rows_workspace_bytes(1, 32, 64, 2, 32)
+    assert lib.tri_attn_bwd_rows(ctypes.byref(b), 32, None, None) == B.TRI_ATTN_ERR_NULL
+    assert lib.tri_attn_bwd_rows(ctypes.byref(b), 32, ctypes.c_void_p(parts + 4), None) == B.TRI_ATTN_ERR_ALIGN
+    assert lib.tri_attn_bwd_rows(ctypes.byref(b), 0, ctypes.c_void_p(parts), None) == B.TRI_ATTN_ERR_SHAPE
+    b.workspace_bytes -= 256
+    assert lib.tri_attn_bwd_rows(ctypes.byref(b), 32, ctypes.c_void_p(parts), None) == B.TRI_ATTN_ERR_WORKSPACE
+    db = B.Tensor4()
+    db.ptr = 0x3000000
+    for x, st in enumerate((2 * 64 * 64, 64 * 64, 64, 1)):
+        db.stride[x] = st
+    assert lib.tri_attn_dbias_sum(None, 2, 1, 2, 64, db, None) == B.TRI_ATTN_ERR_NULL
+    assert lib.tri_attn_dbias_sum(ctypes.c_void_p(parts), 0, 1, 2, 64, db, None) == B.TRI_ATTN_ERR_SHAPE
+    assert lib.tri_attn_dbias_sum(ctypes.c_void_p(parts + 8), 2, 1, 2, 64, db, None) == B.TRI_ATTN_ERR_ALIGN
+    db.stride[2] = 60
+    assert lib.tri_attn_dbias_sum(ctypes.c_void_p(parts), 2, 1, 2, 64, db, None) == B.TRI_ATTN_ERR_STRIDE
+
+
 def test_binding_rejects_wrong_dtypes_before_the_library():
     q = torch.zeros(1, 8, 8, 2, 32, dtype=torch.float32)
     with pytest.raises(B.TriAttnError) as e:
@@ -171,6 +206,11 @@ int main(void){
   printf("%zu %zu %zu %zu %zu %zu\n", sizeof(tri_attn_fwd_args), offsetof(tri_attn_fwd_args, q),
          offsetof(tri_attn_fwd_args, lse), sizeof(tri_attn_bwd_args), offsetof(tri_attn_bwd_args, workspace),
          offsetof(tri_attn_bwd_args, flags));
+  printf("%zu %zu %zu %zu %zu %zu\n", sizeof(tri_mul_fwd_args), offsetof(tri_mul_fwd_args, flags),
+         sizeof(tri_mul_bwd_args), offsetof(tri_mul_bwd_args, db), sizeof(tri_gate_fwd_args),
+         offsetof(tri_gate_fwd_args, y_stride));
+  printf("%zu %zu %zu %zu\n", sizeof(tri_gate_bwd_args), offsetof(tri_gate_bwd_args, dy_stride),
+         offsetof(tri_gate_bwd_args, dwo), offsetof(tri_gate_bwd_args, workspace_bytes));
   return 0; }
 '''
     import subprocess
@@ -182,5 +222,9 @@ int main(void){
         subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), c, "-o", exe], check=True)
         got = list(map(int, subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split()))
     want = [ctypes.sizeof(B.FwdArgs), B.FwdArgs.q.offset, B.FwdArgs.lse.offset, ctypes.sizeof(B.BwdArgs),
-            B.BwdArgs.workspace.offset, B.BwdArgs.flags.offset]
+            B.BwdArgs.workspace.offset, B.BwdArgs.flags.offset,
+            ctypes.sizeof(B.MulFwdArgs), B.MulFwdArgs.flags.offset, ctypes.sizeof(B.MulBwdArgs),
+            B.MulBwdArgs.db.offset, ctypes.sizeof(B.GateFwdArgs), B.GateFwdArgs.y_stride.offset,
+            ctypes.sizeof(B.GateBwdArgs), B.GateBwdArgs.dy_stride.offset, B.GateBwdArgs.dwo.offset,
+            B.GateBwdArgs.workspace_bytes.offset]
     assert got == want
