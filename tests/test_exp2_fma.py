@@ -3,7 +3,9 @@ reduction to x = n + f with n = floor(x), a fitted cubic for 2^f on [0, 1), and
 n added into the exponent field.  Checked here on the CPU, in float32 arithmetic,
 with the coefficients read from the source: the relative error bound the kernels
 rely on (far below the BF16 rounding of the probabilities they feed), the
-behaviour at integer arguments, and the clamp for very negative arguments."""
+behaviour at integer arguments, the clamp for very negative arguments, the large
+positive arguments the gated projection uses, and that projection's sigmoid and
+its complement (sigmoid2 in csrc/tri_gate.cuh)."""
 import os
 import re
 
@@ -69,3 +71,40 @@ def test_coefficients_are_near_the_taylor_series():
     c = coefficients().astype(np.float64)
     taylor = np.array([1.0, np.log(2), np.log(2) ** 2 / 2, np.log(2) ** 3 / 6])
     assert np.all(np.abs(c - taylor) < 0.03)
+
+
+def test_large_positive_arguments_up_to_the_gate_clamp():
+    # the gated projection evaluates 2^x for x = -G log2(e) clamped to <= 126: n is added
+    # into the exponent field, which must not carry into the sign bit anywhere up to 126
+    x = np.concatenate([np.linspace(8, 126, 100001), np.arange(8, 127)]).astype(np.float32)
+    got = ex2_fma(x).astype(np.float64)
+    ref = np.exp2(x.astype(np.float64))
+    assert np.all(np.isfinite(got)) and np.all(got > 0)
+    assert (np.abs(got - ref) / ref).max() < 2e-4
+
+
+def sigmoid2(x):
+    """The gate's g = 1 / (1 + e) and h = 1 - g = e g with e = 2^(-x log2 e) from the
+    FMA-pipe exp2 (argument clamped to [-125, 126]); the hardware reciprocal is taken
+    as the correctly rounded float32 one here."""
+    a = np.minimum(x.astype(np.float32) * np.float32(-1.4426950408889634), np.float32(126.0))
+    e = ex2_fma(a)
+    g = (np.float32(1.0) / (np.float32(1.0) + e)).astype(np.float32)
+    return g, (e * g).astype(np.float32)
+
+
+def test_gate_sigmoid_and_its_complement():
+    x = np.concatenate([np.linspace(-80, 80, 160001), [0.0]]).astype(np.float32)
+    g, h = sigmoid2(x)
+    x64 = x.astype(np.float64)
+    ref_g = 1.0 / (1.0 + np.exp(-x64))
+    ref_h = 1.0 / (1.0 + np.exp(x64))  # 1 - g without cancellation
+    assert (np.abs(g - ref_g) / ref_g).max() < 3e-4
+    assert (np.abs(h - ref_h) / ref_h).max() < 3e-4  # the complement keeps its relative accuracy
+    g0, h0 = sigmoid2(np.array([0.0], dtype=np.float32))
+    assert abs(g0[0] - 0.5) < 1e-4 and abs(h0[0] - 0.5) < 1e-4
+    # saturated logits: g rounds to 1 or to a tiny normal number, never to NaN or inf
+    gs, hs = sigmoid2(np.array([-1e4, -200.0, 200.0, 1e4], dtype=np.float32))
+    assert np.all(np.isfinite(gs)) and np.all(np.isfinite(hs))
+    assert gs[0] < 1e-37 and gs[1] < 1e-37 and gs[2] == 1.0 and gs[3] == 1.0
+    assert abs(hs[0] - 1.0) < 1e-6 and hs[3] < 1e-37
