@@ -493,7 +493,35 @@ def run_gate(args):
                          "unit": "GB/s", "frac": round(b_gbs / hbm, 4), "traffic": None,
                          "peak_source": f"{src} hbm_gbs"},
             "gpu_launches": 3 * args.steps, "clocks": clocks, "e2e": None}
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = gate_cpu_baseline()
     print(json.dumps(line), flush=True)
+
+
+def gate_cpu_baseline(target_s: float = 10.0):
+    """The FP64 oracle of the gated projection (forward + backward) on the host cores
+    over a bounded block of pair positions, in the bench's GB/s (8 x 128 x 2 bytes of
+    BF16 traffic per position)."""
+    import numpy as np
+    from oracle import tri_gate_oracle as G
+    rows = 16384
+    rng = np.random.default_rng(0)
+    z, o, dy = (rng.standard_normal((rows, 128)) for _ in range(3))
+    wg, wo = (rng.standard_normal((128, 128)) / np.sqrt(128) for _ in range(2))
+
+    def one():
+        t = time.perf_counter()
+        G.fwd(z, o, wg, wo)
+        G.bwd(z, o, wg, wo, dy)
+        return time.perf_counter() - t
+    one()
+    t1 = one()
+    n = int(max(1, min(36, round(target_s / max(t1, 1e-4)))))
+    t = sum(one() for _ in range(n))
+    return {"value": round(8 * 128 * 2 * rows * n / t / 1e9, 3), "unit": "GB/s", "cores": os.cpu_count(),
+            "kind": "oracle", "seconds": round(t, 3),
+            "sample": f"{n} blocks of {rows} of the 589,824 pair positions: FP64 oracle forward + backward "
+                      "(numpy matmul)"}
 
 
 def tri_mul_cpu_baseline(target_s: float = 10.0):

@@ -1,6 +1,6 @@
-"""The multi-rank plumbing of bench.py on CPU (gloo ranks, no GPU): the timed region
+"""Host-side parts of bench.py on CPU (gloo ranks, no GPU): the timed region
 is the slowest rank's, every rank receives it, the whole-job value counts every rank's
-steps, and the reference arm runs on rank 0 only."""
+steps, the reference arm runs on rank 0 only, and the oracle baselines run."""
 import argparse
 import os
 import socket
@@ -54,3 +54,9 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
     args = argparse.Namespace(steps=1, warmup=0, gpus=2, workload="crop768", op="attention")
     bench.run_reference(args, rank=1, world=2)
     assert capsys.readouterr().out == ""
+
+
+def test_gate_cpu_baseline_times_the_oracle():
+    line = bench.gate_cpu_baseline(target_s=0.2)
+    assert line["kind"] == "oracle" and line["unit"] == "GB/s"
+    assert line["value"] > 0 and line["cores"] >= 1 and line["seconds"] > 0
