@@ -160,6 +160,26 @@ def test_shards_match_the_whole_problem(N, world, d):
     assert torch.equal(again["dbias"], got["dbias"])  # fixed order: repeatable bit for bit
 
 
+@pytest.mark.gpu
+def test_crop768_two_shards_against_the_whole_problem():
+    # the headline size: one dBias partial per block (no row chunks); the whole problem's
+    # own dBias, already within the oracle gate (test_gpu_parity), is the reference
+    from triangle_attention_biomolecular_b200 import api
+    from triangle_attention_biomolecular_b200 import synthetic as S
+    x = S.make_inputs(S.CROP768, 41)
+    dev = torch.device("cuda")
+    got = run_shards(x, 2, dev)
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "dout"))
+    bias, mask = x["bias"].to(dev), x["mask"].to(dev)
+    o, r, lse = api.forward(q, k, v, bias, mask)
+    dq, dk, dv, db = api.backward(q, k, v, bias, mask, o, r, lse, do)
+    torch.cuda.synchronize()
+    for n, t in {"out": o, "resid": r, "lse": lse, "dq": dq, "dk": dk, "dv": dv}.items():
+        assert torch.equal(got[n], t), n
+    a, b = got["dbias"].double(), db.double()
+    assert float((a - b).norm() / b.norm()) < 2e-3  # two FP32 partials vs one sum: BF16-level differences
+
+
 def _nccl_one_rank(rank, port):
     import torch.distributed as dist
     from triangle_attention_biomolecular_b200 import _binding as Bd
