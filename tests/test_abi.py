@@ -228,3 +228,13 @@ int main(void){
             ctypes.sizeof(B.GateBwdArgs), B.GateBwdArgs.dy_stride.offset, B.GateBwdArgs.dwo.offset,
             B.GateBwdArgs.workspace_bytes.offset]
     assert got == want
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    # no fallback of any kind: without the built library every entry point raises
+    monkeypatch.setattr(B, "_lib", None)
+    monkeypatch.setattr(B, "LIB_PATH", str(tmp_path / "absent" / "libtriattn.so"))
+    for call in (lambda: B.tri_attn_bwd_workspace_bytes(1, 64, 2, 32), lambda: B.tri_gate_bwd_workspace_bytes(1),
+                 lambda: B.tri_attn_abi_version()):
+        with pytest.raises(RuntimeError, match="not found"):
+            call()
