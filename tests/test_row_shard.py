@@ -41,6 +41,35 @@ def test_row_range_partitions_the_rows(N):
         RS.row_range(N, 1, 1)
 
 
+def test_partial_slots_are_the_most_any_block_needs():
+    from triangle_attention_biomolecular_b200 import _binding as Bd
+    # N=80 over 9 ranks: blocks of 9 rows take two partials, the block of 8 takes one
+    per_rank = [Bd.tri_attn_bwd_rows_dbias_parts(1, RS.row_range(80, r, 9)[1], 80, 4, 32) for r in range(9)]
+    assert per_rank == [2] * 8 + [1]
+    assert RS.dbias_parts(1, 80, 4, 32, 9) == 2
+    assert RS.dbias_parts(1, 768, 4, 32, 2) == 1  # crop768: no row chunks
+
+
+def _wrong_parts_worker(rank, port):
+    import torch.distributed as dist
+    from triangle_attention_biomolecular_b200 import _binding as Bd
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=1)
+    try:
+        q = torch.zeros((1, 16, 16, 2, 32), dtype=torch.bfloat16)
+        parts = torch.zeros((5, 1, 2, 16, 16))  # the right count is 2
+        with pytest.raises(Bd.TriAttnError):
+            RS.shard_bwd(q, q, q, None, None, q, q, None, q, q, q, q, None, None, parts)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_shard_bwd_checks_the_partials_buffer_first():
+    import torch.multiprocessing as mp
+    mp.spawn(_wrong_parts_worker, args=(free_port(),), nprocs=1, join=True)
+
+
 def small_problem(seed=3, B=1, N=10, H=2, d=8):
     g = torch.Generator().manual_seed(seed)
     q, k, v, dout = (torch.randn((B, N, N, H, d), generator=g).to(torch.bfloat16) for _ in range(4))
