@@ -169,8 +169,10 @@ tri_attn_status tri_attn_bwd_marked(const tri_attn_bwd_args *args, tri_attn_stre
                                     void *const *markers);
 
 /* ---------------------------------------------------------------------------
- * Row shards (a 1-D split of the rows i across devices, as in Design-CP's
- * row-wise partitioning of the pair representation).  The problems of
+ * Row shards: a 1-D split of the rows i across devices, the row sharding of
+ * the pair representation in "Design-CP: Context Parallelism for Design of
+ * Protein Nanoparticles" (gist.science summary), section "方法论", item
+ * "1. 推理策略" (1D row sharding).  The problems of
  * different rows i are independent except for dBias, the sum over i of the
  * score gradient: each shard returns its share of that sum in FP32, and
  * tri_attn_dbias_sum adds the shares of all shards in a fixed order.

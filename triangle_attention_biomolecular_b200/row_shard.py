@@ -1,9 +1,12 @@
 """Row-sharded triangle attention across ranks (one process per GPU).
 
-The starting-node problems of different rows i are independent (Triton/TurboPairFormer
-pages, "cubic in N" discussion; the Design-CP page's row-wise 1-D partition of the pair
-representation): rank r owns a contiguous block of rows and runs the forward and the
-dq/dk/dv part of the backward on it alone.  The one exchange is dBias, the sum over all
+The starting-node problems of different rows i are independent: each is a softmax
+attention within row i, and only the pair bias is shared by all rows ("16张H100，训练步
+提速1.73倍：TurboPairFormer为什么不是‘装个包就能加速AlphaFold3’", section "它优化了什么，
+而不是只‘少存一点张量’", on the four gradients).  The partition is the 1-D row sharding of
+the pair representation in "Design-CP: Context Parallelism for Design of Protein
+Nanoparticles", section "方法论", item "1. 推理策略": rank r owns a contiguous block of
+rows and runs the forward and the dq/dk/dv part of the backward on it alone.  The one exchange is dBias, the sum over all
 rows i of the score gradient: every rank computes its block's share as FP32 partial
 sums (`tri_attn_bwd_rows`), the shares are all-gathered in rank order, and every rank
 adds the gathered array in ascending index order (`tri_attn_dbias_sum`), so all ranks
