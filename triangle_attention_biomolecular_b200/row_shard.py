@@ -6,11 +6,12 @@ attention within row i, and only the pair bias is shared by all rows ("16张H100
 而不是只‘少存一点张量’", on the four gradients).  The partition is the 1-D row sharding of
 the pair representation in "Design-CP: Context Parallelism for Design of Protein
 Nanoparticles", section "方法论", item "1. 推理策略": rank r owns a contiguous block of
-rows and runs the forward and the dq/dk/dv part of the backward on it alone.  The one exchange is dBias, the sum over all
-rows i of the score gradient: every rank computes its block's share as FP32 partial
-sums (`tri_attn_bwd_rows`), the shares are all-gathered in rank order, and every rank
-adds the gathered array in ascending index order (`tri_attn_dbias_sum`), so all ranks
-hold the same BF16 dBias bit for bit.
+rows and runs the forward and the dq/dk/dv part of the backward on it alone.
+
+The one exchange is dBias, the sum over all rows i of the score gradient: every rank
+computes its block's share as FP32 partial sums (`tri_attn_bwd_rows`), the shares are
+all-gathered in rank order, and every rank adds the gathered array in ascending index
+order (`tri_attn_dbias_sum`), so all ranks hold the same BF16 dBias bit for bit.
 
 The bias itself is an input replicated on every rank; the pair tensors, the mask, lse
 and the gradients of a rank are views of its own rows.
