@@ -226,13 +226,18 @@ tri_attn_status tri_attn_dbias_sum(const float *parts, int nparts, int B, int H,
  * in the library's own device memory, reserved when the library's module for
  * it is loaded onto a device; args->workspace and args->workspace_bytes are
  * ignored.
- *   - Limit: sizes whose tri_attn_bwd_workspace_bytes(B,N,H,d) exceeds
+ *   - Order of checks: the argument errors of tri_attn_bwd first (on the
+ *     host, before any CUDA call), then the limit: sizes whose
+ *     tri_attn_bwd_workspace_bytes(B,N,H,d) exceeds
  *     TRI_ATTN_STATIC_SCRATCH_BYTES are rejected with
  *     TRI_ATTN_ERR_SCRATCH_LIMIT before anything is enqueued.
  *   - Set-up: the first call on each device (the current device at the call)
  *     looks up the array's device address, which loads the module there; call
  *     it once on each device before any stream capture begins, so that this
- *     set-up happens outside a capture.
+ *     set-up happens outside a capture.  The address is kept per device
+ *     together with the CUDA context it belongs to; after a device reset (a
+ *     new context) the next call looks it up again, so that call is a set-up
+ *     call too.
  *   - Initial contents: nothing in the scratch has to start at zero; every
  *     word the kernels read is written earlier in the same call.
  *   - Races: all calls on one device share the one array.  Two calls whose

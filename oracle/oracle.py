@@ -72,7 +72,10 @@ def _load():
             lib.tri_attn_oracle_bwd_rows.argtypes = [i, i, i, i, d, dp, dp, dp, dp, dp, dp, ip, i,
                                                      dp, dp, dp, i]
             lib.tri_attn_oracle_dbias.argtypes = [i, i, i, i, d, dp, dp, dp, dp, dp, dp, ip, i, dp, i]
-            for f in (lib.tri_attn_oracle_fwd, lib.tri_attn_oracle_bwd_rows, lib.tri_attn_oracle_dbias):
+            lib.tri_attn_oracle_row.argtypes = [i, i, i, d, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp]
+            lib.tri_attn_oracle_dbias_row_add.argtypes = [i, i, i, d, dp, dp, dp, dp, dp, dp, i, i, dp]
+            for f in (lib.tri_attn_oracle_fwd, lib.tri_attn_oracle_bwd_rows, lib.tri_attn_oracle_dbias,
+                      lib.tri_attn_oracle_row, lib.tri_attn_oracle_dbias_row_add):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -173,6 +176,46 @@ def bwd(q, k, v, bias, mask, dout, scale=None, planted: int = 0):
     dq, dk, dv = bwd_rows(q, k, v, bias, mask, dout, scale, None, planted)
     db = dbias(q, k, v, bias, mask, dout, scale, None, planted)
     return dq, dk, dv, db
+
+
+# ---- one pair row at a time (crops whose pair stack is too large for FP64 on the host) ----
+
+def row(q_row, k_row, v_row, bias_b, mask_row=None, dout_row=None, scale=None):
+    """Pair row (b,i) alone: q_row, k_row, v_row, dout_row are that row's [N,H,d],
+    bias_b the batch's [H,N,N], mask_row its [N] (or None).  Returns out [N,H,d],
+    lse [H,N] and, with dout_row, dq, dk, dv [N,H,d] -- the same arithmetic as
+    ``fwd``/``bwd_rows`` on that row (equal bit for bit)."""
+    q_row, k_row, v_row, bias_b, mask_row, dout_row = map(_f64, (q_row, k_row, v_row, bias_b, mask_row, dout_row))
+    N, H, d = q_row.shape
+    assert k_row.shape == v_row.shape == (N, H, d) and bias_b.shape == (H, N, N)
+    scale = default_scale(d) if scale is None else float(scale)
+    out = np.full((N, H, d), np.nan)
+    lse = np.full((H, N), np.nan)
+    grads = dout_row is not None
+    dq, dk, dv = ((np.full((N, H, d), np.nan) for _ in range(3)) if grads else (None, None, None))
+    st = _load().tri_attn_oracle_row(N, H, d, scale, _ptr(q_row), _ptr(k_row), _ptr(v_row), _ptr(bias_b),
+                                     _ptr(mask_row), _ptr(dout_row), _ptr(out), _ptr(lse), _ptr(dq), _ptr(dk),
+                                     _ptr(dv))
+    _check(st)
+    return (out, lse, dq, dk, dv) if grads else (out, lse)
+
+
+def dbias_streamed(get_row, bias_b, h, j, scale=None):
+    """dbias[b,h,j,:] as the ascending sum over rows i of ds[b,i,j,h,:], fetching one
+    row at a time: ``get_row(i)`` returns (q_row, k_row, v_row, mask_row, dout_row)
+    of row i.  Same FP64 operations and order as ``dbias`` (equal bit for bit)."""
+    bias_b = _f64(bias_b)
+    H, N, _ = bias_b.shape
+    acc = np.zeros(N)
+    lib = _load()
+    for i in range(N):
+        q_row, k_row, v_row, mask_row, dout_row = map(_f64, get_row(i))
+        d = q_row.shape[2]
+        sc = default_scale(d) if scale is None else float(scale)
+        st = lib.tri_attn_oracle_dbias_row_add(N, H, d, sc, _ptr(q_row), _ptr(k_row), _ptr(v_row), _ptr(bias_b),
+                                               _ptr(mask_row), _ptr(dout_row), int(h), int(j), _ptr(acc))
+        _check(st)
+    return acc
 
 
 # ---- ending-node orientation: swap pair axes 1 and 2 around the starting-node definition ----

@@ -345,3 +345,109 @@ int tri_attn_oracle_dbias(int B, int N, int H, int d, double scale,
     }
     return err;
 }
+
+/*
+ * One pair row (b,i) on its own, for crops too large to hold the whole pair
+ * stack in FP64 on the host.  Row i of the starting-node definition reads only
+ * that row's q, k, v, dout ([N,H,d] each), the batch's bias ([H,N,N]) and the
+ * row's mask ([N], or NULL); it is the full definition above with B = 1 and
+ * the row at i = 0, and runs the very same code (problem_probs, problem_ds, the
+ * dq/dk/dv loops), so its results equal the whole-stack functions' row bit for
+ * bit.  Writes out_row, dq_row, dk_row, dv_row ([N,H,d]) and lse_row ([H,N]);
+ * dout_row and the gradient outputs may be NULL to run the forward only.
+ */
+int tri_attn_oracle_row(int N, int H, int d, double scale,
+                        const double *q, const double *k, const double *v,
+                        const double *bias, const double *mask_row, const double *dout,
+                        double *out, double *lse_row, double *dq, double *dk, double *dv)
+{
+    if (N <= 0 || H <= 0 || d <= 0 || !q || !k || !v || !bias || !out || !lse_row)
+        return ORC_ERR_ARGS;
+    if (mask_row) {
+        int any = 0;
+        for (int kk = 0; kk < N; ++kk)
+            if (mask_row[kk] > ORC_MASKED_AT) { any = 1; break; }
+        if (!any) return ORC_ERR_FULLY_MASKED;
+    }
+    const int grads = dout && dq && dk && dv;
+    int err = 0;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < H; ++h) {
+        double *P = problem_probs(1, N, H, d, scale, q, k, bias, mask_row, 0, 0, h, lse_row + (size_t)h * N, 0);
+        double *ds = grads ? (double *)malloc(sizeof(double) * (size_t)N * N) : NULL;
+        if (!P || (grads && !ds)) {
+            free(P); free(ds);
+            #pragma omp atomic write
+            err = ORC_ERR_NOMEM;
+            continue;
+        }
+        for (int j = 0; j < N; ++j)
+            for (int c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (int kk = 0; kk < N; ++kk)
+                    acc += P[(size_t)j * N + kk] * v[ix5(0, 0, kk, h, c, N, H, d)];
+                out[ix5(0, 0, j, h, c, N, H, d)] = acc;
+            }
+        if (grads) {
+            problem_ds(N, H, d, P, v, dout, 0, 0, h, ds, 0);
+            for (int kk = 0; kk < N; ++kk)
+                for (int c = 0; c < d; ++c) {
+                    double av = 0.0, ak = 0.0;
+                    for (int j = 0; j < N; ++j) {
+                        av += P[(size_t)j * N + kk] * dout[ix5(0, 0, j, h, c, N, H, d)];
+                        ak += ds[(size_t)j * N + kk] * q[ix5(0, 0, j, h, c, N, H, d)];
+                    }
+                    dv[ix5(0, 0, kk, h, c, N, H, d)] = av;
+                    dk[ix5(0, 0, kk, h, c, N, H, d)] = scale * ak;
+                }
+            for (int j = 0; j < N; ++j)
+                for (int c = 0; c < d; ++c) {
+                    double aq = 0.0;
+                    for (int kk = 0; kk < N; ++kk)
+                        aq += ds[(size_t)j * N + kk] * k[ix5(0, 0, kk, h, c, N, H, d)];
+                    dq[ix5(0, 0, j, h, c, N, H, d)] = scale * aq;
+                }
+        }
+        free(P);
+        free(ds);
+    }
+    return err;
+}
+
+/*
+ * dbias accumulation one pair row at a time: adds row i's ds[b,i,j,h,:] for
+ * one (h, j) to acc[N].  Called for i = 0, 1, ..., N-1 in turn, it performs the
+ * same FP64 operations in the same order as tri_attn_oracle_dbias does for
+ * that (b,h,j), so the two agree bit for bit.  Inputs are one row's q, k, v,
+ * dout ([N,H,d]), the batch's bias ([H,N,N]) and the row's mask ([N] or NULL).
+ */
+int tri_attn_oracle_dbias_row_add(int N, int H, int d, double scale,
+                                  const double *q, const double *k, const double *v,
+                                  const double *bias, const double *mask_row, const double *dout,
+                                  int h, int j, double *acc)
+{
+    if (N <= 0 || H <= 0 || d <= 0 || h < 0 || h >= H || j < 0 || j >= N || !q || !k || !v || !bias ||
+        !dout || !acc)
+        return ORC_ERR_ARGS;
+    double *s = (double *)malloc(sizeof(double) * (size_t)N);
+    double *p = (double *)malloc(sizeof(double) * (size_t)N);
+    double *o = (double *)malloc(sizeof(double) * (size_t)d);
+    if (!s || !p || !o) { free(s); free(p); free(o); return ORC_ERR_NOMEM; }
+    scores(1, N, H, d, scale, q, k, bias, mask_row, 0, 0, h, j, s, 0);
+    softmax_row(N, s, p);
+    for (int c = 0; c < d; ++c) {
+        double a = 0.0;
+        for (int kk = 0; kk < N; ++kk) a += p[kk] * v[ix5(0, 0, kk, h, c, N, H, d)];
+        o[c] = a;
+    }
+    double Dj = 0.0;
+    for (int c = 0; c < d; ++c) Dj += dout[ix5(0, 0, j, h, c, N, H, d)] * o[c];
+    for (int kk = 0; kk < N; ++kk) {
+        double dp = 0.0;
+        for (int c = 0; c < d; ++c)
+            dp += dout[ix5(0, 0, j, h, c, N, H, d)] * v[ix5(0, 0, kk, h, c, N, H, d)];
+        acc[kk] += p[kk] * (dp - Dj);
+    }
+    free(s); free(p); free(o);
+    return ORC_OK;
+}

@@ -250,3 +250,27 @@ def test_pins_pass_on_the_unmodified_oracle():
 @pytest.mark.parametrize("planted", [1, 2, 3, 4, 5, 6, 7])
 def test_pins_catch_planted_mistakes(planted):
     assert not _pins_pass(planted)
+
+
+@pytest.mark.parametrize("mk", ["none", "ragged"])
+def test_row_functions_equal_the_whole_stack(mk):
+    """``row`` and ``dbias_streamed`` (one pair row at a time, for crops whose
+    FP64 pair stack does not fit the host) run the whole-stack arithmetic on
+    that row: bitwise equal to ``fwd``/``bwd_rows``/``dbias``, and pinned to
+    the library attention as well."""
+    q, k, v, do, bias, mask = _rand(41, 2, 11, 2, 4, mk)
+    out, lse = O.fwd(q, k, v, bias, mask)
+    dq, dk, dv = O.bwd_rows(q, k, v, bias, mask, do)
+    db = O.dbias(q, k, v, bias, mask, do)
+    ref_out = _sdpa(q, k, v, bias, mask, 0.5).numpy()
+    for b, i in [(0, 0), (1, 7), (1, 10)]:
+        m = None if mask is None else mask[b, i]
+        o_r, l_r, dq_r, dk_r, dv_r = O.row(q[b, i], k[b, i], v[b, i], bias[b], m, do[b, i])
+        assert np.array_equal(o_r, out[b, i]) and np.array_equal(l_r, lse[b, :, i])
+        assert np.array_equal(dq_r, dq[b, i]) and np.array_equal(dk_r, dk[b, i]) and np.array_equal(dv_r, dv[b, i])
+        assert _rel(o_r, ref_out[b, i]) < 1e-12
+        o_f, l_f = O.row(q[b, i], k[b, i], v[b, i], bias[b], m)  # forward only
+        assert np.array_equal(o_f, o_r) and np.array_equal(l_f, l_r)
+    for b, h, j in [(0, 0, 0), (1, 1, 10), (0, 1, 5)]:
+        get = lambda i: (q[b, i], k[b, i], v[b, i], None if mask is None else mask[b, i], do[b, i])
+        assert np.array_equal(O.dbias_streamed(get, bias[b], h, j), db[b, h, j])

@@ -52,6 +52,21 @@ def test_static_scratch_host_side_rejections(lib):
     # invalid sizes keep the regular argument errors
     a = _fake_bwd_args(64, d=48)
     assert lib.tri_attn_bwd_static_scratch(ctypes.byref(a), None) == Bd.TRI_ATTN_ERR_UNSUPPORTED
+    # argument errors come before the size limit and before any CUDA call: on a
+    # machine without a GPU every CUDA call fails, so these statuses also show
+    # that nothing reached the runtime
+    a = _fake_bwd_args(64)
+    a.dq.ptr = None
+    assert lib.tri_attn_bwd_static_scratch(ctypes.byref(a), None) == Bd.TRI_ATTN_ERR_NULL
+    a = _fake_bwd_args(2048)
+    a.dk.ptr = None  # oversized and a NULL gradient: the argument error wins
+    assert lib.tri_attn_bwd_static_scratch(ctypes.byref(a), None) == Bd.TRI_ATTN_ERR_NULL
+    a = _fake_bwd_args(64)
+    a.dv.ptr += 2
+    assert lib.tri_attn_bwd_static_scratch(ctypes.byref(a), None) == Bd.TRI_ATTN_ERR_ALIGN
+    a = _fake_bwd_args(64)
+    a.dout.stride[2] = 12
+    assert lib.tri_attn_bwd_static_scratch(ctypes.byref(a), None) == Bd.TRI_ATTN_ERR_STRIDE
     # the documented limit covers the 768-residue crop at both head widths
     for d in (32, 64):
         assert Bd.tri_attn_bwd_workspace_bytes(1, 768, 4, d) <= Bd.TRI_ATTN_STATIC_SCRATCH_BYTES

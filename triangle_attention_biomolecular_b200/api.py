@@ -58,6 +58,15 @@ def backward(q, k, v, bias, mask, o, resid, lse, dout, scale: Optional[float] = 
     return dq, dk, dv, dbias
 
 
+def _abi_layout(t: torch.Tensor) -> torch.Tensor:
+    """t itself if the C ABI accepts its layout (innermost stride 1, other strides
+    non-negative multiples of 8 elements, 16-byte aligned data), else a dense copy
+    (e.g. the stride-0 gradient that ``out.sum().backward()`` hands over)."""
+    st = t.stride()
+    ok = st[-1] == 1 and all(s >= 0 and s % 8 == 0 for s in st[:-1]) and t.data_ptr() % 16 == 0
+    return t if ok else t.contiguous()
+
+
 class TriangleAttentionFunction(torch.autograd.Function):
     @staticmethod
     def forward(ctx, q, k, v, bias, mask, scale, orientation):
@@ -73,7 +82,7 @@ class TriangleAttentionFunction(torch.autograd.Function):
     def backward(ctx, grad_out):
         qf, kf, vf, bias, mask, o, resid, lse = ctx.saved_tensors
         mask = mask if ctx.has_mask else None
-        g = _frame(grad_out.to(torch.bfloat16), ctx.orientation)
+        g = _frame(_abi_layout(grad_out.to(torch.bfloat16)), ctx.orientation)
         dq, dk, dv, dbias = backward(qf, kf, vf, bias, mask, o, resid, lse, g, ctx.scale)
         f = lambda x: _frame(x, ctx.orientation)
         return f(dq), f(dk), f(dv), dbias, None, None, None

@@ -425,10 +425,9 @@ tri_attn_status fwd_impl(const tri_attn_fwd_args* a, int R, tri_attn_stream_t st
     return cudaGetLastError() == cudaSuccess ? TRI_ATTN_OK : TRI_ATTN_ERR_CUDA;
 }
 
-// the backward over rows 0 .. R-1; parts == nullptr: dBias (BF16) for those rows
-// as the whole sum over i; otherwise dBias leaves as FP32 partial sums in parts
-tri_attn_status bwd_impl(const tri_attn_bwd_args* a, int R, float* parts, tri_attn_stream_t stream,
-                         void* const* markers) {
+// host-side argument checks of the backward over rows 0 .. R-1 (everything but the
+// workspace); no CUDA call
+tri_attn_status bwd_check_args(const tri_attn_bwd_args* a, int R, const float* parts) {
     if (!a) return TRI_ATTN_ERR_NULL;
     tri_attn_status st = check_fwd_args(&a->f);
     if (st) return st;
@@ -441,6 +440,15 @@ tri_attn_status bwd_impl(const tri_attn_bwd_args* a, int R, float* parts, tri_at
     } else if ((st = check_t4(a->dbias))) {
         return st;
     }
+    return TRI_ATTN_OK;
+}
+
+// the backward over rows 0 .. R-1; parts == nullptr: dBias (BF16) for those rows
+// as the whole sum over i; otherwise dBias leaves as FP32 partial sums in parts
+tri_attn_status bwd_impl(const tri_attn_bwd_args* a, int R, float* parts, tri_attn_stream_t stream,
+                         void* const* markers) {
+    tri_attn_status st = bwd_check_args(a, R, parts);
+    if (st) return st;
     const int B = a->f.B, N = a->f.N, H = a->f.H, d = a->f.d;
     const tri::BwdWorkspace ws = tri::bwd_workspace_layout(B, R, N, H, d);
     const size_t need = parts ? ws.off_part : ws.total;  // shard calls keep no partials of their own
@@ -452,6 +460,12 @@ tri_attn_status bwd_impl(const tri_attn_bwd_args* a, int R, float* parts, tri_at
 }
 
 }  // namespace
+
+// argument checks of tri_attn_bwd, shared with the static-scratch entry point
+// (csrc/bwd_static.cu) so that it rejects bad arguments before any CUDA call
+namespace tri {
+tri_attn_status bwd_validate(const tri_attn_bwd_args* a) { return bwd_check_args(a, a ? a->f.N : 0, nullptr); }
+}  // namespace tri
 
 extern "C" {
 

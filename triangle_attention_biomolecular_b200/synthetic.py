@@ -98,6 +98,36 @@ def make_inputs(wl: Workload, seed: int, with_dout: bool = True) -> dict:
     return out
 
 
+def make_inputs_device(wl: Workload, seed: int, device) -> dict:
+    """The same recipe as ``make_inputs``, drawn on ``device`` with a seeded torch
+    generator there (for pair stacks whose FP32 draws would crowd the host, e.g.
+    N = 4096).  Returns device tensors in the storage frame; the values differ
+    from ``make_inputs``'s for the same seed (another generator), the
+    distributions do not."""
+    g = torch.Generator(device=device).manual_seed(int(seed))
+    shp = (wl.B, wl.N, wl.N, wl.H, wl.d)
+    out = {}
+    for key in ("q", "k", "v", "dout"):
+        out[key] = torch.randn(shp, generator=g, dtype=torch.float32, device=device).to(torch.bfloat16)
+    out["bias"] = (torch.randn((wl.B, wl.H, wl.N, wl.N), generator=g, dtype=torch.float32, device=device)
+                   * wl.bias_std).to(torch.bfloat16)
+    if wl.mask == "ragged":
+        lengths = torch.randint(wl.len_lo, wl.len_hi + 1, (wl.B,), generator=g, device=device)
+    else:
+        lengths = torch.full((wl.B,), wl.N, dtype=torch.int64, device=device)
+    if wl.mask == "none":
+        out["mask"] = None
+    else:
+        kidx = torch.arange(wl.N, device=device).view(1, 1, wl.N)
+        mask = torch.where(kidx >= lengths.view(-1, 1, 1), MASK_NEG, 0.0).to(torch.float32)
+        out["mask"] = mask.expand(wl.B, wl.N, wl.N).contiguous()
+    out["lengths"] = lengths
+    if wl.orientation == "end":
+        for key in ("q", "k", "v", "dout"):
+            out[key] = out[key].transpose(1, 2).contiguous()
+    return out
+
+
 def to_attention_frame(x: torch.Tensor, orientation: str) -> torch.Tensor:
     """View a stored [B,N,N,H,d] pair tensor in the attention's own frame."""
     return x.transpose(1, 2) if orientation == "end" else x
