@@ -21,6 +21,7 @@
 #include "sm100.cuh"
 #include "fwd.cuh"
 #include "bwd.cuh"
+#include "dbias.cuh"
 #include "tri_mul.cuh"
 #include "tri_gate.cuh"
 
@@ -264,10 +265,10 @@ bool bwd_set_attributes() {
                                MainLayout<32>::SMEM) == cudaSuccess;
     ok &= cudaFuncSetAttribute(tri_attn_bwd_main_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                MainLayout<64>::SMEM) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(tri_attn_bwd_dbias_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               DbLayout<32>::SMEM) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(tri_attn_bwd_dbias_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               DbLayout<64>::SMEM) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(tri_attn_bwd_dbias_kernel<32, TRI_DBIAS_FMA_PAIRS>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, DbLayout<32>::SMEM) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(tri_attn_bwd_dbias_kernel<64, TRI_DBIAS_FMA_PAIRS>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, DbLayout<64>::SMEM) == cudaSuccess;
     return ok;
 }
 
@@ -328,7 +329,7 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, int R, float* parts, cons
         mark(1);
         tri_attn_bwd_main_kernel<32><<<ws.grid_main, MainLayout<32>::THREADS, MainLayout<32>::SMEM, stream>>>(mq, mk, mv, mdo, p);
         mark(2);
-        tri_attn_bwd_dbias_kernel<32><<<db_grid, DbLayout<32>::THREADS, DbLayout<32>::SMEM, stream>>>(
+        tri_attn_bwd_dbias_kernel<32, TRI_DBIAS_FMA_PAIRS><<<db_grid, DbLayout<32>::THREADS, DbLayout<32>::SMEM, stream>>>(
             mq, mk, mv, mdo, bias, f.bias.stride[0], f.bias.stride[1], f.bias.stride[2], p);
     } else {
         tri_attn_bwd_prep_kernel<64><<<prep_grid, 256, 0, stream>>>(
@@ -339,7 +340,7 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, int R, float* parts, cons
         mark(1);
         tri_attn_bwd_main_kernel<64><<<ws.grid_main, MainLayout<64>::THREADS, MainLayout<64>::SMEM, stream>>>(mq, mk, mv, mdo, p);
         mark(2);
-        tri_attn_bwd_dbias_kernel<64><<<db_grid, DbLayout<64>::THREADS, DbLayout<64>::SMEM, stream>>>(
+        tri_attn_bwd_dbias_kernel<64, TRI_DBIAS_FMA_PAIRS><<<db_grid, DbLayout<64>::THREADS, DbLayout<64>::SMEM, stream>>>(
             mq, mk, mv, mdo, bias, f.bias.stride[0], f.bias.stride[1], f.bias.stride[2], p);
     }
     if (ws.chunks > 1 && !parts) {

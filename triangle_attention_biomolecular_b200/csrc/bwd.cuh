@@ -741,306 +741,7 @@ __global__ void __launch_bounds__(640, 1)
     }
 }
 
-// ===========================================================================
-// 3. dBias kernel: one CTA per (b, h, jt, kt, row chunk), rows i ascending
-// ===========================================================================
-template <int D>
-struct DbLayout {
-    static constexpr int NS = (D == 32) ? 4 : 2;
-    static constexpr int ROWB = D * 2;
-    static constexpr int QKV_TILE = 128 * ROWB;
-    static constexpr int STAGE = 4 * QKV_TILE;  // Q, dO, K, V
-    // warps 0-15: four softmax warpgroups, warpgroup w owns keys 32w..32w+31 of the
-    // tile; warp 16 producer, warp 17 MMA, 18-19 spare
-    static constexpr int THREADS = 640, SOFTMAX_WARPS = 16, W_PRODUCER = 16, W_MMA = 17;
-    static constexpr int OFF_BIAS = NS * STAGE;  // [128 rows][128 keys] fp32, log2 units, swizzled
-    // [NS][lse*log2e 128, D 128, mask*log2e 128 (fp32), key-tile flags 32 (int)]
-    static constexpr int OFF_VEC = OFF_BIAS + 128 * 128 * 4;
-    static constexpr int VEC = 1664;
-    static constexpr int OFF_BAR = OFF_VEC + NS * VEC;
-    static constexpr int B_FULL = 0, B_EMPTY = NS, B_SDPFULL = 2 * NS, B_SDPFREE = 2 * NS + 2,
-                         B_DRAIN = 2 * NS + 4, NBAR = B_DRAIN + 1;
-    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort
-    static constexpr int SMEM = OFF_MISC + 16;
-    static_assert(SMEM <= 232448, "shared memory budget");
-};
-
-template <int D>
-__global__ void __launch_bounds__(640, 1)
-    tri_attn_bwd_dbias_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                              const __nv_bfloat16* __restrict__ bias, int64_t bs0, int64_t bs1, int64_t bs2,
-                              const BwdParams p) {
-    using L = DbLayout<D>;
-    extern __shared__ __align__(1024) uint8_t smem[];
-    const uint32_t sb = smem_addr(smem);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    auto BAR = [&](int idx) -> uint32_t { return sb + L::OFF_BAR + idx * 8; };
-    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::OFF_MISC);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
-
-    const int nt = p.nt;
-    int item = blockIdx.x;
-    const int chunk = item % p.chunks;
-    item /= p.chunks;
-    const int kt = item % nt;
-    item /= nt;
-    const int jt = item % nt;
-    item /= nt;
-    const int h = item % p.H;
-    const int b = item / p.H;
-    const int rows_per = (p.R + p.chunks - 1) / p.chunks;
-    const int i_begin = chunk * rows_per;
-    const int i_end = min(p.R, i_begin + rows_per);
-    const int nrows = max(0, i_end - i_begin);
-
-    if (threadIdx.x == 0) {
-        *abort_flag = device_error_pending() ? 1 : 0;
-        if (sb & 1023u) {
-            atomicCAS(&g_error_word, 0u, ERR_TIMEOUT_BIT | KERNEL_BWD_DBIAS | 0xFFu);
-            *abort_flag = 1;
-        }
-        for (int s = 0; s < L::NS; ++s) {
-            mbar_init(BAR(L::B_FULL + s), 1);
-            mbar_init(BAR(L::B_EMPTY + s), 1 + L::SOFTMAX_WARPS);
-        }
-        for (int x = 0; x < 2; ++x) {
-            mbar_init(BAR(L::B_SDPFULL + x), 1);
-            mbar_init(BAR(L::B_SDPFREE + x), L::SOFTMAX_WARPS);
-        }
-        mbar_init(BAR(L::B_DRAIN), 1);
-        fence_mbar_init();
-    }
-    if (warp == 0) {
-        tmem_alloc(smem_addr(const_cast<uint32_t*>(tmem_slot)), 512);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const WaitCtx wc{p.wait_limit_ns, KERNEL_BWD_DBIAS, abort_flag};
-    const bool aborted_early = *abort_flag != 0;
-    constexpr float LOG2E = 1.4426950408889634f;
-
-    if (warp == L::W_PRODUCER) {
-        regs_shrink640();
-        int armed[L::NS];
-#pragma unroll
-        for (int s = 0; s < L::NS; ++s) armed[s] = 0;
-        const bool leader = elect_one();
-        if (!aborted_early) {
-            if (leader) {
-                tma_prefetch_map(&tm_q);
-                tma_prefetch_map(&tm_k);
-                tma_prefetch_map(&tm_v);
-                tma_prefetch_map(&tm_do);
-            }
-            for (int n = 0; n < nrows; ++n) {
-                const int i = i_begin + n;
-                const int s = n % L::NS;
-                if (n >= L::NS && !mbar_wait_warp(BAR(L::B_EMPTY + s), ((n / L::NS) - 1) & 1, wc, 1)) break;
-                if (leader) {
-                    const uint32_t bar = BAR(L::B_FULL + s);
-                    const uint32_t base = sb + s * L::STAGE;
-                    const uint32_t vec = sb + L::OFF_VEC + s * L::VEC;
-                    const int64_t vrow = ((static_cast<int64_t>(b) * p.H + h) * p.R + i) * p.Np + jt * 128;
-                    const int64_t mrow = (static_cast<int64_t>(b) * p.R + i) * p.Np + kt * 128;
-                    mbar_arrive_expect_tx(bar, L::STAGE + L::VEC);
-                    auto ld = [&](uint32_t dst, const CUtensorMap* m, int row0) {
-                        tma_load_5d(dst, m, bar, 0, h, row0, i, b);
-                    };
-                    ld(base, &tm_q, jt * 128);
-                    ld(base + L::QKV_TILE, &tm_do, jt * 128);
-                    ld(base + 2 * L::QKV_TILE, &tm_k, kt * 128);
-                    ld(base + 3 * L::QKV_TILE, &tm_v, kt * 128);
-                    bulk_load(vec, p.Lv + vrow, 512, bar);
-                    bulk_load(vec + 512, p.Dv + vrow, 512, bar);
-                    bulk_load(vec + 1024, p.Mv + mrow, 512, bar);
-                    bulk_load(vec + 1536, p.Fv + (static_cast<int64_t>(b) * p.R + i) * 32, 128, bar);
-                }
-                armed[s]++;
-            }
-        }
-        if (leader) {
-#pragma unroll
-            for (int s = 0; s < L::NS; ++s)
-                if (armed[s] > 0) drain_wait(BAR(L::B_FULL + s), (armed[s] - 1) & 1, 100000000ull);
-        }
-    } else if (warp == L::W_MMA) {
-        regs_shrink640();
-        const bool leader = elect_one();
-        if (!aborted_early) {
-            constexpr uint32_t SW = (D == 32) ? SWZ_64B : SWZ_128B;
-            constexpr uint32_t SBO = 8 * L::ROWB;
-            constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
-            const uint64_t d0 = smem_desc(sb, 16, SBO, SW);
-            TRI_TRACE_DECL
-            for (int n = 0; n < nrows; ++n) {
-                const int s = n % L::NS, x = n & 1;
-                TRI_TP(2)
-                if (!mbar_wait_warp(BAR(L::B_FULL + s), (n / L::NS) & 1, wc, 2)) break;
-                TRI_TP(0)
-                if (n >= 2 && !mbar_wait_warp(BAR(L::B_SDPFREE + x), ((n >> 1) - 1) & 1, wc, 3)) break;
-                TRI_TP(1)
-                tc_fence_after();
-                const uint64_t qd = desc_add(d0, s * L::STAGE);
-                if (leader) {
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        mma_ss(tmem + x * 256, desc_add(qd, kk * 32), desc_add(qd, 2 * L::QKV_TILE + kk * 32), IDESC_S,
-                               kk > 0 ? 1u : 0u);
-                        mma_ss(tmem + x * 256 + 128, desc_add(qd, L::QKV_TILE + kk * 32),
-                               desc_add(qd, 3 * L::QKV_TILE + kk * 32), IDESC_S, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(BAR(L::B_SDPFULL + x));
-                    mma_commit(BAR(L::B_EMPTY + s));
-                }
-                __syncwarp();
-            }
-            TRI_TP(2)
-            TRI_TRACE_FLUSH_AT(30000)
-            if (leader) mma_commit(BAR(L::B_DRAIN));
-            __syncwarp();
-            drain_wait(BAR(L::B_DRAIN), 0, 100000000ull);
-        }
-        __syncwarp();
-    } else if (warp >= L::SOFTMAX_WARPS) {
-        regs_shrink640();  // spare warps of the control warpgroup
-    } else {
-        regs_grow640();
-        if (!aborted_early) {
-        const int w = warp >> 2;  // key quarter of the tile
-        const int qd = warp & 3;  // TMEM lane quarter = query rows 32qd..32qd+31
-        const int row = qd * 32 + lane;
-        const uint32_t tl = tmem + (static_cast<uint32_t>(qd * 32) << 16);
-        const int j = jt * 128 + row;
-        const float c2 = p.scale * LOG2E;
-        // this thread's 32 bias values (row j, keys kt*128 + 32w ..), log2 units, kept in
-        // shared memory: a row is 512 B = 32 chunks of 16 B; chunk w*8+c sits at
-        // w*8 + (c xor (row & 7)), so eight consecutive rows hit eight different bank groups
-        const uint32_t brow = sb + L::OFF_BIAS + row * 512 + w * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            float v[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int k = kt * 128 + w * 32 + 4 * c + e;
-                float bv = 0.f;
-                if (j < p.N && k < p.N)
-                    bv = __bfloat162float(bias[b * bs0 + h * bs1 + static_cast<int64_t>(j) * bs2 + k]);
-                v[e] = bv * LOG2E;
-            }
-            sts128(brow + ((c ^ (row & 7)) << 4),
-                   make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]), __float_as_uint(v[3])));
-        }
-        float acc[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) acc[e] = 0.f;
-        bool ok = true;
-        TRI_TRACE_DECL
-        for (int n = 0; n < nrows; ++n) {
-            const int x = n & 1, s = n % L::NS;
-            if (!mbar_wait_warp(BAR(L::B_SDPFULL + x), (n >> 1) & 1, wc, 4)) { ok = false; break; }
-            TRI_TP(0)
-            tc_fence_after();
-            if (!mbar_wait_warp(BAR(L::B_FULL + s), (n / L::NS) & 1, wc, 5)) { ok = false; break; }
-            const float* vec = reinterpret_cast<const float*>(smem + L::OFF_VEC + s * L::VEC);
-            const float lse2 = vec[row];
-            const float Dj = vec[128 + row];
-            const bool has_mask = reinterpret_cast<const int*>(vec + 384)[kt] != 0;
-            const uint32_t ma = sb + L::OFF_VEC + s * L::VEC + 1024 + w * 128;
-            const float2 c22 = make_float2(c2, c2), nl2 = make_float2(-lse2, -lse2), nD2 = make_float2(-Dj, -Dj);
-            TRI_TP(1)
-            // dS = P (dP - D) accumulated over rows; in key tiles without a mask a quarter of
-            // the exponentials run on the FMA pipe (ex2_fma2) beside the MUFU unit
-            auto row_step = [&](auto masked) {
-                constexpr bool kMasked = decltype(masked)::value;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t sv[16], dv[16];
-                    tmem_ld16(tl + x * 256 + w * 32 + half * 16, sv);
-                    tmem_ld16(tl + x * 256 + 128 + w * 32 + half * 16, dv);
-                    tmem_wait_ld();
-                    reg_fence16(sv);
-                    reg_fence16(dv);
-                    if (half == 1) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(BAR(L::B_SDPFREE + x));
-                    }
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int cc = half * 4 + c;
-                        const float4 bq = lds128f(brow + ((cc ^ (row & 7)) << 4));
-                        float2 b01 = make_float2(bq.x, bq.y), b23 = make_float2(bq.z, bq.w);
-                        if constexpr (kMasked) {
-                            const float4 mq = lds128f(ma + cc * 16);
-                            b01 = fadd2(b01, make_float2(mq.x, mq.y));
-                            b23 = fadd2(b23, make_float2(mq.z, mq.w));
-                        }
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int xl = 4 * c + 2 * e;
-                            const float2 t = ffma2(make_float2(__uint_as_float(sv[xl]), __uint_as_float(sv[xl + 1])),
-                                                   c22, e ? b23 : b01);
-                            const float2 y = fadd2(t, nl2);
-                            const float2 pv = (!kMasked && (xl & 6) == 6) ? ex2_fma2(y) : make_float2(ex2(y.x), ex2(y.y));
-                            const float2 dd =
-                                fadd2(make_float2(__uint_as_float(dv[xl]), __uint_as_float(dv[xl + 1])), nD2);
-                            const float2 a = ffma2(pv, dd, make_float2(acc[16 * half + xl], acc[16 * half + xl + 1]));
-                            acc[16 * half + xl] = a.x;
-                            acc[16 * half + xl + 1] = a.y;
-                        }
-                    }
-                }
-            };
-            if (has_mask) row_step(std::true_type{});
-            else row_step(std::false_type{});
-            TRI_TP(2)
-            __syncwarp();
-            if (lane == 0) mbar_arrive(BAR(L::B_EMPTY + s));
-        }
-        TRI_TP(3)
-        if (ok && j < p.N) {
-            const int k0 = kt * 128 + w * 32;
-            if (p.chunks == 1 && !p.part_out) {
-                __nv_bfloat16* dst = p.dbias + b * p.dbs[0] + h * p.dbs[1] + static_cast<int64_t>(j) * p.dbs[2] + k0;
-#pragma unroll
-                for (int e = 0; e < 32; e += 8) {
-                    if (k0 + e + 8 <= p.N) {
-                        uint4 v;
-                        v.x = pack_bf16(acc[e], acc[e + 1]);
-                        v.y = pack_bf16(acc[e + 2], acc[e + 3]);
-                        v.z = pack_bf16(acc[e + 4], acc[e + 5]);
-                        v.w = pack_bf16(acc[e + 6], acc[e + 7]);
-                        *reinterpret_cast<uint4*>(dst + e) = v;
-                    } else {
-#pragma unroll
-                        for (int u = 0; u < 8; ++u)
-                            if (k0 + e + u < p.N) dst[e + u] = __float2bfloat16_rn(acc[e + u]);
-                    }
-                }
-            } else {
-                float* dst = p.part + (((static_cast<int64_t>(chunk) * p.B + b) * p.H + h) * p.N + j) * p.N + k0;
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    if (k0 + e < p.N) dst[e] = acc[e];
-            }
-        }
-        TRI_TP(4)
-        TRI_TRACE_FLUSH_AT(30000)
-    }
-
-    }
-
-    tc_fence_before();
-    cta_end_barrier640();
-    if (warp == 0) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 512);
-    }
-}
+// 3. the dBias kernel is in dbias.cuh
 
 // ascending-index sum of dBias partials (the chunks of one launch, or the chunks of
 // every row shard in rank order) -> BF16

@@ -436,16 +436,18 @@ __global__ void __launch_bounds__(384, 1)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(BAR(L::B_EMPTY + s));
-            // row maximum: four independent chains of three-input maxima
+            // row maximum: four independent chains of three-input maxima over x[4..123],
+            // then the last four scores
             float ma0 = x[0], ma1 = x[1], ma2 = x[2], ma3 = x[3];
 #pragma unroll
-            for (int e = 4; e < 128; e += 8) {
+            for (int e = 4; e < 124; e += 8) {
                 ma0 = fmax3(ma0, x[e], x[e + 1]);
                 ma1 = fmax3(ma1, x[e + 2], x[e + 3]);
                 ma2 = fmax3(ma2, x[e + 4], x[e + 5]);
                 ma3 = fmax3(ma3, x[e + 6], x[e + 7]);
             }
-            const float mt = fmaxf(fmaxf(ma0, ma1), fmaxf(ma2, ma3));
+            const float mt = fmaxf(fmaxf(fmaxf(ma0, x[124]), fmaxf(ma1, x[125])),
+                                   fmaxf(fmaxf(ma2, x[126]), fmaxf(ma3, x[127])));
             TRI_TP(3)
             bool need = false;
             float alpha = 1.f;

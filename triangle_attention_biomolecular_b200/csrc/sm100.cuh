@@ -335,10 +335,26 @@ __device__ __forceinline__ void regs_shrink640() {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSmall640));
 }
 __device__ __forceinline__ void regs_grow640() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsLarge640)); }
+// A wider split of the same 640-thread launch for kernels whose control warps
+// need few registers: 512 * 112 + 128 * 32 = 61440, the launch total.
+constexpr int kRegsSmall640w = 32, kRegsLarge640w = 112;
+static_assert(128 * kRegsSmall640w + 512 * kRegsLarge640w <= 640 * kRegsLaunch640, "register split must fit the launch");
+__device__ __forceinline__ void regs_shrink640w() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSmall640w));
+}
+__device__ __forceinline__ void regs_grow640w() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsLarge640w)); }
 __device__ __forceinline__ void regs_grow() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsLarge)); }
+// The same for 768-thread kernels (four softmax warpgroups and two control /
+// epilogue warpgroups, 80 registers each at launch, 61440 total):
+// 512 * 96 + 256 * 48 = 61440.
+constexpr int kRegsLaunch768 = 80, kRegsSmall768 = 48, kRegsLarge768 = 96;
+static_assert(256 * kRegsSmall768 + 512 * kRegsLarge768 <= 768 * kRegsLaunch768, "register split must fit the launch");
+__device__ __forceinline__ void regs_shrink768() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSmall768)); }
+__device__ __forceinline__ void regs_grow768() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsLarge768)); }
 // every role of the CTA meets here before tensor memory is released
 __device__ __forceinline__ void cta_end_barrier() { asm volatile("bar.sync 1, 384;" ::: "memory"); }
 __device__ __forceinline__ void cta_end_barrier640() { asm volatile("bar.sync 1, 640;" ::: "memory"); }
+__device__ __forceinline__ void cta_end_barrier768() { asm volatile("bar.sync 1, 768;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // arithmetic helpers
@@ -423,10 +439,12 @@ __device__ __forceinline__ float2 ex2_fma2(float2 x) {
     float2 q = ffma2(make_float2(kEx2C3, kEx2C3), f, make_float2(kEx2C2, kEx2C2));
     q = ffma2(q, f, make_float2(kEx2C1, kEx2C1));
     q = ffma2(q, f, make_float2(kEx2C0, kEx2C0));
-    // floor(x) sits in the low mantissa bits of t; shifting t left by 23 moves it into the
-    // exponent field (the constant high bits shift out)
-    return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
-                       __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+    // floor(x) sits in the low mantissa bits of t; t * 2^23 (mod 2^32) moves it into the
+    // exponent field (the constant high bits shift out), added to q's bits in one IMAD
+    uint32_t rx, ry;
+    asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(rx) : "r"(__float_as_uint(t.x)), "r"(__float_as_uint(q.x)));
+    asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(ry) : "r"(__float_as_uint(t.y)), "r"(__float_as_uint(q.y)));
+    return make_float2(__uint_as_float(rx), __uint_as_float(ry));
 }
 // max of three
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
