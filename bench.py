@@ -133,7 +133,7 @@ def kernel_source_digest() -> str:
     code and shared helpers), in name order."""
     import hashlib
     csrc = os.path.join(ROOT, "triangle_attention_biomolecular_b200", "csrc")
-    files = [os.path.join(csrc, n) for n in ("bwd.cuh", "fwd.cuh", "sm100.cuh")]
+    files = [os.path.join(csrc, n) for n in ("bwd.cuh", "dbias.cuh", "fwd.cuh", "sm100.cuh")]
     h = hashlib.sha256()
     for fn in files:
         h.update(os.path.basename(fn).encode())
@@ -190,6 +190,7 @@ def run_ours(args, rank, world, local_rank):
             Bd.tri_attn_bwd_marked(q, k, v, bias, mask, o, r, lse, do, dq, dk, dv, db, ws, ev[1:5], 0.0, 0,
                                    stream)
 
+    torch.cuda.reset_peak_memory_stats(dev)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -301,8 +302,11 @@ def run_ours(args, rank, world, local_rank):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
                "ms_per_step": round(ems / n_e2e, 4),
                "pipelining": "two buffer sets; H2D, compute and D2H on three streams"}
+    mem = {"peak_allocated_bytes": int(torch.cuda.max_memory_allocated(dev)),
+           "bwd_workspace_bytes": int(ws.numel()),
+           "saved_state_bytes": int(2 * o.numel() * o.element_size() + lse.numel() * lse.element_size())}
     return {"ms": ms, "kern_ms": kern_ms, "clocks": clocks, "e2e": e2e, "shape": (Bn, N, H, d),
-            "step_stats": step_stats, "lengths": lengths}
+            "step_stats": step_stats, "lengths": lengths, "memory": mem}
 
 
 # ---------------------------------------------------------------------------
@@ -347,8 +351,12 @@ def run_sweep(args):
             torch.cuda.synchronize()
             return e0.elapsed_time(e1) / n
         n_iter = max(5, min(200, int(2e12 / (14.0 * Bn * H * N ** 3 * d))))
+        sampler = ClockSampler(0)
+        sampler.start()
+        time.sleep(0.3)
         t_f = timed(fwd, n_iter)
         t_fb = timed(lambda: (fwd(), bwd()), n_iter)
+        clocks = sampler.stop()
         st, word = Bd.tri_attn_device_error(True)
         if st != 0:
             raise RuntimeError(f"device error word {word:#x} in {wl.name}")
@@ -364,7 +372,7 @@ def run_sweep(args):
                 "fwd_bwd_ms": round(t_fb, 4), "fwd_bwd_tflops": round(14.0 * cube / (t_fb * 1e-3) / 1e12, 2),
                 "fwd_bwd_tflops_effective": round(14.0 * eff / (t_fb * 1e-3) / 1e12, 2),
                 "pct_of_bf16_peak": round(100.0 * 14.0 * cube / (t_fb * 1e-3) / 1e12 / peak, 2),
-                "peak_source": f"{src} bf16_tflops {peak}"}
+                "peak_source": f"{src} bf16_tflops {peak}", "clocks": clocks}
         if N <= 512:
             gbs = fwd_bytes / (t_f * 1e-3) / 1e9
             line["fwd_algorithmic_gbs"] = round(gbs, 1)
@@ -559,11 +567,16 @@ def oracle_sample(rows_n: int):
     q, k, v, do, bias = (f64(x[n]) for n in ("q", "k", "v", "dout", "bias"))
     mask = x["mask"].numpy().astype(np.float64)
     rows = [(0, (37 * r) % wl.N) for r in range(rows_n)]
+    acc = np.zeros((wl.H, wl.N, wl.N))
 
     def run(rs):
+        # the whole step restricted to the sampled pair rows: forward, dq/dk/dv, and the
+        # rows' share of the dBias sum over i
         t = time.perf_counter()
         O.fwd(q, k, v, bias, mask, rows=rs)
         O.bwd_rows(q, k, v, bias, mask, do, rows=rs)
+        for b, i in rs:
+            O.dbias_add_row(acc, q[b, i], k[b, i], v[b, i], bias[b], mask[b, i], do[b, i])
         return time.perf_counter() - t
     return wl, rows, run
 
@@ -584,15 +597,16 @@ def run_cpu_baseline(target_s: float = 15.0):
     t = run(rows[:n])
     return {"value": round(cpu_rate(wl, n, t), 6), "unit": "TFLOP/s", "cores": os.cpu_count(),
             "kind": "oracle", "seconds": round(t, 3),
-            "sample": f"{n} pair rows (all 4 heads) of the crop768 workload: FP64 oracle forward + dq/dk/dv; "
-                      f"rate counts 14*H*N^2*d flops per row"}
+            "sample": f"{n} pair rows (all 4 heads) of the crop768 workload: FP64 oracle forward, dq/dk/dv "
+                      f"and the rows' share of dbias; rate counts 14*H*N^2*d flops per row"}
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    wl, rows, run = oracle_sample(64)
-    per_step_rows = 2
+    cores = os.cpu_count() or 1
+    per_step_rows = cores  # one pair row per host core and step, so every core has work
+    wl, rows, run = oracle_sample(max(64, 4 * per_step_rows))
     for s in range(args.warmup):
         run(rows[:1])
     times = []
@@ -606,9 +620,10 @@ def run_reference(args, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * tot / max(1, args.steps), 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD + " -- each step a bounded sample of 2 pair rows"},
+        "config": {"workload": WORKLOAD + f" -- each step a bounded sample of {per_step_rows} pair rows"},
         "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
-                         "sample": f"{per_step_rows} pair rows per step (all 4 heads), FP64 oracle fwd + dq/dk/dv"},
+                         "sample": f"{per_step_rows} pair rows per step (all 4 heads), FP64 oracle forward, "
+                                   "dq/dk/dv and the rows' share of dbias"},
         "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -737,6 +752,7 @@ def main():
         "effective_tflops": round(whole_job_rate(world, eff_flops, args.steps, ms), 3),
         "gpu_launches": 4 * args.steps,
         "clocks": res["clocks"],
+        "memory": res["memory"],
         "e2e": res["e2e"],
     }
     if world == 1 and not args.no_cpu_baseline:

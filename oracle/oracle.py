@@ -74,8 +74,10 @@ def _load():
             lib.tri_attn_oracle_dbias.argtypes = [i, i, i, i, d, dp, dp, dp, dp, dp, dp, ip, i, dp, i]
             lib.tri_attn_oracle_row.argtypes = [i, i, i, d, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp]
             lib.tri_attn_oracle_dbias_row_add.argtypes = [i, i, i, d, dp, dp, dp, dp, dp, dp, i, i, dp]
+            lib.tri_attn_oracle_dbias_row_add_all.argtypes = [i, i, i, d, dp, dp, dp, dp, dp, dp, dp]
             for f in (lib.tri_attn_oracle_fwd, lib.tri_attn_oracle_bwd_rows, lib.tri_attn_oracle_dbias,
-                      lib.tri_attn_oracle_row, lib.tri_attn_oracle_dbias_row_add):
+                      lib.tri_attn_oracle_row, lib.tri_attn_oracle_dbias_row_add,
+                      lib.tri_attn_oracle_dbias_row_add_all):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -215,6 +217,20 @@ def dbias_streamed(get_row, bias_b, h, j, scale=None):
         st = lib.tri_attn_oracle_dbias_row_add(N, H, d, sc, _ptr(q_row), _ptr(k_row), _ptr(v_row), _ptr(bias_b),
                                                _ptr(mask_row), _ptr(dout_row), int(h), int(j), _ptr(acc))
         _check(st)
+    return acc
+
+
+def dbias_add_row(acc, q_row, k_row, v_row, bias_b, mask_row, dout_row, scale=None):
+    """Add pair row i's ds[b,i,j,h,:] for every (h, j) into acc ([H,N,N] FP64, in
+    place).  Over all rows in ascending order this equals ``dbias`` for the batch
+    bit for bit."""
+    q_row, k_row, v_row, bias_b, mask_row, dout_row = map(_f64, (q_row, k_row, v_row, bias_b, mask_row, dout_row))
+    N, H, d = q_row.shape
+    assert acc.dtype == np.float64 and acc.shape == (H, N, N) and acc.flags.c_contiguous
+    scale = default_scale(d) if scale is None else float(scale)
+    st = _load().tri_attn_oracle_dbias_row_add_all(N, H, d, scale, _ptr(q_row), _ptr(k_row), _ptr(v_row),
+                                                   _ptr(bias_b), _ptr(mask_row), _ptr(dout_row), _ptr(acc))
+    _check(st)
     return acc
 
 

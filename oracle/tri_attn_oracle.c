@@ -451,3 +451,31 @@ int tri_attn_oracle_dbias_row_add(int N, int H, int d, double scale,
     free(s); free(p); free(o);
     return ORC_OK;
 }
+
+/*
+ * Row i's share of dbias for every (h, j): adds ds[b,i,j,h,:] into acc
+ * ([H][N][N], the batch's dbias accumulator), with the operations of
+ * tri_attn_oracle_dbias_row_add.  Called for i = 0, 1, ..., N-1 in turn it
+ * reproduces tri_attn_oracle_dbias for the batch bit for bit; called for a
+ * subset of rows it is that subset's part of the sum (what a row-sampled
+ * timing of the whole backward has to include).
+ */
+int tri_attn_oracle_dbias_row_add_all(int N, int H, int d, double scale,
+                                      const double *q, const double *k, const double *v,
+                                      const double *bias, const double *mask_row, const double *dout,
+                                      double *acc)
+{
+    if (N <= 0 || H <= 0 || d <= 0 || !acc) return ORC_ERR_ARGS;
+    int err = 0;
+    #pragma omp parallel for schedule(dynamic, 8) collapse(2)
+    for (int h = 0; h < H; ++h)
+        for (int j = 0; j < N; ++j) {
+            int st = tri_attn_oracle_dbias_row_add(N, H, d, scale, q, k, v, bias, mask_row, dout, h, j,
+                                                   acc + ((size_t)h * N + j) * (size_t)N);
+            if (st) {
+                #pragma omp atomic write
+                err = st;
+            }
+        }
+    return err;
+}

@@ -274,3 +274,8 @@ def test_row_functions_equal_the_whole_stack(mk):
     for b, h, j in [(0, 0, 0), (1, 1, 10), (0, 1, 5)]:
         get = lambda i: (q[b, i], k[b, i], v[b, i], None if mask is None else mask[b, i], do[b, i])
         assert np.array_equal(O.dbias_streamed(get, bias[b], h, j), db[b, h, j])
+    for b in range(2):  # every (h, j) at once, one row at a time
+        acc = np.zeros((2, 11, 11))
+        for i in range(11):
+            O.dbias_add_row(acc, q[b, i], k[b, i], v[b, i], bias[b], None if mask is None else mask[b, i], do[b, i])
+        assert np.array_equal(acc, db[b])

@@ -83,8 +83,8 @@ struct BwdParams {
     int B, N, H, nt, Np;
     int R;            // rows i this launch covers (N, or a shard of the rows)
     float scale;
-    const float* Lv;  // [B,H,R,Np] lse * log2(e); +inf past N
-    const float* Dv;  // [B,H,R,Np] D; 0 past N
+    const float* Lv;  // [B,H,R,Np] -lse * log2(e); -inf past N
+    const float* Dv;  // [B,H,R,Np] -D; 0 past N
     const float* Mv;  // [B,R,Np]   mask * log2(e); -inf past N
     const int* Fv;    // [B,R,32]   1 where a key tile needs the mask add
     const __nv_bfloat16* bias;  // [B,H,N,N] (read directly by the softmax warps of the main kernel)
@@ -102,9 +102,10 @@ struct BwdParams {
 // ===========================================================================
 // 1. pre-pass: the per-row vectors both backward kernels stream, laid out so
 //    that every 128-wide tile is one aligned 512-byte bulk copy:
-//      D  = rowsum(dout * (o + resid))  (FP32; the residual restores what BF16
+//      ND = -rowsum(dout * (o + resid))  (FP32; the residual restores what BF16
 //           rounding of the output dropped), 0 past N
-//      L  = lse * log2(e), +inf past N (so padded query rows get P = 0)
+//      NL = -lse * log2(e), -inf past N (so padded query rows get P = 0)
+//      (both negated: the kernels add them)
 //      M  = mask * log2(e) (0 without a mask), -inf past N (padded keys)
 //      F  = per (b, i, key tile): 1 if that tile needs the mask add at all
 // ===========================================================================
@@ -133,7 +134,7 @@ __global__ void __launch_bounds__(256) tri_attn_bwd_prep_kernel(
             const int i = static_cast<int>(t % R);
             const int b = static_cast<int>(t / R);
             const int64_t out = ((static_cast<int64_t>(b) * H + h) * R + i) * Np + j;
-            float dsum = 0.f, lv = INFINITY;
+            float dsum = 0.f, lv = -INFINITY;
             if (j < N) {
                 const uint4* pd = reinterpret_cast<const uint4*>(dout + b * s0 + i * s1 + j * s2 + h * s3);
                 const uint4* po = reinterpret_cast<const uint4*>(o + b * o0 + i * o1 + j * o2 + h * o3);
@@ -151,9 +152,9 @@ __global__ void __launch_bounds__(256) tri_attn_bwd_prep_kernel(
                         dsum = fmaf(bf16hi(aw[e]), bf16hi(ow[e]) + bf16hi(rw[e]), dsum);
                     }
                 }
-                lv = __ldg(lse + ((static_cast<int64_t>(b) * H + h) * R + i) * N + j) * LOG2E;
+                lv = -(__ldg(lse + ((static_cast<int64_t>(b) * H + h) * R + i) * N + j) * LOG2E);
             }
-            Dv[out] = dsum;
+            Dv[out] = -dsum;
             Lv[out] = lv;
         } else if (idx < n1 + n2) {
             const int64_t e = idx - n1;
@@ -648,14 +649,14 @@ __global__ void __launch_bounds__(640, 1)
                     if (!mbar_wait_warp(BAR(L::B_TFULL + ts), (g / L::NS) & 1, wc, 14)) { ok = false; break; }
                     TRI_TP(2)
                     const float* vec = reinterpret_cast<const float*>(smem + L::OFF_VEC + ts * 1024);
-                    const float lse2 = vec[row];
-                    const float Dj = vec[128 + row];
+                    const float nlse2 = vec[row];  // -lse * log2(e)
+                    const float nDj = vec[128 + row];  // -D
                     // P and dS of this warpgroup's 32 keys, packed BF16 pairs, computed in two
                     // 16-key halves while the previous tile's gradient MMAs still read the
                     // shared-memory tiles
                     uint32_t pw[16], dw[16];
                     const float2 sc2 = make_float2(scale, scale), l2e = make_float2(LOG2E, LOG2E);
-                    const float2 nl2 = make_float2(-lse2, -lse2), nD2 = make_float2(-Dj, -Dj);
+                    const float2 nl2 = make_float2(nlse2, nlse2), nD2 = make_float2(nDj, nDj);
                     // all 32 keys of S and dP first, so the S/dP columns are released to the MMA
                     // warp before any arithmetic
                     uint32_t sv[32], dv[32];

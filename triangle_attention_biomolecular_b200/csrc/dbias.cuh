@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(640, 1)
         // ====== augmentation blocks: -(lse/scale) and -D as hi + mid + lo BF16 ======
         regs_shrink640w();
         if (!aborted_early) {
-            // Lv holds lse * log2(e); lse / scale = Lv / c.  Padded query rows (Lv = +inf)
+            // Lv holds -lse * log2(e); -lse / scale = Lv / c.  Padded query rows (Lv = -inf)
             // get a large finite negative term so that their scores underflow to 0.
             const float inv_c = 1.0f / (p.scale * LOG2E);
             for (int n = 0; n < nrows; ++n) {
@@ -233,9 +233,9 @@ __global__ void __launch_bounds__(640, 1)
                 for (int q = 0; q < 4; ++q) {
                     const int r = q * 32 + lane;
                     const float lv = vec[r];
-                    const float xl = (lv < 3.0e38f) ? -lv * inv_c : -3.0e38f;
+                    const float xl = (lv > -3.0e38f) ? lv * inv_c : -3.0e38f;
                     sts128(al + aug_offset(r, 0), split3_bf16(xl));
-                    sts128(ad + aug_offset(r, 0), split3_bf16(-vec[128 + r]));
+                    sts128(ad + aug_offset(r, 0), split3_bf16(vec[128 + r]));
                 }
                 fence_proxy_async_smem();
                 __syncwarp();

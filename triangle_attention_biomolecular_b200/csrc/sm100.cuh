@@ -344,17 +344,9 @@ __device__ __forceinline__ void regs_shrink640w() {
 }
 __device__ __forceinline__ void regs_grow640w() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsLarge640w)); }
 __device__ __forceinline__ void regs_grow() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsLarge)); }
-// The same for 768-thread kernels (four softmax warpgroups and two control /
-// epilogue warpgroups, 80 registers each at launch, 61440 total):
-// 512 * 96 + 256 * 48 = 61440.
-constexpr int kRegsLaunch768 = 80, kRegsSmall768 = 48, kRegsLarge768 = 96;
-static_assert(256 * kRegsSmall768 + 512 * kRegsLarge768 <= 768 * kRegsLaunch768, "register split must fit the launch");
-__device__ __forceinline__ void regs_shrink768() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSmall768)); }
-__device__ __forceinline__ void regs_grow768() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsLarge768)); }
 // every role of the CTA meets here before tensor memory is released
 __device__ __forceinline__ void cta_end_barrier() { asm volatile("bar.sync 1, 384;" ::: "memory"); }
 __device__ __forceinline__ void cta_end_barrier640() { asm volatile("bar.sync 1, 640;" ::: "memory"); }
-__device__ __forceinline__ void cta_end_barrier768() { asm volatile("bar.sync 1, 768;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // arithmetic helpers
