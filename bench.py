@@ -168,7 +168,7 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    wl = {"crop768": S.CROP768, "crop640": S.CROP640, "crop384": S.CROP384}[args.workload]
+    wl = {"crop768": S.CROP768, "crop640": S.CROP640, "crop384": S.CROP384, "b2n256": S.sweep(256, 32)}[args.workload]
     Bn, N, H, d = wl.B, wl.N, wl.H, wl.d
     x = S.make_inputs(wl, S.seed_for(3, rank))
     q, k, v, do, bias = (x[n].to(dev) for n in ("q", "k", "v", "dout", "bias"))
@@ -636,8 +636,9 @@ def main():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", choices=("crop768", "crop640", "crop384"), default="crop768",
-                    help="crop768 is the headline; the smaller crops serve profiler captures")
+    ap.add_argument("--workload", choices=("crop768", "crop640", "crop384", "b2n256"), default="crop768",
+                    help="crop768 is the headline; the smaller crops and the batched B=2, N=256, d=32 ragged "
+                         "sweep case serve profiler captures")
     ap.add_argument("--gate-rows", type=int, default=768 * 768,
                     help="pair positions R of the --op gate workload (default 768^2; smaller only for profiling)")
     ap.add_argument("--op", choices=("attention", "tri_mul", "gate"), default="attention",

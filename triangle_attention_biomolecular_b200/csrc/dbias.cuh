@@ -29,9 +29,9 @@
 #include "sm100.cuh"
 #include "bwd.cuh"
 
-// pairs of every four that take the FMA-pipe exponential (key tiles without a mask)
+// pairs of every eight that take the FMA-pipe exponential (key tiles without a mask)
 #ifndef TRI_DBIAS_FMA_PAIRS
-#define TRI_DBIAS_FMA_PAIRS 1
+#define TRI_DBIAS_FMA_PAIRS 2
 #endif
 
 namespace tri {
@@ -83,7 +83,7 @@ __device__ __forceinline__ uint4 split3_bf16(float x) {
     return make_uint4((hi_w & 0xFFFFu) | (mid_w << 16), lo_w & 0xFFFFu, 0u, 0u);
 }
 
-// FMA_PAIRS: how many of every four score pairs take the FMA-pipe exponential
+// FMA_PAIRS: how many of every eight score pairs take the FMA-pipe exponential
 // in key tiles without a mask (the rest, and every masked tile, use MUFU)
 template <int D, int FMA_PAIRS>
 __global__ void __launch_bounds__(640, 1)
@@ -363,7 +363,7 @@ __global__ void __launch_bounds__(640, 1)
                         const int xl = 4 * cc + 2 * e;
                         const float2 y = ffma2(make_float2(__uint_as_float(sv[xl]), __uint_as_float(sv[xl + 1])),
                                                c22, e ? b23 : b01);
-                        const int pair = (xl >> 1) & 3;  // position of this pair within four
+                        const int pair = (xl >> 1) & 7;  // position of this pair within eight
                         const float2 pv = (!kMasked && pair < FMA_PAIRS) ? ex2_fma2(y)
                                                                          : make_float2(ex2(y.x), ex2(y.y));
                         const float2 a = ffma2(pv, make_float2(__uint_as_float(dv[xl]), __uint_as_float(dv[xl + 1])),

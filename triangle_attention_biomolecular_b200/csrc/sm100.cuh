@@ -431,12 +431,10 @@ __device__ __forceinline__ float2 ex2_fma2(float2 x) {
     float2 q = ffma2(make_float2(kEx2C3, kEx2C3), f, make_float2(kEx2C2, kEx2C2));
     q = ffma2(q, f, make_float2(kEx2C1, kEx2C1));
     q = ffma2(q, f, make_float2(kEx2C0, kEx2C0));
-    // floor(x) sits in the low mantissa bits of t; t * 2^23 (mod 2^32) moves it into the
-    // exponent field (the constant high bits shift out), added to q's bits in one IMAD
-    uint32_t rx, ry;
-    asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(rx) : "r"(__float_as_uint(t.x)), "r"(__float_as_uint(q.x)));
-    asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(ry) : "r"(__float_as_uint(t.y)), "r"(__float_as_uint(q.y)));
-    return make_float2(__uint_as_float(rx), __uint_as_float(ry));
+    // floor(x) sits in the low mantissa bits of t; shifting t left by 23 moves it into the
+    // exponent field (the constant high bits shift out)
+    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 // max of three
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
