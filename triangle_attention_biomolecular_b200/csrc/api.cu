@@ -298,6 +298,7 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, int R, float* parts, cons
     p.Dv = Dv; p.Lv = Lv; p.Mv = Mv; p.Fv = Fv;
     p.bias = static_cast<const __nv_bfloat16*>(f.bias.ptr);
     p.bs0 = f.bias.stride[0]; p.bs1 = f.bias.stride[1]; p.bs2 = f.bias.stride[2];
+    p.bias_tiles = reinterpret_cast<const uint4*>(wsb + ws.off_BT);
     p.dq_slots = reinterpret_cast<float*>(wsb + ws.off_dq);
     p.part = parts ? parts : reinterpret_cast<float*>(wsb + ws.off_part);
     p.part_out = parts ? 1 : 0;
@@ -319,6 +320,14 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, int R, float* parts, cons
     const unsigned db_grid = static_cast<unsigned>(B) * H * p.nt * p.nt * ws.chunks;
     const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(f.bias.ptr);
     const auto& so = f.o.stride; const auto& sr = f.resid.stride; const auto& sd = a->dout.stride;
+    // pre-pass 1b: the bias in the main kernel's read order
+    auto launch_bias_tiles = [&]() {
+        const int64_t chunks16 = static_cast<int64_t>(B) * H * ws.Np * (ws.Np / 8);
+        const unsigned g = static_cast<unsigned>(std::min<int64_t>((chunks16 + 255) / 256, 148 * 16));
+        tri_attn_bwd_bias_tiles_kernel<<<g, 256, 0, stream>>>(bias, f.bias.stride[0], f.bias.stride[1],
+                                                              f.bias.stride[2], B, H, N, p.nt,
+                                                              reinterpret_cast<uint4*>(wsb + ws.off_BT));
+    };
     mark(0);
     if (d == 32) {
         tri_attn_bwd_prep_kernel<32><<<prep_grid, 256, 0, stream>>>(
@@ -326,6 +335,7 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, int R, float* parts, cons
             static_cast<const __nv_bfloat16*>(f.o.ptr), so[0], so[1], so[2], so[3],
             static_cast<const __nv_bfloat16*>(f.resid.ptr), sr[0], sr[1], sr[2], sr[3], use_resid, f.lse, f.mask.ptr,
             sm[0], sm[1], sm[2], Dv, Lv, Mv, Fv, B, N, R, H, ws.Np, p.nt);
+        launch_bias_tiles();
         mark(1);
         tri_attn_bwd_main_kernel<32><<<ws.grid_main, MainLayout<32>::THREADS, MainLayout<32>::SMEM, stream>>>(mq, mk, mv, mdo, p);
         mark(2);
@@ -337,6 +347,7 @@ tri_attn_status bwd_launch(const tri_attn_bwd_args* a, int R, float* parts, cons
             static_cast<const __nv_bfloat16*>(f.o.ptr), so[0], so[1], so[2], so[3],
             static_cast<const __nv_bfloat16*>(f.resid.ptr), sr[0], sr[1], sr[2], sr[3], use_resid, f.lse, f.mask.ptr,
             sm[0], sm[1], sm[2], Dv, Lv, Mv, Fv, B, N, R, H, ws.Np, p.nt);
+        launch_bias_tiles();
         mark(1);
         tri_attn_bwd_main_kernel<64><<<ws.grid_main, MainLayout<64>::THREADS, MainLayout<64>::SMEM, stream>>>(mq, mk, mv, mdo, p);
         mark(2);

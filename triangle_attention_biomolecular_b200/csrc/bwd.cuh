@@ -42,7 +42,7 @@ constexpr int kDqSlots = 148;   // persistent CTAs of the main kernel (B200 SM c
 constexpr int kChunkTarget = 148;
 
 struct BwdWorkspace {
-    size_t off_D, off_L, off_M, off_F, off_dq, off_part, total;
+    size_t off_D, off_L, off_M, off_F, off_dq, off_BT, off_part, total;
     int chunks;     // row chunks of the dBias kernel
     int grid_main;  // CTAs of the main kernel
     int Np;         // N rounded up to whole 128-wide tiles
@@ -73,7 +73,8 @@ inline BwdWorkspace bwd_workspace_layout(int B, int R, int N, int H, int d) {
     w.off_M = w.off_L + align256(bhnp * 4);
     w.off_F = w.off_M + align256(bnp * 4);
     w.off_dq = w.off_F + align256(static_cast<size_t>(B) * R * 32 * 4);
-    w.off_part = w.off_dq + align256(static_cast<size_t>(kDqSlots) * N * d * 4);
+    w.off_BT = w.off_dq + align256(static_cast<size_t>(kDqSlots) * N * d * 4);
+    w.off_part = w.off_BT + align256(static_cast<size_t>(B) * H * w.Np * w.Np * 2);
     const size_t bhnn = static_cast<size_t>(B) * H * N * N;
     w.total = w.off_part + (chunks > 1 ? align256(static_cast<size_t>(chunks) * bhnn * 4) : 0);
     return w;
@@ -87,8 +88,9 @@ struct BwdParams {
     const float* Dv;  // [B,H,R,Np] -D; 0 past N
     const float* Mv;  // [B,R,Np]   mask * log2(e); -inf past N
     const int* Fv;    // [B,R,32]   1 where a key tile needs the mask add
-    const __nv_bfloat16* bias;  // [B,H,N,N] (read directly by the softmax warps of the main kernel)
+    const __nv_bfloat16* bias;  // [B,H,N,N] as given (the dBias pass reads it)
     int64_t bs0, bs1, bs2;
+    const uint4* bias_tiles;    // [B,H,nt,nt][32 KB] the bias in main-kernel read order (pre-pass 1b)
     float* dq_slots;  // [kDqSlots][N][d] (used when dq_tmem == 0)
     int dq_tmem;      // 1: dQ for every query tile stays in TMEM across key tiles
     float* part;      // [chunks][B,H,N,N] (chunks > 1, or always when part_out)
@@ -180,6 +182,52 @@ __global__ void __launch_bounds__(256) tri_attn_bwd_prep_kernel(
             }
             Fv[e] = f;
         }
+    }
+}
+
+// ===========================================================================
+// 1b. pre-pass: the pair bias rearranged into the order in which the main
+//     kernel's softmax threads read it.  A softmax thread owns one query row j
+//     and 32 keys of every 128 x 128 tile, so in the stored [B,H,N,N] layout
+//     the 32 lanes of a warp read 32 rows 2N bytes apart and every 16-byte
+//     load touches 32 cache lines.  Here each tile (b, h, jt, kt) becomes one
+//     32 KB block of 16-byte chunks, chunk index
+//         ((w * 4 + qd) * 4 + c) * 32 + lane,
+//     for row j = 128 jt + 32 qd + lane and keys k = 128 kt + 32 w + 8 c + 0..7,
+//     so that the four loads of a warp per tile each cover 512 contiguous
+//     bytes.  Values are copied bit for bit; zeros past N (padded rows get
+//     P = 0 from the -inf lse, padded keys the -inf mask).
+// ===========================================================================
+__global__ void __launch_bounds__(256) tri_attn_bwd_bias_tiles_kernel(const __nv_bfloat16* __restrict__ bias,
+                                                                      int64_t s0, int64_t s1, int64_t s2, int B,
+                                                                      int H, int N, int nt, uint4* __restrict__ out) {
+    const int Np = nt * 128, kcs = Np / 8;
+    const int64_t total = static_cast<int64_t>(B) * H * Np * kcs;
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        int64_t t = idx;
+        const int k0 = static_cast<int>(t % kcs) * 8;  // neighbouring threads read one row: coalesced
+        t /= kcs;
+        const int j = static_cast<int>(t % Np);
+        t /= Np;
+        const int h = static_cast<int>(t % H);
+        const int b = static_cast<int>(t / H);
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (j < N && k0 < N) {
+            const __nv_bfloat16* src = bias + b * s0 + h * s1 + static_cast<int64_t>(j) * s2 + k0;
+            if (k0 + 8 <= N) {
+                v = __ldg(reinterpret_cast<const uint4*>(src));
+            } else {  // ragged key tail: element loads, zeros past N
+                uint16_t e8[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) e8[u] = (k0 + u < N) ? __bfloat16_as_ushort(src[u]) : 0;
+                v = make_uint4(e8[0] | (e8[1] << 16), e8[2] | (e8[3] << 16), e8[4] | (e8[5] << 16),
+                               e8[6] | (static_cast<uint32_t>(e8[7]) << 16));
+            }
+        }
+        const int row = j & 127, kk = k0 & 127;
+        const int64_t tile = (static_cast<int64_t>(b * H + h) * nt + (j >> 7)) * nt + (k0 >> 7);
+        out[(tile << 11) + ((((kk >> 5) * 4 + (row >> 5)) * 4 + ((kk & 31) >> 3)) << 5) + (row & 31)] = v;
     }
 }
 
@@ -615,28 +663,17 @@ __global__ void __launch_bounds__(640, 1)
                 const uint32_t maskv = sb + L::OFF_MASKV + ks * 512 + w * 128;
                 for (int jt = 0; jt < nt; ++jt) {
                     const int ts = g % L::NS;
-                    // this thread's 32 bias values (row j, keys kt*128 + 32w ..), straight from global
-                    // memory (L2-resident: shared by every row i); issued before the waits below
+                    // this thread's 32 bias values (row j, keys kt*128 + 32w ..) from the rearranged
+                    // tiles of pre-pass 1b (L2-resident: shared by every row i; each load of the warp
+                    // covers 512 contiguous bytes); issued before the waits below
                     uint32_t bw[16];
                     {
-                        const int j = jt * 128 + row;
-                        const int k0 = kt * 128 + w * 32;
-                        const __nv_bfloat16* bp = p.bias + b * p.bs0 + h * p.bs1 + static_cast<int64_t>(j) * p.bs2 + k0;
+                        const uint4* bp = p.bias_tiles +
+                                          ((static_cast<int64_t>((b * p.H + h) * nt + jt) * nt + kt) << 11) +
+                                          ((w * 4 + qd) << 7) + lane;
 #pragma unroll
                         for (int c = 0; c < 4; ++c) {
-                            uint4 v = make_uint4(0, 0, 0, 0);
-                            if (j < p.N) {
-                                if (k0 + 8 * c + 8 <= p.N) {
-                                    v = __ldg(reinterpret_cast<const uint4*>(bp + 8 * c));
-                                } else if (k0 + 8 * c < p.N) {  // ragged key tail: element loads, zeros past N
-                                    uint16_t e8[8];
-#pragma unroll
-                                    for (int u = 0; u < 8; ++u)
-                                        e8[u] = (k0 + 8 * c + u < p.N) ? __bfloat16_as_ushort(bp[8 * c + u]) : 0;
-                                    v = make_uint4(e8[0] | (e8[1] << 16), e8[2] | (e8[3] << 16), e8[4] | (e8[5] << 16),
-                                                   e8[6] | (static_cast<uint32_t>(e8[7]) << 16));
-                                }
-                            }
+                            const uint4 v = __ldg(bp + c * 32);
                             bw[4 * c] = v.x;
                             bw[4 * c + 1] = v.y;
                             bw[4 * c + 2] = v.z;
