@@ -261,7 +261,9 @@ struct MainLayout {
                          B_DKVFULL = B_SDPFULL + 8, B_DKVFREE = B_SDPFULL + 9, B_DRAIN = B_SDPFULL + 10,
                          NBAR = B_DRAIN + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
-    static constexpr int SMEM = OFF_MISC + 16;
+    static constexpr int OFF_TRACE = (OFF_MISC + 16 + 7) & ~7;  // phase timing (TRI_TRACE builds only)
+    static constexpr int TRACE_BYTES = (OFF_TRACE + kTraceBytes <= 232448) ? kTraceBytes : 0;
+    static constexpr int SMEM = OFF_TRACE + TRACE_BYTES;
     static_assert(SMEM <= 232448, "shared memory budget");
     // TMEM columns; dQ is one D-wide block per query tile when they all fit
     // (256 + 2D + nt*D <= 512), else a single block drained every tile

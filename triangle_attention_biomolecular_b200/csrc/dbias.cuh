@@ -61,7 +61,9 @@ struct DbLayout {
                          B_SDPFULL = 3 * NS + 2 * NV, B_SDPFREE = B_SDPFULL + 2, B_DRAIN = B_SDPFULL + 4,
                          NBAR = B_DRAIN + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort
-    static constexpr int SMEM = OFF_MISC + 16;
+    static constexpr int OFF_TRACE = (OFF_MISC + 16 + 7) & ~7;  // phase timing (TRI_TRACE builds only)
+    static constexpr int TRACE_BYTES = (OFF_TRACE + kTraceBytes <= 232448) ? kTraceBytes : 0;
+    static constexpr int SMEM = OFF_TRACE + TRACE_BYTES;
     static_assert(SMEM <= 232448, "shared memory budget");
     static_assert(STAGE % 1024 == 0 && QKV_TILE % 1024 == 0, "swizzled tiles need 1 KB alignment");
     static_assert(OFF_BAR % 8 == 0, "mbarrier alignment");

@@ -67,7 +67,9 @@ struct FwdLayout {
                          B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2, B_PVDONE = B_PFULL + 2,
                          B_EXPD = B_PVDONE + 2, B_QFREE = B_EXPD + 2, B_DRAIN = B_QFREE + 1, NBAR = B_DRAIN + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag, mask flags[NS][2]
-    static constexpr int SMEM = OFF_MISC + 16 + NS * 2 * 4;
+    static constexpr int OFF_TRACE = (OFF_MISC + 16 + NS * 2 * 4 + 7) & ~7;  // phase timing (TRI_TRACE builds only)
+    static constexpr int TRACE_BYTES = (OFF_TRACE + kTraceBytes <= 232448) ? kTraceBytes : 0;
+    static constexpr int SMEM = OFF_TRACE + TRACE_BYTES;
     static_assert(SMEM <= 232448, "shared memory budget");
     static_assert(QKV_TILE % 1024 == 0 && STAGE % 1024 == 0, "1 KB tile alignment");
 };
@@ -467,6 +469,7 @@ __global__ void __launch_bounds__(384, 1)
                 const int turn = w == 1 ? gt : gt - 1;
                 if (!mbar_wait_warp(BAR(L::B_EXPD + (1 - w)), turn & 1, wc, 10)) { ok = false; break; }
             }
+            TRI_TP(6)
             // probabilities into packed BF16 registers first; the previous PV may still be
             // reading the P columns
             const float2 l2e = make_float2(LOG2E, LOG2E), nmb = make_float2(-mb, -mb);

@@ -20,19 +20,27 @@ namespace tri {
 __device__ uint32_t g_error_word;
 
 // Optional phase timing (instrumentation only; compiled out unless TRI_TRACE is
-// defined): each warp accumulates clock64() cycles per phase and lane 0 writes
-// them to a buffer of [blocks][12 warps][16 phases].
+// defined): lane 0 of each warp accumulates clock64() cycles per phase in shared
+// memory (TRACE_BYTES at the kernel layout's OFF_TRACE, so that the timing takes
+// no registers from the code it times; global memory where the layout has no room)
+// and writes them at the end to a buffer of [blocks][32 warps][16 phases].
 #ifdef TRI_TRACE
 __device__ unsigned long long* g_trace;
-#define TRI_TRACE_DECL                                  \
-    unsigned long long tri_acc_[16];                    \
-    for (int tri_q_ = 0; tri_q_ < 16; ++tri_q_) tri_acc_[tri_q_] = 0; \
+constexpr int kTraceBytes = 24 * 16 * 8;
+// accumulators of kernels whose layout has no room left for them (slower: global memory)
+__device__ unsigned long long g_trace_spill[256 * 32 * 16];
+#define TRI_TRACE_DECL                                                                                        \
+    unsigned long long* tri_acc_ = (L::TRACE_BYTES > 0)                                                        \
+        ? reinterpret_cast<unsigned long long*>(smem + L::OFF_TRACE) + (threadIdx.x >> 5) * 16                 \
+        : g_trace_spill + ((blockIdx.x % 256) * 32 + (threadIdx.x >> 5)) * 16;                                 \
+    if ((threadIdx.x & 31) == 0)                                                                            \
+        for (int tri_q_ = 0; tri_q_ < 16; ++tri_q_) tri_acc_[tri_q_] = 0;                                  \
     unsigned long long tri_last_ = clock64();
-#define TRI_TP(p)                                       \
-    {                                                   \
-        const unsigned long long tri_t_ = clock64();    \
-        tri_acc_[p] += tri_t_ - tri_last_;              \
-        tri_last_ = tri_t_;                             \
+#define TRI_TP(p)                                                  \
+    {                                                              \
+        const unsigned long long tri_t_ = clock64();               \
+        if ((threadIdx.x & 31) == 0) tri_acc_[p] += tri_t_ - tri_last_; \
+        tri_last_ = tri_t_;                                        \
     }
 #define TRI_TRACE_FLUSH_AT(base)                                                                          \
     {                                                                                                     \
@@ -42,6 +50,7 @@ __device__ unsigned long long* g_trace;
                     tri_acc_[tri_q_];                                                                     \
     }
 #else
+constexpr int kTraceBytes = 0;
 #define TRI_TRACE_DECL
 #define TRI_TP(p)
 #define TRI_TRACE_FLUSH_AT(base)

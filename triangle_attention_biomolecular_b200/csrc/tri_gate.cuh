@@ -59,7 +59,9 @@ struct TriGateLayout {
                          B_AFULL = B_GFREE + 2, B_YFULL = B_AFULL + 1, B_YFREE = B_YFULL + 2, B_DRAIN = B_YFREE + 2,
                          NBAR = B_DRAIN + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-    static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack for 1 KB alignment
+    static constexpr int OFF_TRACE = (OFF_MISC + 16 + 7) & ~7;  // phase timing (TRI_TRACE builds only)
+    static constexpr int TRACE_BYTES = (OFF_TRACE + kTraceBytes + 1024 <= 232448) ? kTraceBytes : 0;
+    static constexpr int SMEM = OFF_TRACE + TRACE_BYTES + 1024;  // + slack for 1 KB alignment
     static constexpr int EPI_WARPS = 8, W_PRODUCER = 8, W_MMA = 9, THREADS = 320;
     static_assert(SMEM <= 232448, "shared memory budget");
 };
@@ -419,7 +421,9 @@ struct TriGateBwdLayout {
                          B_DLFULL = B_A2DONE + 1, B_DZFULL = B_DLFULL + 1, B_BDONE = B_DZFULL + 1,
                          B_ACC = B_BDONE + 1, NBAR = B_ACC + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-    static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack for 1 KB alignment
+    static constexpr int OFF_TRACE = (OFF_MISC + 16 + 7) & ~7;  // phase timing (TRI_TRACE builds only)
+    static constexpr int TRACE_BYTES = (OFF_TRACE + kTraceBytes + 1024 <= 232448) ? kTraceBytes : 0;
+    static constexpr int SMEM = OFF_TRACE + TRACE_BYTES + 1024;  // + slack for 1 KB alignment
     static constexpr int EPI_WARPS = 8, W_PRODUCER = 8, W_MMA = 9, THREADS = 320;
     static constexpr int PARTIAL_FLOATS = 2 * C * C;  // per CTA
     static_assert(SMEM <= 232448, "shared memory budget");
