@@ -533,6 +533,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (!ok) break;
         if (!mbar_wait_warp(BAR(L::B_PVDONE + w), (gt - 1) & 1, wc, 9)) { ok = false; break; }
+        TRI_TP(10)
         {
             tc_fence_after();
             const bool store = (j < p.N) && (w == 0 || t.has1);
@@ -567,6 +568,7 @@ __global__ void __launch_bounds__(384, 1)
                     m_ref + lg2(l) * 0.6931471805599453f;
             }
         }
+        TRI_TP(11)
         }  // items
         TRI_TP(8)
         TRI_TRACE_FLUSH_AT(0)
