@@ -363,12 +363,39 @@ def run_sweep(args):
             e1.record()
             torch.cuda.synchronize()
             return e0.elapsed_time(e1) / n
+        def timed_graph(fn, n):
+            # the same calls captured once into a CUDA graph and replayed: device time
+            # without the per-call host marshalling of the Python binding (tens of
+            # microseconds, which bounds the eager rate at small N)
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                for _ in range(3):
+                    fn()
+            torch.cuda.current_stream().wait_stream(side)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for _ in range(n):
+                    fn()
+            g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            del g
+            return e0.elapsed_time(e1) / n
+
         n_iter = max(5, min(200, int(2e12 / (14.0 * Bn * H * N ** 3 * d))))
         sampler = ClockSampler(0)
         sampler.start()
         time.sleep(0.3)
-        t_f = timed(fwd, n_iter)
-        t_fb = timed(lambda: (fwd(), bwd()), n_iter)
+        t_f_eager = timed(fwd, n_iter)
+        t_fb_eager = timed(lambda: (fwd(), bwd()), n_iter)
+        t_f = timed_graph(fwd, n_iter)
+        t_fb = timed_graph(lambda: (fwd(), bwd()), n_iter)
         clocks = sampler.stop()
         st, word = Bd.tri_attn_device_error(True)
         if st != 0:
@@ -380,6 +407,8 @@ def run_sweep(args):
         fwd_bytes = 5 * pair + Bn * H * N * N * (2 + 4) + Bn * N * N * 4
         line = {"metric": "tri-attn TFLOP/s per workload", "workload": wl.name, "B": Bn, "N": N, "H": H, "d": d,
                 "mask": wl.mask, "orientation": wl.orientation, "iters": n_iter,
+                "timing": "CUDA graph of the calls, replayed (device time); *_eager: back-to-back Python calls",
+                "fwd_ms_eager": round(t_f_eager, 4), "fwd_bwd_ms_eager": round(t_fb_eager, 4),
                 "fwd_ms": round(t_f, 4), "fwd_tflops": round(4.0 * cube / (t_f * 1e-3) / 1e12, 2),
                 "fwd_tflops_effective": round(4.0 * eff / (t_f * 1e-3) / 1e12, 2),
                 "fwd_bwd_ms": round(t_fb, 4), "fwd_bwd_tflops": round(14.0 * cube / (t_fb * 1e-3) / 1e12, 2),

@@ -160,37 +160,27 @@ def _check_tensor(t, name, dtype, dims):
         raise TriAttnError(TRI_ATTN_ERR_SHAPE, f"{name} must have {dims} dims")
 
 
+_I64x5, _I64x4, _I64x3 = ctypes.c_int64 * 5, ctypes.c_int64 * 4, ctypes.c_int64 * 3
+
+
 def t5(t, name="tensor") -> Tensor5:
     import torch
     _check_tensor(t, name, torch.bfloat16, 5)
-    s = Tensor5()
-    s.ptr = t.data_ptr()
-    for a in range(5):
-        s.stride[a] = t.stride(a)
-    return s
+    return Tensor5(t.data_ptr(), _I64x5(*t.stride()))
 
 
 def t4(t, name="bias") -> Tensor4:
     import torch
     _check_tensor(t, name, torch.bfloat16, 4)
-    s = Tensor4()
-    s.ptr = t.data_ptr()
-    for a in range(4):
-        s.stride[a] = t.stride(a)
-    return s
+    return Tensor4(t.data_ptr(), _I64x4(*t.stride()))
 
 
 def mask3(m) -> Mask:
     import torch
-    s = Mask()
     if m is None:
-        s.ptr = None
-        return s
+        return Mask()
     _check_tensor(m, "mask", torch.float32, 3)
-    s.ptr = m.data_ptr()
-    for a in range(3):
-        s.stride[a] = m.stride(a)
-    return s
+    return Mask(m.data_ptr(), _I64x3(*m.stride()))
 
 
 def _stream_handle(stream):
