@@ -237,8 +237,10 @@ __global__ void __launch_bounds__(256) tri_attn_bwd_bias_tiles_kernel(const __nv
 template <int D>
 struct MainLayout {
     // warps 0-15: four softmax warpgroups, warpgroup w owns keys 32w..32w+31 of every
-    // tile; warp 16 producer, warp 17 MMA, 18-19 spare
-    static constexpr int THREADS = 640, SOFTMAX_WARPS = 16, W_PRODUCER = 16, W_MMA = 17;
+    // tile; warp 16 producer, warp 17 issues the gradient MMAs, warp 18 the S and dP
+    // MMAs (so a tile's S/dP never waits in one warp's issue order behind the previous
+    // tile's gradient MMAs), 19 spare
+    static constexpr int THREADS = 640, SOFTMAX_WARPS = 16, W_PRODUCER = 16, W_MMA = 17, W_SMMA = 18;
     static constexpr int KVS = (D == 32) ? 2 : 1;  // K/V buffers
     static constexpr int NS = (D == 32) ? 3 : 2;   // per-tile stages (Q, dO, vectors)
     static constexpr int ROWB = D * 2;
@@ -317,7 +319,7 @@ __global__ void __launch_bounds__(640, 1)
         mbar_init(BAR(L::B_DQFREE), L::SOFTMAX_WARPS);
         mbar_init(BAR(L::B_DKVFULL), 1);
         mbar_init(BAR(L::B_DKVFREE), L::SOFTMAX_WARPS);
-        mbar_init(BAR(L::B_DRAIN), 1);
+        mbar_init(BAR(L::B_DRAIN), 2);  // both MMA-issuing warps
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -405,8 +407,8 @@ __global__ void __launch_bounds__(640, 1)
             for (int s = 0; s < L::NS; ++s)
                 if (armed_t[s] > 0) drain_wait(BAR(L::B_TFULL + s), (armed_t[s] - 1) & 1, 100000000ull);
         }
-    } else if (warp == L::W_MMA) {
-        // =========================== MMA issuer =============================
+    } else if (warp == L::W_MMA || warp == L::W_SMMA) {
+        // =========================== MMA issuers ============================
         regs_shrink640();
         const bool leader = elect_one();
         if (!aborted_early) {
@@ -424,103 +426,113 @@ __global__ void __launch_bounds__(640, 1)
             const uint64_t d_dsmn = smem_desc(sb + L::OFF_PDS + L::PT_TILE, L::PT_TILE / 2, 1024, SWZ_128B);
             const uint64_t d_dsk = smem_desc(sb + L::OFF_PDS + L::PT_TILE, 16, 1024, SWZ_128B);
             TRI_TRACE_DECL
-            struct Pending {
-                int g, ts, ks, jt, kt, kcount;
-                bool valid;
-            } pend{0, 0, 0, 0, 0, 0, false};
             bool ok = true;
-            int ep_count = 0;  // dQ epilogue tiles issued so far
-            auto issue_grads = [&](const Pending& t) -> bool {
-                // a dQ epilogue tile: every tile (single block) or the last key tile of a query tile
-                const bool ep = !p.dq_tmem || t.kt == nt - 1;
-                TRI_TP(7)
-                const int pb = t.g & 1;  // P/dS buffer of this tile
-                if (!mbar_wait_warp(BAR(L::B_PDSFULL + pb), (t.g >> 1) & 1, wc, 3)) return false;
-                TRI_TP(4)
-                // the previous epilogue has read its dQ block (keeps DQ_FULL at most one phase ahead,
-                // and before a new problem overwrites the last query tile's block)
-                const bool reuse = p.dq_tmem && t.kt == 0 && t.jt == nt - 1;
-                if ((ep || reuse) && ep_count > 0 && !mbar_wait_warp(BAR(L::B_DQFREE), (ep_count - 1) & 1, wc, 4))
-                    return false;
-                TRI_TP(5)
-                if (t.jt == 0 && t.kcount > 0 && !mbar_wait_warp(BAR(L::B_DKVFREE), (t.kcount - 1) & 1, wc, 5))
-                    return false;
-                TRI_TP(6)
-                tc_fence_after();
-                const uint32_t toff = t.ts * L::T_STAGE;
-                const uint64_t bdo = desc_add(d_tmn, toff + L::QKV_TILE), bq = desc_add(d_tmn, toff);
-                const uint64_t bk = desc_add(d_kvmn, t.ks * 2 * L::QKV_TILE);
-                const uint32_t dq_col = p.dq_tmem ? L::T_DQ + t.jt * D : L::T_DQ;
-                const bool dq_acc = p.dq_tmem && t.kt > 0;
-                if (leader) {
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {  // contraction over 128 queries
-                    const uint32_t acc = (t.jt > 0 || kk > 0) ? 1u : 0u;
-                    // A = P^T / dS^T: MN-major, 64-element chunks 16 KB apart, 8-row groups 1 KB apart
-                    mma_ss(tmem + L::T_DV, desc_add(d_pmn, pb * L::PDS_BUF + kk * 2048), desc_add(bdo, kk * 16 * L::ROWB),
-                           IDESC_G, acc);
-                    mma_ss(tmem + L::T_DK, desc_add(d_dsmn, pb * L::PDS_BUF + kk * 2048), desc_add(bq, kk * 16 * L::ROWB),
-                           IDESC_G, acc);
-                }
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)  // contraction over 128 keys; A = dS rows j, K-major halves 16 KB apart
-                    mma_ss(tmem + dq_col, desc_add(d_dsk, pb * L::PDS_BUF + (kk >> 2) * (L::PT_TILE / 2) + (kk & 3) * 32),
-                           desc_add(bk, kk * 16 * L::ROWB), IDESC_Q, (dq_acc || kk > 0) ? 1u : 0u);
-                mma_commit(BAR(L::B_PDSFREE + pb));
-                mma_commit(BAR(L::B_TEMPTY + t.ts));
-                if (ep) mma_commit(BAR(L::B_DQFULL));
-                if (t.jt == nt - 1) {
-                    mma_commit(BAR(L::B_DKVFULL));
-                    mma_commit(BAR(L::B_KVEMPTY + t.ks));
-                }
-                }
-                __syncwarp();
-                if (ep) ++ep_count;
-                return true;
-            };
-            int gk = 0, g = 0;
-            for (int pr = blockIdx.x; ok && pr < problems; pr += gridDim.x) {
-                for (int kt = 0; ok && kt < nt; ++kt) {
-                    const int ks = gk % L::KVS;
-                    if (L::KVS == 1 && pend.valid && pend.jt == nt - 1) {
-                        // the single K/V buffer is released only by this tile's gradients
-                        if (!(ok = issue_grads(pend))) break;
-                        pend.valid = false;
-                    }
-                    TRI_TP(7)
-                    if (!mbar_wait_warp(BAR(L::B_KVFULL + ks), (gk / L::KVS) & 1, wc, 6)) { ok = false; break; }
-                    TRI_TP(0)
-                    const uint64_t kd = desc_add(d_kvk, ks * 2 * L::QKV_TILE);
-                    const uint64_t vd = desc_add(kd, L::QKV_TILE);
-                    for (int jt = 0; jt < nt; ++jt) {
-                        const int ts = g % L::NS;
+            if (warp == L::W_SMMA) {
+                // ---- S = Q K^T and dP = dO V^T of every tile, as soon as the softmax warps have
+                // taken the previous tile's columns ----
+                int gk = 0, g = 0;
+                for (int pr = blockIdx.x; ok && pr < problems; pr += gridDim.x) {
+                    for (int kt = 0; ok && kt < nt; ++kt) {
+                        const int ks = gk % L::KVS;
                         TRI_TP(7)
-                        if (!mbar_wait_warp(BAR(L::B_TFULL + ts), (g / L::NS) & 1, wc, 7)) { ok = false; break; }
-                        TRI_TP(1)
-                        if (g > 0 && !mbar_wait_warp(BAR(L::B_SDPFREE), (g - 1) & 1, wc, 8)) { ok = false; break; }
-                        TRI_TP(2)
-                        tc_fence_after();
-                        const uint64_t qd = desc_add(d_tk, ts * L::T_STAGE), dod = desc_add(qd, L::QKV_TILE);
-                        if (leader) {
+                        if (!mbar_wait_warp(BAR(L::B_KVFULL + ks), (gk / L::KVS) & 1, wc, 6)) { ok = false; break; }
+                        TRI_TP(0)
+                        const uint64_t kd = desc_add(d_kvk, ks * 2 * L::QKV_TILE);
+                        const uint64_t vd = desc_add(kd, L::QKV_TILE);
+                        for (int jt = 0; jt < nt; ++jt) {
+                            const int ts = g % L::NS;
+                            if (!mbar_wait_warp(BAR(L::B_TFULL + ts), (g / L::NS) & 1, wc, 7)) { ok = false; break; }
+                            TRI_TP(1)
+                            if (g > 0 && !mbar_wait_warp(BAR(L::B_SDPFREE), (g - 1) & 1, wc, 8)) { ok = false; break; }
+                            TRI_TP(2)
+                            tc_fence_after();
+                            const uint64_t qd = desc_add(d_tk, ts * L::T_STAGE), dod = desc_add(qd, L::QKV_TILE);
+                            if (leader) {
 #pragma unroll
-                            for (int kk = 0; kk < D / 16; ++kk) {
-                                mma_ss(tmem + L::T_S, desc_add(qd, kk * 32), desc_add(kd, kk * 32), IDESC_S, kk > 0 ? 1u : 0u);
-                                mma_ss(tmem + L::T_DP, desc_add(dod, kk * 32), desc_add(vd, kk * 32), IDESC_S, kk > 0 ? 1u : 0u);
+                                for (int kk = 0; kk < D / 16; ++kk) {
+                                    mma_ss(tmem + L::T_S, desc_add(qd, kk * 32), desc_add(kd, kk * 32), IDESC_S,
+                                           kk > 0 ? 1u : 0u);
+                                    mma_ss(tmem + L::T_DP, desc_add(dod, kk * 32), desc_add(vd, kk * 32), IDESC_S,
+                                           kk > 0 ? 1u : 0u);
+                                }
+                                mma_commit(BAR(L::B_SDPFULL));
                             }
-                            mma_commit(BAR(L::B_SDPFULL));
+                            __syncwarp();
+                            TRI_TP(3)
+                            ++g;
                         }
-                        __syncwarp();
-                        TRI_TP(3)
-                        if (pend.valid) {
-                            if (!(ok = issue_grads(pend))) break;
-                        }
-                        pend = Pending{g, ts, ks, jt, kt, gk, true};
-                        ++g;
+                        ++gk;
                     }
-                    ++gk;
+                }
+            } else {
+                // ---- dV += P^T dO, dK += dS^T Q, dQ (+)= dS K of every tile once its P and dS are
+                // in SMEM.  Stages, K/V buffers and the P/dS buffer are released by this warp's
+                // commits; they also cover the S/dP products of the same tile, which completed
+                // before the softmax warps could store its P and dS ----
+                int ep_count = 0;  // dQ epilogue tiles issued so far
+                int gk = 0, g = 0;
+                for (int pr = blockIdx.x; ok && pr < problems; pr += gridDim.x) {
+                    for (int kt = 0; ok && kt < nt; ++kt) {
+                        const int ks = gk % L::KVS;
+                        for (int jt = 0; jt < nt; ++jt) {
+                            const int ts = g % L::NS;
+                            // a dQ epilogue tile: every tile (single block) or the last key tile of a query tile
+                            const bool ep = !p.dq_tmem || kt == nt - 1;
+                            TRI_TP(7)
+                            const int pb = g & 1;  // P/dS buffer of this tile
+                            if (!mbar_wait_warp(BAR(L::B_PDSFULL + pb), (g >> 1) & 1, wc, 3)) { ok = false; break; }
+                            TRI_TP(4)
+                            // the previous epilogue has read its dQ block (keeps DQ_FULL at most one phase
+                            // ahead, and before a new problem overwrites the last query tile's block)
+                            const bool reuse = p.dq_tmem && kt == 0 && jt == nt - 1;
+                            if ((ep || reuse) && ep_count > 0 &&
+                                !mbar_wait_warp(BAR(L::B_DQFREE), (ep_count - 1) & 1, wc, 4)) {
+                                ok = false;
+                                break;
+                            }
+                            TRI_TP(5)
+                            if (jt == 0 && gk > 0 && !mbar_wait_warp(BAR(L::B_DKVFREE), (gk - 1) & 1, wc, 5)) {
+                                ok = false;
+                                break;
+                            }
+                            TRI_TP(6)
+                            tc_fence_after();
+                            const uint32_t toff = ts * L::T_STAGE;
+                            const uint64_t bdo = desc_add(d_tmn, toff + L::QKV_TILE), bq = desc_add(d_tmn, toff);
+                            const uint64_t bk = desc_add(d_kvmn, ks * 2 * L::QKV_TILE);
+                            const uint32_t dq_col = p.dq_tmem ? L::T_DQ + jt * D : L::T_DQ;
+                            const bool dq_acc = p.dq_tmem && kt > 0;
+                            if (leader) {
+#pragma unroll
+                                for (int kk = 0; kk < 8; ++kk) {  // contraction over 128 queries
+                                    const uint32_t acc = (jt > 0 || kk > 0) ? 1u : 0u;
+                                    // A = P^T / dS^T: MN-major, 64-element chunks 16 KB apart, 8-row groups 1 KB apart
+                                    mma_ss(tmem + L::T_DV, desc_add(d_pmn, pb * L::PDS_BUF + kk * 2048),
+                                           desc_add(bdo, kk * 16 * L::ROWB), IDESC_G, acc);
+                                    mma_ss(tmem + L::T_DK, desc_add(d_dsmn, pb * L::PDS_BUF + kk * 2048),
+                                           desc_add(bq, kk * 16 * L::ROWB), IDESC_G, acc);
+                                }
+#pragma unroll
+                                for (int kk = 0; kk < 8; ++kk)  // contraction over 128 keys; A = dS rows j, K-major halves 16 KB apart
+                                    mma_ss(tmem + dq_col,
+                                           desc_add(d_dsk, pb * L::PDS_BUF + (kk >> 2) * (L::PT_TILE / 2) + (kk & 3) * 32),
+                                           desc_add(bk, kk * 16 * L::ROWB), IDESC_Q, (dq_acc || kk > 0) ? 1u : 0u);
+                                mma_commit(BAR(L::B_PDSFREE + pb));
+                                mma_commit(BAR(L::B_TEMPTY + ts));
+                                if (ep) mma_commit(BAR(L::B_DQFULL));
+                                if (jt == nt - 1) {
+                                    mma_commit(BAR(L::B_DKVFULL));
+                                    mma_commit(BAR(L::B_KVEMPTY + ks));
+                                }
+                            }
+                            __syncwarp();
+                            if (ep) ++ep_count;
+                            ++g;
+                        }
+                        ++gk;
+                    }
                 }
             }
-            if (ok && pend.valid) ok = issue_grads(pend);
             TRI_TP(7)
             TRI_TRACE_FLUSH_AT(20000)
             if (leader) mma_commit(BAR(L::B_DRAIN));
