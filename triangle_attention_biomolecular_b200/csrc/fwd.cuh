@@ -14,9 +14,10 @@
 //
 // B200 mapping:
 //  * one CTA = 384 threads: warps 0-3 softmax for row i0, warps 4-7 softmax
-//    for row i1, warp 8 TMA producer, warp 9 MMA issuer (one thread), warps
-//    10-11 idle; the last warpgroup hands most of its registers to the
-//    softmax warpgroups;
+//    for row i1, warp 8 TMA producer, warp 9 issues the PV products, warp 10
+//    the S products (so an S never waits in one warp's issue order behind a
+//    PV that waits for the other row's probabilities), warp 11 idle; the last
+//    warpgroup hands most of its registers to the softmax warpgroups;
 //  * both rows share every bias tile (the bias is the same for all rows i),
 //    so each 32 KB bias tile crosses L2->SMEM once per two rows;
 //  * TMEM (512 columns): per warpgroup w, S at 256w, P (BF16 pairs) at
@@ -148,7 +149,7 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(BAR(L::B_EXPD + w), 4);
         }
         mbar_init(BAR(L::B_QFREE), 1);
-        mbar_init(BAR(L::B_DRAIN), 1);
+        mbar_init(BAR(L::B_DRAIN), 2);  // both MMA-issuing warps
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -257,8 +258,8 @@ __global__ void __launch_bounds__(384, 1)
             for (int s = 0; s < L::NS; ++s)
                 if (armed[s] > 0) drain_wait(BAR(L::B_FULL + s), (armed[s] - 1) & 1, 100000000ull);
         }
-    } else if (warp == 9) {
-        // =========================== MMA issuer =============================
+    } else if (warp == 9 || warp == 10) {
+        // =========================== MMA issuers ============================
         regs_shrink();
         const bool leader = elect_one();
         if (!aborted_early) {
@@ -270,81 +271,76 @@ __global__ void __launch_bounds__(384, 1)
             const uint64_t dq0 = smem_desc(sb + L::OFF_Q, 16, SBO, SW);
             const uint64_t dst0 = smem_desc(sb + L::OFF_STAGES, 16, SBO, SW);          // K-major rows
             const uint64_t dvt0 = smem_desc(sb + L::OFF_STAGES, L::QKV_TILE, SBO, SW);  // MN-major rows
-            auto issue_pv = [&](int w, int s, int ktile) {
-                const uint64_t vd = desc_add(dvt0, s * L::STAGE + (w ? L::OFF_V1 : L::OFF_V0));
-                const uint32_t tS = tmem + w * 256;
-                if (leader) {
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ts(tS + 192, tS + 128 + kk * 8, desc_add(vd, kk * 16 * L::ROWB), IDESC_PV,
-                               (ktile > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(BAR(L::B_PVDONE + w));
-                }
-                __syncwarp();
-            };
             TRI_TRACE_DECL
             bool ok = true;
             int gs = 0, gt = 0, it = 0;  // stages consumed, tiles, items (all continue across items)
-            for (int item = blockIdx.x; ok && item < items; item += gridDim.x, ++it) {
-                if (!mbar_wait_warp(BAR(L::B_Q), it & 1, wc, 2)) { ok = false; break; }
-                TRI_TP(9)
-                for (int kt = 0; kt < nkt; ++kt, ++gs, ++gt) {
-                    const int s = gs % L::NS;
-                    TRI_TP(4)
-                    if (!mbar_wait_warp(BAR(L::B_FULL + s), (gs / L::NS) & 1, wc, 3)) { ok = false; break; }
-                    TRI_TP(0)
-                    tc_fence_after();
+            if (warp == 10) {
+                // ---- S = Q K^T for both rows of every key tile ----
+                for (int item = blockIdx.x; ok && item < items; item += gridDim.x, ++it) {
+                    if (!mbar_wait_warp(BAR(L::B_Q), it & 1, wc, 2)) { ok = false; break; }
+                    TRI_TP(9)
+                    for (int kt = 0; kt < nkt; ++kt, ++gs, ++gt) {
+                        const int s = gs % L::NS;
+                        TRI_TP(4)
+                        if (!mbar_wait_warp(BAR(L::B_FULL + s), (gs / L::NS) & 1, wc, 3)) { ok = false; break; }
+                        TRI_TP(0)
+                        tc_fence_after();
 #pragma unroll
-                    for (int w = 0; w < 2; ++w) {
-                        if (gt > 0) {
-                            TRI_TP(4)
-                            if (!mbar_wait_warp(BAR(L::B_SFREE + w), (gt - 1) & 1, wc, 4)) { ok = false; break; }
-                            TRI_TP(1)
-                            tc_fence_after();
-                        }
-                        const uint64_t qd = desc_add(dq0, w * L::QKV_TILE);
-                        const uint64_t kd = desc_add(dst0, s * L::STAGE + (w ? L::OFF_K1 : L::OFF_K0));
-                        if (leader) {
+                        for (int w = 0; w < 2; ++w) {
+                            if (gt > 0) {
+                                TRI_TP(4)
+                                if (!mbar_wait_warp(BAR(L::B_SFREE + w), (gt - 1) & 1, wc, 4)) { ok = false; break; }
+                                TRI_TP(1)
+                                tc_fence_after();
+                            }
+                            const uint64_t qd = desc_add(dq0, w * L::QKV_TILE);
+                            const uint64_t kd = desc_add(dst0, s * L::STAGE + (w ? L::OFF_K1 : L::OFF_K0));
+                            if (leader) {
 #pragma unroll
-                            for (int kk = 0; kk < D / 16; ++kk)
-                                mma_ss(tmem + w * 256, desc_add(qd, kk * 32), desc_add(kd, kk * 32), IDESC_QK,
-                                       kk > 0 ? 1u : 0u);
-                            mma_commit(BAR(L::B_SFULL + w));
+                                for (int kk = 0; kk < D / 16; ++kk)
+                                    mma_ss(tmem + w * 256, desc_add(qd, kk * 32), desc_add(kd, kk * 32), IDESC_QK,
+                                           kk > 0 ? 1u : 0u);
+                                mma_commit(BAR(L::B_SFULL + w));
+                            }
+                            __syncwarp();
                         }
-                        __syncwarp();
+                        if (!ok) break;
+                        if (kt == nkt - 1) {  // the item's last S products: Q is free once they finish
+                            if (leader) mma_commit(BAR(L::B_QFREE));
+                            __syncwarp();
+                        }
                     }
-                    if (!ok) break;
-                    if (kt == nkt - 1) {  // the item's last S products: Q is free once they finish
-                        if (leader) mma_commit(BAR(L::B_QFREE));
-                        __syncwarp();
-                    }
-                    if (kt > 0) {
-                        const int sp = (gs - 1) % L::NS;
+                }
+            } else {
+                // ---- O += P V for both rows of every key tile; the stage (K, V, bias, mask) goes
+                // back to the producer after them (its S products completed before the
+                // probabilities they gave were written) ----
+                for (int item = blockIdx.x; ok && item < items; item += gridDim.x, ++it) {
+                    for (int kt = 0; kt < nkt; ++kt, ++gs, ++gt) {
+                        const int s = gs % L::NS;
+                        const uint64_t vbase = desc_add(dvt0, s * L::STAGE);
 #pragma unroll
                         for (int w = 0; w < 2; ++w) {
                             TRI_TP(4)
-                            if (!mbar_wait_warp(BAR(L::B_PFULL + w), (gt - 1) & 1, wc, 5)) { ok = false; break; }
+                            if (!mbar_wait_warp(BAR(L::B_PFULL + w), gt & 1, wc, 5)) { ok = false; break; }
                             TRI_TP(2)
                             tc_fence_after();
-                            issue_pv(w, sp, kt - 1);
+                            const uint64_t vd = desc_add(vbase, w ? L::OFF_V1 : L::OFF_V0);
+                            const uint32_t tS = tmem + w * 256;
+                            if (leader) {
+#pragma unroll
+                                for (int kk = 0; kk < 8; ++kk)
+                                    mma_ts(tS + 192, tS + 128 + kk * 8, desc_add(vd, kk * 16 * L::ROWB), IDESC_PV,
+                                           (kt > 0 || kk > 0) ? 1u : 0u);
+                                mma_commit(BAR(L::B_PVDONE + w));
+                            }
+                            __syncwarp();
                         }
                         if (!ok) break;
-                        if (leader) mma_commit(BAR(L::B_EMPTY + sp));
+                        if (leader) mma_commit(BAR(L::B_EMPTY + s));
                         __syncwarp();
                     }
                 }
-                if (!ok) break;
-                // the item's last PV
-                const int sp = (gs - 1) % L::NS;
-#pragma unroll
-                for (int w = 0; w < 2; ++w) {
-                    if (!mbar_wait_warp(BAR(L::B_PFULL + w), (gt - 1) & 1, wc, 5)) { ok = false; break; }
-                    tc_fence_after();
-                    issue_pv(w, sp, nkt - 1);
-                }
-                if (!ok) break;
-                if (leader) mma_commit(BAR(L::B_EMPTY + sp));
-                __syncwarp();
             }
             TRI_TP(5)
             TRI_TRACE_FLUSH_AT(0)
@@ -354,8 +350,8 @@ __global__ void __launch_bounds__(384, 1)
             drain_wait(BAR(L::B_DRAIN), 0, 100000000ull);
         }
         __syncwarp();
-    } else if (warp >= 10) {
-        regs_shrink();  // spare warps of the last warpgroup
+    } else if (warp >= 11) {
+        regs_shrink();  // spare warp of the last warpgroup
     } else {
         regs_grow();
         if (!aborted_early) {
