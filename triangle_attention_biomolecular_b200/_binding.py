@@ -10,6 +10,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+import struct
 import threading
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -83,6 +84,15 @@ class BwdArgs(ctypes.Structure):
     _fields_ = [("f", FwdArgs), ("dout", Tensor5), ("dq", Tensor5), ("dk", Tensor5), ("dv", Tensor5),
                 ("dbias", Tensor4), ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
                 ("flags", ctypes.c_uint)]
+
+
+# The same two argument blocks as flat little-endian layouts (explicit padding), so a
+# call fills one buffer with a single pack instead of building a ctypes structure per
+# tensor; checked against the ctypes structures above at import.
+_FWD_PACK = struct.Struct("<4if4x" + "Q5q" * 3 + "Q4q" + "Q3q" + "Q5q" * 2 + "Q")
+_BWD_TAIL = struct.Struct("<" + "Q5q" * 4 + "Q4q" + "QQi4x")
+assert _FWD_PACK.size == ctypes.sizeof(FwdArgs) and FwdArgs.lse.offset == _FWD_PACK.size - 8
+assert _FWD_PACK.size + _BWD_TAIL.size == ctypes.sizeof(BwdArgs) and BwdArgs.dout.offset == _FWD_PACK.size
 
 
 _lib = None
@@ -192,7 +202,8 @@ def _stream_handle(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def fwd_args(q, k, v, bias, mask, o, resid, lse, scale: float = 0.0, rows_ok: bool = False) -> FwdArgs:
+def fwd_args(q, k, v, bias, mask, o, resid, lse, scale: float = 0.0, rows_ok: bool = False,
+             _room: bool = False) -> FwdArgs:
     """Pair tensors [B,R,N,H,d]: R = N for the whole problem; with rows_ok, R <= N rows
     of a row shard (views starting at its first row), lse [B,H,R,N], mask [B,R,N]."""
     import torch
@@ -209,15 +220,32 @@ def fwd_args(q, k, v, bias, mask, o, resid, lse, scale: float = 0.0, rows_ok: bo
     _check_tensor(lse, "lse", torch.float32, 4)
     if tuple(lse.shape) != (B, H, R, N) or not lse.is_contiguous():
         raise TriAttnError(TRI_ATTN_ERR_SHAPE, "lse must be a contiguous [B,H,N,N] float32 tensor")
-    a = FwdArgs()
-    a.B, a.N, a.H, a.d = B, N, H, d
-    a.scale = float(scale)
-    a.q, a.k, a.v = t5(q, "q"), t5(k, "k"), t5(v, "v")
-    a.bias = t4(bias)
-    a.mask = mask3(mask)
-    a.o, a.resid = t5(o, "o"), t5(resid, "resid")
-    a.lse = lse.data_ptr()
-    return a
+    buf = bytearray(ctypes.sizeof(BwdArgs) if _room else _FWD_PACK.size)
+    _pack_fwd(buf, B, N, H, d, scale, q, k, v, bias, mask, o, resid, lse)
+    return buf if _room else FwdArgs.from_buffer(buf)
+
+
+def _v5(t, name):
+    import torch
+    _check_tensor(t, name, torch.bfloat16, 5)
+    return (t.data_ptr(), *t.stride())
+
+
+def _v4(t, name):
+    import torch
+    _check_tensor(t, name, torch.bfloat16, 4)
+    return (t.data_ptr(), *t.stride())
+
+
+def _pack_fwd(buf, B, N, H, d, scale, q, k, v, bias, mask, o, resid, lse):
+    import torch
+    if mask is None:
+        vm = (0, 0, 0, 0)
+    else:
+        _check_tensor(mask, "mask", torch.float32, 3)
+        vm = (mask.data_ptr(), *mask.stride())
+    _FWD_PACK.pack_into(buf, 0, B, N, H, d, float(scale), *_v5(q, "q"), *_v5(k, "k"), *_v5(v, "v"),
+                        *_v4(bias, "bias"), *vm, *_v5(o, "o"), *_v5(resid, "resid"), lse.data_ptr())
 
 
 # ---------------------------------------------------------------------------
@@ -247,24 +275,21 @@ def tri_attn_fwd(q, k, v, bias, mask, o, resid, lse, scale: float = 0.0, stream=
 def bwd_args(q, k, v, bias, mask, o, resid, lse, dout, dq, dk, dv, dbias, workspace,
              scale: float = 0.0, flags: int = 0, rows_ok: bool = False) -> BwdArgs:
     import torch
-    a = BwdArgs()
-    a.f = fwd_args(q, k, v, bias, mask, o, resid, lse, scale, rows_ok)
-    shape = tuple(q.shape)
+    buf = fwd_args(q, k, v, bias, mask, o, resid, lse, scale, rows_ok, _room=True)
+    shape = q.shape
     for name, t in (("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv)):
-        if tuple(t.shape) != shape:
-            raise TriAttnError(TRI_ATTN_ERR_SHAPE, f"{name} shape {tuple(t.shape)} != {shape}")
-    a.dout = t5(dout, "dout")
-    a.dq, a.dk, a.dv = t5(dq, "dq"), t5(dk, "dk"), t5(dv, "dv")
-    if dbias is not None:
-        a.dbias = t4(dbias, "dbias")
+        if t.shape != shape:
+            raise TriAttnError(TRI_ATTN_ERR_SHAPE, f"{name} shape {tuple(t.shape)} != {tuple(shape)}")
+    vb = (0, 0, 0, 0, 0) if dbias is None else _v4(dbias, "dbias")
     if workspace is None:
-        a.workspace, a.workspace_bytes = None, 0
+        ws = (0, 0)
     else:
         if workspace.dtype != torch.uint8:
             raise TriAttnError(TRI_ATTN_ERR_DTYPE, "workspace must be a uint8 tensor")
-        a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel()
-    a.flags = int(flags)
-    return a
+        ws = (workspace.data_ptr(), workspace.numel())
+    _BWD_TAIL.pack_into(buf, _FWD_PACK.size, *_v5(dout, "dout"), *_v5(dq, "dq"), *_v5(dk, "dk"), *_v5(dv, "dv"),
+                        *vb, *ws, int(flags))
+    return BwdArgs.from_buffer(buf)
 
 
 def tri_attn_bwd(q, k, v, bias, mask, o, resid, lse, dout, dq, dk, dv, dbias, workspace,
