@@ -305,22 +305,15 @@ __global__ void __launch_bounds__(640, 1)
         const int j = jt * 128 + row;
         const float c2 = p.scale * LOG2E;
         // this thread's 32 bias values (row j, keys kt*128 + 32w ..), log2 units, kept in
-        // shared memory: a row is 512 B = 32 chunks of 16 B; chunk w*8+c sits at
-        // w*8 + (c xor (row & 7)), so eight consecutive rows hit eight different bank groups
-        const uint32_t brow = sb + L::OFF_BIAS + row * 512 + w * 128;
+        // registers for the whole row walk (the tile is fixed; S' and dP' are taken from TMEM
+        // 16 keys at a time, which leaves room for them)
+        float bl[32];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            float v[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int k = kt * 128 + w * 32 + 4 * c + e;
-                float bv = 0.f;
-                if (j < p.N && k < p.N)
-                    bv = __bfloat162float(bias[b * bs0 + h * bs1 + static_cast<int64_t>(j) * bs2 + k]);
-                v[e] = bv * LOG2E;
-            }
-            sts128(brow + ((c ^ (row & 7)) << 4),
-                   make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]), __float_as_uint(v[3])));
+        for (int e = 0; e < 32; ++e) {
+            const int k = kt * 128 + w * 32 + e;
+            float bv = 0.f;
+            if (j < p.N && k < p.N) bv = __bfloat162float(bias[b * bs0 + h * bs1 + static_cast<int64_t>(j) * bs2 + k]);
+            bl[e] = bv * LOG2E;
         }
         float acc[32];
 #pragma unroll
@@ -341,37 +334,44 @@ __global__ void __launch_bounds__(640, 1)
             // dS = p dP', p = 2^(c S' + bias [+ mask]), summed over rows
             auto row_step = [&](auto masked) {
                 constexpr bool kMasked = decltype(masked)::value;
-                // all 32 keys of S' and dP' behind one TMEM wait
-                uint32_t sv[32], dv[32];
-                tmem_ld32(tl + x * 256 + w * 32, sv);
-                tmem_ld32(tl + x * 256 + 128 + w * 32, dv);
-                tmem_wait_ld();
-                reg_fence32(sv);
-                reg_fence32(dv);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(BAR(L::B_SDPFREE + x));
+                // S' and dP' of this warpgroup's 32 keys, 16 keys at a time; the columns go back
+                // to the MMA warp once the second half is in registers
 #pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                    const float4 bq = lds128f(brow + ((cc ^ (row & 7)) << 4));
-                    float2 b01 = make_float2(bq.x, bq.y), b23 = make_float2(bq.z, bq.w);
-                    if constexpr (kMasked) {
-                        const float4 mq = lds128f(ma + cc * 16);
-                        b01 = fadd2(b01, make_float2(mq.x, mq.y));
-                        b23 = fadd2(b23, make_float2(mq.z, mq.w));
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t sv[16], dv[16];
+                    tmem_ld16(tl + x * 256 + w * 32 + hf * 16, sv);
+                    tmem_ld16(tl + x * 256 + 128 + w * 32 + hf * 16, dv);
+                    tmem_wait_ld();
+                    reg_fence16(sv);
+                    reg_fence16(dv);
+                    if (hf == 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(BAR(L::B_SDPFREE + x));
                     }
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int xl = 4 * cc + 2 * e;
-                        const float2 y = ffma2(make_float2(__uint_as_float(sv[xl]), __uint_as_float(sv[xl + 1])),
-                                               c22, e ? b23 : b01);
-                        const int pair = (xl >> 1) & 7;  // position of this pair within eight
-                        const float2 pv = (!kMasked && pair < FMA_PAIRS) ? ex2_fma2(y)
-                                                                         : make_float2(ex2(y.x), ex2(y.y));
-                        const float2 a = ffma2(pv, make_float2(__uint_as_float(dv[xl]), __uint_as_float(dv[xl + 1])),
-                                               make_float2(acc[xl], acc[xl + 1]));
-                        acc[xl] = a.x;
-                        acc[xl + 1] = a.y;
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const int cc = 4 * hf + c4;  // 4-key chunk of the thread's 32 keys
+                        float2 b01 = make_float2(bl[4 * cc], bl[4 * cc + 1]), b23 = make_float2(bl[4 * cc + 2], bl[4 * cc + 3]);
+                        if constexpr (kMasked) {
+                            const float4 mq = lds128f(ma + cc * 16);
+                            b01 = fadd2(b01, make_float2(mq.x, mq.y));
+                            b23 = fadd2(b23, make_float2(mq.z, mq.w));
+                        }
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int xh = 4 * c4 + 2 * e;  // within the half
+                            const int xl = 4 * cc + 2 * e;  // within the thread's 32 keys
+                            const float2 y = ffma2(make_float2(__uint_as_float(sv[xh]), __uint_as_float(sv[xh + 1])),
+                                                   c22, e ? b23 : b01);
+                            const int pair = (xl >> 1) & 7;  // position of this pair within eight
+                            const float2 pv = (!kMasked && pair < FMA_PAIRS) ? ex2_fma2(y)
+                                                                             : make_float2(ex2(y.x), ex2(y.y));
+                            const float2 a = ffma2(pv, make_float2(__uint_as_float(dv[xh]), __uint_as_float(dv[xh + 1])),
+                                                   make_float2(acc[xl], acc[xl + 1]));
+                            acc[xl] = a.x;
+                            acc[xl + 1] = a.y;
+                        }
                     }
                 }
             };
