@@ -16,7 +16,9 @@
 // products are exact and accumulate in FP32).  Then per score, in base 2,
 //     p = 2^(c S' + bias log2 e [+ mask log2 e]),  c = scale log2 e,
 //     acc += p * dP'                                   (= dS)
-// i.e. two packed FP32 instructions and one exponential per pair of scores.
+// i.e. two packed FP32 instructions and one exponential per pair of scores.  The
+// tile's bias (log2 units) stays in each softmax thread's registers for the whole
+// row walk, and S', dP' come from TMEM 16 keys at a time to leave room for it.
 //
 // Roles (640 threads): warps 0-15 four softmax warpgroups (warpgroup w owns
 // keys 32w..32w+31 of the tile, warp%4 the TMEM lane quarter); warp 16 TMA
@@ -48,8 +50,7 @@ struct DbLayout {
     static constexpr int OFF_AL = 4 * QKV_TILE, OFF_AD = OFF_AL + AUG_TILE;
     static constexpr int STAGE = 4 * QKV_TILE + 2 * AUG_TILE;
     static constexpr int THREADS = 640, SOFTMAX_WARPS = 16, W_PRODUCER = 16, W_MMA = 17, W_AUG = 18;
-    static constexpr int OFF_BIAS = NS * STAGE;             // [128 rows][128 keys] fp32 log2 units, swizzled
-    static constexpr int OFF_ONES = OFF_BIAS + 128 * 128 * 4;  // B block of ones (keys x 16), AUG layout
+    static constexpr int OFF_ONES = NS * STAGE;  // B block of ones (keys x 16), AUG layout
     // per-row vectors, in a deeper ring of their own so that a row's tiles are
     // released as soon as its products finish: lse*log2e 128, D 128,
     // mask*log2e 128 (fp32), key-tile flags 32 (int)
