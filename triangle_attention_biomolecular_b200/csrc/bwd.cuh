@@ -13,12 +13,16 @@
 // row).  A CTA cannot keep accumulators for all three on chip at N=768 (TMEM
 // holds 128 x 512 FP32), so the work is split:
 //
-//  1. tri_attn_bwd_prep_kernel: D[b,h,i,j] = sum_c dout * (o + resid), FP32.
+//  1. tri_attn_bwd_prep_kernel: D[b,h,i,j] = sum_c dout * (o + resid), FP32, and
+//     the padded per-row vectors; tri_attn_bwd_bias_tiles_kernel: the pair bias
+//     copied into the main kernel's read order (one 32 KB block per tile).
 //  2. tri_attn_bwd_main_kernel (problem-stationary): one persistent CTA walks
 //     whole problems (b,i,h): key tiles kt outer, query tiles jt inner.  Per
 //     tile it recomputes S and dP with tcgen05, forms P and dS once, stages
 //     them in SMEM (BF16, 128B-swizzled) and issues dV += P^T dO,
-//     dK += dS^T Q, dQ_tile = dS K.  dK/dV finish in TMEM per key tile; dQ
+//     dK += dS^T Q, dQ_tile = dS K (S/dP and the gradient products from two
+//     warps).  dK/dV finish in TMEM per key tile; dQ stays in TMEM for every
+//     query tile when the columns allow (N <= 768 at d=32), else it
 //     accumulates over key tiles in a per-CTA FP32 slot of the workspace, in
 //     ascending kt order, by the same thread each time.
 //  3. tri_attn_bwd_dbias_kernel (tile-stationary): one CTA per (b,h,jt,kt)
