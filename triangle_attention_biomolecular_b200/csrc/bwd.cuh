@@ -706,10 +706,6 @@ __global__ void __launch_bounds__(640, 1)
                     const float* vec = reinterpret_cast<const float*>(smem + L::OFF_VEC + ts * 1024);
                     const float nlse2 = vec[row];  // -lse * log2(e)
                     const float nDj = vec[128 + row];  // -D
-                    // P and dS of this warpgroup's 32 keys, packed BF16 pairs, computed in two
-                    // 16-key halves while the previous tile's gradient MMAs still read the
-                    // shared-memory tiles
-                    uint32_t pw[16], dw[16];
                     const float2 sc2 = make_float2(scale, scale), l2e = make_float2(LOG2E, LOG2E);
                     const float2 nl2 = make_float2(nlse2, nlse2), nD2 = make_float2(nDj, nDj);
                     // all 32 keys of S and dP first, so the S/dP columns are released to the MMA
@@ -724,6 +720,15 @@ __global__ void __launch_bounds__(640, 1)
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(BAR(L::B_SDPFREE));
+                    // the gradient MMAs of two tiles ago have finished reading this tile's P/dS
+                    // buffer (the other one may still be read); each 8-key chunk of P and dS is
+                    // stored as soon as it is formed, so the stores drain during the arithmetic
+                    const int pb = g & 1;
+                    if (g >= 2 && !mbar_wait_warp(BAR(L::B_PDSFREE + pb), ((g >> 1) - 1) & 1, wc, 15)) { ok = false; break; }
+                    TRI_TP(3)
+                    // this warpgroup's 32 keys = four 16-byte chunks of one 64-key SW128 half
+                    const uint32_t prow = sb + L::OFF_PDS + pb * L::PDS_BUF + (w >> 1) * (L::PT_TILE / 2) + row * 128;
+                    const uint32_t drow = prow + L::PT_TILE;
                     auto tile = [&](auto masked) {
                         constexpr bool kMasked = decltype(masked)::value;
 #pragma unroll
@@ -734,6 +739,7 @@ __global__ void __launch_bounds__(640, 1)
                                 mk[0] = m0.x; mk[1] = m0.y; mk[2] = m0.z; mk[3] = m0.w;
                                 mk[4] = m1.x; mk[5] = m1.y; mk[6] = m1.z; mk[7] = m1.w;
                             }
+                            uint32_t pw[4], dw[4];
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
                                 const int xl = cc * 8 + 2 * e;
@@ -745,27 +751,17 @@ __global__ void __launch_bounds__(640, 1)
                                 const float2 pp = (!kMasked && e == 3) ? ex2_fma2(y) : make_float2(ex2(y.x), ex2(y.y));
                                 const float2 ds = fmul2(pp, fadd2(make_float2(__uint_as_float(dv[xl]),
                                                                               __uint_as_float(dv[xl + 1])), nD2));
-                                pw[cc * 4 + e] = pack_bf16(pp.x, pp.y);
-                                dw[cc * 4 + e] = pack_bf16(ds.x, ds.y);
+                                pw[e] = pack_bf16(pp.x, pp.y);
+                                dw[e] = pack_bf16(ds.x, ds.y);
                             }
+                            const uint32_t off = ((((w & 1) * 4) + cc) ^ (row & 7)) << 4;
+                            sts128(prow + off, make_uint4(pw[0], pw[1], pw[2], pw[3]));
+                            sts128(drow + off, make_uint4(dw[0], dw[1], dw[2], dw[3]));
                         }
                     };
                     if (has_mask) tile(std::true_type{});
                     else tile(std::false_type{});
                     TRI_TP(4)
-                    // the gradient MMAs of two tiles ago have finished reading this P/dS buffer
-                    const int pb = g & 1;  // P/dS buffer of this tile (the other one may still be read)
-                    if (g >= 2 && !mbar_wait_warp(BAR(L::B_PDSFREE + pb), ((g >> 1) - 1) & 1, wc, 15)) { ok = false; break; }
-                    TRI_TP(3)
-                    // this warpgroup's 32 keys = four 16-byte chunks of one 64-key SW128 half
-                    const uint32_t prow = sb + L::OFF_PDS + pb * L::PDS_BUF + (w >> 1) * (L::PT_TILE / 2) + row * 128;
-                    const uint32_t drow = prow + L::PT_TILE;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint32_t off = ((((w & 1) * 4) + c) ^ (row & 7)) << 4;
-                        sts128(prow + off, make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]));
-                        sts128(drow + off, make_uint4(dw[4 * c], dw[4 * c + 1], dw[4 * c + 2], dw[4 * c + 3]));
-                    }
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
