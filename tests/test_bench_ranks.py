@@ -60,3 +60,12 @@ def test_gate_cpu_baseline_times_the_oracle():
     line = bench.gate_cpu_baseline(target_s=0.2)
     assert line["kind"] == "oracle" and line["unit"] == "GB/s"
     assert line["value"] > 0 and line["cores"] >= 1 and line["seconds"] > 0
+
+
+@pytest.mark.parametrize("B,N,H", [(1, 768, 4), (1, 384, 4), (2, 256, 4), (2, 128, 4), (1, 64, 2), (2, 1024, 4)])
+def test_launch_count_follows_the_library_chunk_rule(B, N, H):
+    """The bench's per-step kernel count includes the dBias reduce exactly when the
+    library's workspace holds row-chunk partials (its size beyond the rows-only part)."""
+    from triangle_attention_biomolecular_b200 import _binding as Bd
+    has_partials = Bd.tri_attn_bwd_workspace_bytes(B, N, H, 32) > Bd.tri_attn_bwd_rows_workspace_bytes(B, N, N, H, 32)
+    assert bench.attn_launches_per_step(B, N, H) == 5 + int(has_partials)
