@@ -654,14 +654,18 @@ __global__ void __launch_bounds__(640, 1)
                     __nv_bfloat16* dst = (is_dk
                         ? p.dk + t.b * p.dks[0] + t.i * p.dks[1] + k * p.dks[2] + t.h * p.dks[3]
                         : p.dv + t.b * p.dvs[0] + t.i * p.dvs[1] + k * p.dvs[2] + t.h * p.dvs[3]) + c_off;
+                    uint32_t o[D / 4];  // the D/2 values as BF16 pairs
 #pragma unroll
-                    for (int e = 0; e < D / 2; e += 8) {
-                        uint4 v;
-                        v.x = pack_bf16(__uint_as_float(g16[e]) * f, __uint_as_float(g16[e + 1]) * f);
-                        v.y = pack_bf16(__uint_as_float(g16[e + 2]) * f, __uint_as_float(g16[e + 3]) * f);
-                        v.z = pack_bf16(__uint_as_float(g16[e + 4]) * f, __uint_as_float(g16[e + 5]) * f);
-                        v.w = pack_bf16(__uint_as_float(g16[e + 6]) * f, __uint_as_float(g16[e + 7]) * f);
-                        *reinterpret_cast<uint4*>(dst + e) = v;
+                    for (int e = 0; e < D / 2; e += 2)
+                        o[e / 2] = pack_bf16(__uint_as_float(g16[e]) * f, __uint_as_float(g16[e + 1]) * f);
+                    if ((reinterpret_cast<uintptr_t>(dst) & 31u) == 0) {
+                        // 32-byte stores: half the store instructions, each still one row
+#pragma unroll
+                        for (int e = 0; e < D / 4; e += 8) st_global_v8(dst + 2 * e, o + e);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < D / 4; e += 4)
+                            *reinterpret_cast<uint4*>(dst + 2 * e) = make_uint4(o[e], o[e + 1], o[e + 2], o[e + 3]);
                     }
                 }
             }
