@@ -124,21 +124,60 @@ __global__ void __launch_bounds__(256) tri_attn_bwd_prep_kernel(
     float* __restrict__ Dv, float* __restrict__ Lv, float* __restrict__ Mv, int* __restrict__ Fv, int B, int N,
     int R, int H, int Np, int nt) {
     constexpr float LOG2E = 1.4426950408889634f;
+    const int lane = threadIdx.x & 31;
     const int64_t n1 = static_cast<int64_t>(B) * H * R * Np;
     const int64_t n2 = static_cast<int64_t>(B) * R * Np;
     const int64_t n3 = static_cast<int64_t>(B) * R * 32;
-    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < n1 + n2 + n3;
+    // F first, one warp per (b, i, key tile): the warp reads the tile's 128 mask values in
+    // one round (four per lane, coalesced along k) and votes, so no thread walks a tile
+    // alone while the rest of the grid streams.
+    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t e = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); e < n3;
+         e += nwarps) {
+        const int kt = static_cast<int>(e & 31);
+        const int64_t t = e >> 5;
+        const int i = static_cast<int>(t % R);
+        const int b = static_cast<int>(t / R);
+        int f = 0;
+        if (kt < nt) {
+            if ((kt + 1) * 128 > N) {
+                f = 1;  // padded keys need the -inf
+            } else if (mask) {
+                const float* mr = mask + b * m0 + i * m1 + static_cast<int64_t>(kt * 128 + lane) * m2;
+                const float a0 = __ldg(mr), a1 = __ldg(mr + 32 * m2), a2 = __ldg(mr + 64 * m2),
+                            a3 = __ldg(mr + 96 * m2);
+                f = __any_sync(0xffffffffu, a0 != 0.f || a1 != 0.f || a2 != 0.f || a3 != 0.f) ? 1 : 0;
+            }
+        }
+        if (lane == 0) Fv[e] = f;
+    }
+    // D, L (head fastest) and then M; the index decode runs in 32-bit arithmetic whenever
+    // the item count allows (three 64-bit divisions per item cost more issue slots than
+    // the item's loads)
+    const bool small = n1 + n2 <= static_cast<int64_t>(0xffffffffu);
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < n1 + n2;
          idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         if (idx < n1) {
             // head fastest: neighbouring threads read the heads of one pair row, which are
             // contiguous in memory, so a warp streams whole 256-byte rows
-            int64_t t = idx;
-            const int h = static_cast<int>(t % H);
-            t /= H;
-            const int j = static_cast<int>(t % Np);
-            t /= Np;
-            const int i = static_cast<int>(t % R);
-            const int b = static_cast<int>(t / R);
+            int h, j, i, b;
+            if (small) {
+                uint32_t t = static_cast<uint32_t>(idx);
+                h = static_cast<int>(t % static_cast<uint32_t>(H));
+                t /= static_cast<uint32_t>(H);
+                j = static_cast<int>(t % static_cast<uint32_t>(Np));
+                t /= static_cast<uint32_t>(Np);
+                i = static_cast<int>(t % static_cast<uint32_t>(R));
+                b = static_cast<int>(t / static_cast<uint32_t>(R));
+            } else {
+                int64_t t = idx;
+                h = static_cast<int>(t % H);
+                t /= H;
+                j = static_cast<int>(t % Np);
+                t /= Np;
+                i = static_cast<int>(t % R);
+                b = static_cast<int>(t / R);
+            }
             const int64_t out = ((static_cast<int64_t>(b) * H + h) * R + i) * Np + j;
             float dsum = 0.f, lv = -INFINITY;
             if (j < N) {
@@ -162,29 +201,24 @@ __global__ void __launch_bounds__(256) tri_attn_bwd_prep_kernel(
             }
             Dv[out] = -dsum;
             Lv[out] = lv;
-        } else if (idx < n1 + n2) {
+        } else {
             const int64_t e = idx - n1;
-            const int k = static_cast<int>(e % Np);
-            const int64_t t = e / Np;
-            const int i = static_cast<int>(t % R);
-            const int b = static_cast<int>(t / R);
+            int k, i, b;
+            if (small) {
+                uint32_t t = static_cast<uint32_t>(e);
+                k = static_cast<int>(t % static_cast<uint32_t>(Np));
+                t /= static_cast<uint32_t>(Np);
+                i = static_cast<int>(t % static_cast<uint32_t>(R));
+                b = static_cast<int>(t / static_cast<uint32_t>(R));
+            } else {
+                k = static_cast<int>(e % Np);
+                const int64_t t = e / Np;
+                i = static_cast<int>(t % R);
+                b = static_cast<int>(t / R);
+            }
             float mv = -INFINITY;
             if (k < N) mv = mask ? __ldg(mask + b * m0 + i * m1 + k * m2) * LOG2E : 0.f;
             Mv[e] = mv;
-        } else {
-            const int64_t e = idx - n1 - n2;
-            const int kt = static_cast<int>(e % 32);
-            const int64_t t = e / 32;
-            const int i = static_cast<int>(t % R);
-            const int b = static_cast<int>(t / R);
-            int f = 0;
-            if (kt < nt) {
-                if ((kt + 1) * 128 > N) f = 1;  // padded keys need the -inf
-                if (mask && !f)
-                    for (int k = kt * 128; k < (kt + 1) * 128; ++k)
-                        if (__ldg(mask + b * m0 + i * m1 + k * m2) != 0.f) { f = 1; break; }
-            }
-            Fv[e] = f;
         }
     }
 }

@@ -543,19 +543,30 @@ __global__ void __launch_bounds__(384, 1)
                 tmem_wait_ld();
                 reg_fence32(o);
                 if (store) {
+                    // 32 columns -> 16 packed words each of o and resid; one 32-byte store per
+                    // 16 columns where the row start allows it (a warp's rows are H*d*2 bytes
+                    // apart, so 16-byte stores would fill half a sector each)
+                    const bool v8 = ((reinterpret_cast<uintptr_t>(op + c0) | reinterpret_cast<uintptr_t>(rp + c0)) & 31u) == 0;
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t ow[4], rw[4];
+                    for (int c = 0; c < 4; c += 2) {
+                        uint32_t ow[8], rw[8];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
+                        for (int e = 0; e < 8; ++e) {
                             const float a0 = __uint_as_float(o[8 * c + 2 * e]) * inv_l;
                             const float a1 = __uint_as_float(o[8 * c + 2 * e + 1]) * inv_l;
                             const uint32_t w16 = pack_bf16(a0, a1);
                             ow[e] = w16;
                             rw[e] = pack_bf16(a0 - bf16lo(w16), a1 - bf16hi(w16));
                         }
-                        *reinterpret_cast<uint4*>(op + c0 + 8 * c) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-                        *reinterpret_cast<uint4*>(rp + c0 + 8 * c) = make_uint4(rw[0], rw[1], rw[2], rw[3]);
+                        if (v8) {
+                            st_global_v8(op + c0 + 8 * c, ow);
+                            st_global_v8(rp + c0 + 8 * c, rw);
+                        } else {
+                            *reinterpret_cast<uint4*>(op + c0 + 8 * c) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                            *reinterpret_cast<uint4*>(op + c0 + 8 * c + 8) = make_uint4(ow[4], ow[5], ow[6], ow[7]);
+                            *reinterpret_cast<uint4*>(rp + c0 + 8 * c) = make_uint4(rw[0], rw[1], rw[2], rw[3]);
+                            *reinterpret_cast<uint4*>(rp + c0 + 8 * c + 8) = make_uint4(rw[4], rw[5], rw[6], rw[7]);
+                        }
                     }
                 }
             }
