@@ -69,3 +69,8 @@ def test_launch_count_follows_the_library_chunk_rule(B, N, H):
     from triangle_attention_biomolecular_b200 import _binding as Bd
     has_partials = Bd.tri_attn_bwd_workspace_bytes(B, N, H, 32) > Bd.tri_attn_bwd_rows_workspace_bytes(B, N, N, H, 32)
     assert bench.attn_launches_per_step(B, N, H) == 5 + int(has_partials)
+
+
+def test_l2_note_follows_the_input_size():
+    assert bench.l2_note(604_000_000).startswith("inputs (604 MB) larger than the 126 MB L2")
+    assert "fit in the 126 MB L2" in bench.l2_note(50_000_000)
