@@ -74,3 +74,38 @@ def test_launch_count_follows_the_library_chunk_rule(B, N, H):
 def test_l2_note_follows_the_input_size():
     assert bench.l2_note(604_000_000).startswith("inputs (604 MB) larger than the 126 MB L2")
     assert "fit in the 126 MB L2" in bench.l2_note(50_000_000)
+
+
+def test_json_line_carries_every_contract_key(monkeypatch, capsys):
+    """The line's assembly from a measured step (the GPU part replaced by fixed
+    numbers): every key of the output contract is present, the whole-job value
+    follows from the step time, and the roofline fraction is achieved / peak."""
+    import json
+    import sys
+    ms_step = 2.6
+    fake = {"ms": 20 * ms_step,
+            "kern_ms": {"fwd": 0.78, "bwd_prep": 0.10, "bwd_main": 1.14, "bwd_dbias": 0.61},
+            "clocks": {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 5},
+            "e2e": {"value": 55.0, "unit": "TFLOP/s", "h2d_bytes_per_step": 1, "d2h_bytes_per_step": 1},
+            "shape": (1, 768, 4, 32), "step_stats": {"median": ms_step}, "lengths": [768],
+            "memory": {"peak_allocated_bytes": 1}, "mask": "zeros", "bias_std": 2.0}
+    monkeypatch.setattr(bench, "run_ours", lambda *a: fake)
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--steps", "20", "--warmup", "5", "--no-cpu-baseline"])
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    bench.main()
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+        assert key in line, key
+    assert line["n_gpus"] == 1 and line["steps"] == 20 and line["warmup"] == 5
+    assert line["higher_is_better"] is True and line["scaling"] == "weak" and line["vs_baseline"] is None
+    assert abs(line["ms_per_step"] - ms_step) < 1e-9
+    flops = 14.0 * 4 * 768 ** 3 * 32
+    assert abs(line["value"] - flops / (ms_step * 1e-3) / 1e12) < 1e-2
+    r = line["roofline"]
+    for key in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        assert key in r, key
+    assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-3
+    assert line["config"]["workload"].startswith("crop768")
+    assert line["gpu_launches"] == 5 * 20
