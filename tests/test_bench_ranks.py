@@ -109,3 +109,18 @@ def test_json_line_carries_every_contract_key(monkeypatch, capsys):
     assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-3
     assert line["config"]["workload"].startswith("crop768")
     assert line["gpu_launches"] == 5 * 20
+
+
+def test_reference_arm_line_on_rank_zero(capsys):
+    """The reference arm (the FP64 oracle on host cores) prints one line with the
+    same metric and unit as ours, marked as the reference, with its CPU baseline
+    and an end-to-end entry that moves no device bytes."""
+    import json
+    args = argparse.Namespace(steps=1, warmup=0, gpus=1, workload="crop768", op="attention")
+    bench.run_reference(args, rank=0, world=1)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == "TFLOP/s"
+    assert line["higher_is_better"] is True and line["dtype"] == "f64" and line["value"] > 0
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
