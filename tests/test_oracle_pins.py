@@ -9,6 +9,7 @@
   bias or mask change nothing; probability rows sum to one; masked keys get
   exactly zero probability and gradient; every dbias row sums to zero).
 * FP64 central finite differences of L = sum(dout * out) for dq, dk, dv, dbias.
+* Brute force: the definition as scalar Python loops on tiny sizes.
 * Planted mistakes: each deliberate error the C oracle can be switched into is
   caught by at least one of these pins.
 
@@ -279,3 +280,89 @@ def test_row_functions_equal_the_whole_stack(mk):
         for i in range(11):
             O.dbias_add_row(acc, q[b, i], k[b, i], v[b, i], bias[b], None if mask is None else mask[b, i], do[b, i])
         assert np.array_equal(acc, db[b])
+
+
+def _literal_loops(q, k, v, bias, mask, do, scale):
+    """The definition written out as plain Python loops over scalars (no array
+    arithmetic), for tiny sizes: forward out and lse, then dv, dp, D, ds, dq, dk
+    and dbias = sum over i of ds.  Shares nothing with the C oracle."""
+    import math
+    B, N, _, H, d = q.shape
+    q, k, v, bias, do = (x.tolist() for x in (q, k, v, bias, do))
+    mask = None if mask is None else mask.tolist()
+    out = [[[[[0.0] * d for _ in range(H)] for _ in range(N)] for _ in range(N)] for _ in range(B)]
+    lse = [[[[0.0] * N for _ in range(N)] for _ in range(H)] for _ in range(B)]
+    dq = [[[[[0.0] * d for _ in range(H)] for _ in range(N)] for _ in range(N)] for _ in range(B)]
+    dk = [[[[[0.0] * d for _ in range(H)] for _ in range(N)] for _ in range(N)] for _ in range(B)]
+    dv = [[[[[0.0] * d for _ in range(H)] for _ in range(N)] for _ in range(N)] for _ in range(B)]
+    db = [[[[0.0] * N for _ in range(N)] for _ in range(H)] for _ in range(B)]
+    for b in range(B):
+        for i in range(N):
+            for h in range(H):
+                p = [[0.0] * N for _ in range(N)]
+                for j in range(N):
+                    s = []
+                    for kk in range(N):
+                        dot = 0.0
+                        for c in range(d):
+                            dot += q[b][i][j][h][c] * k[b][i][kk][h][c]
+                        x = scale * dot + bias[b][h][j][kk]
+                        if mask is not None:
+                            x += mask[b][i][kk]
+                        s.append(x)
+                    m = max(s)
+                    z = 0.0
+                    for kk in range(N):
+                        z += math.exp(s[kk] - m)
+                    lse[b][h][i][j] = m + math.log(z)
+                    for kk in range(N):
+                        p[j][kk] = math.exp(s[kk] - m) / z
+                    for c in range(d):
+                        acc = 0.0
+                        for kk in range(N):
+                            acc += p[j][kk] * v[b][i][kk][h][c]
+                        out[b][i][j][h][c] = acc
+                for j in range(N):
+                    Dj = 0.0
+                    for c in range(d):
+                        Dj += do[b][i][j][h][c] * out[b][i][j][h][c]
+                    for kk in range(N):
+                        dp = 0.0
+                        for c in range(d):
+                            dp += do[b][i][j][h][c] * v[b][i][kk][h][c]
+                        ds = p[j][kk] * (dp - Dj)
+                        db[b][h][j][kk] += ds
+                        for c in range(d):
+                            dv[b][i][kk][h][c] += p[j][kk] * do[b][i][j][h][c]
+                            dq[b][i][j][h][c] += scale * ds * k[b][i][kk][h][c]
+                            dk[b][i][kk][h][c] += scale * ds * q[b][i][j][h][c]
+    return tuple(np.array(x) for x in (out, lse, dq, dk, dv, db))
+
+
+@pytest.mark.parametrize("N,mk", [(2, "none"), (3, "random"), (5, "ragged"), (8, "random")])
+def test_oracle_equals_literal_loops_on_tiny_sizes(N, mk):
+    """Brute force: the definition as scalar Python loops agrees with the C oracle
+    to 1e-12 on tiny pair stacks (H=2, d=4), forward and all four gradients."""
+    q, k, v, do, bias, mask = _rand(40 + N, 2 if N < 8 else 1, N, 2, 4, mk)
+    scale = 1.0 / np.sqrt(4)
+    out_l, lse_l, dq_l, dk_l, dv_l, db_l = _literal_loops(q.numpy(), k.numpy(), v.numpy(), bias.numpy(),
+                                                         None if mask is None else mask.numpy(), do.numpy(), scale)
+    out, lse = O.fwd(q, k, v, bias, mask, scale)
+    dq, dk, dv, db = O.bwd(q, k, v, bias, mask, do, scale)
+    for got, ref in ((out, out_l), (lse, lse_l), (dq, dq_l), (dk, dk_l), (dv, dv_l), (db, db_l)):
+        assert _rel(got, ref) < 1e-12
+
+
+@pytest.mark.parametrize("planted", [1, 2, 3, 4, 5, 6, 7])
+def test_literal_loops_catch_planted_mistakes(planted):
+    """The brute-force pin on its own also catches every planted mistake."""
+    N = 5
+    q, k, v, do, bias, mask = _rand(45, 1, N, 2, 3, "random")
+    scale = 1.0 / np.sqrt(3)
+    ref = _literal_loops(q.numpy(), k.numpy(), v.numpy(), bias.numpy(), mask.numpy(), do.numpy(), scale)
+    try:
+        out, lse = O.fwd(q, k, v, bias, mask, scale, planted=planted)
+        got = (out, lse) + tuple(O.bwd(q, k, v, bias, mask, do, scale, planted=planted))
+    except O.OracleError:
+        return
+    assert max(_rel(g, r) for g, r in zip(got, ref)) > 1e-12
